@@ -1,0 +1,98 @@
+"""Seeded synthetic inputs shared by the tests, the smoke check and the bench.
+
+This module only draws random numbers; it holds none of the attention
+arithmetic, so the CUDA path and the CPU oracle can both be fed from it
+without sharing any of the method's code.
+
+Recipe (the pages fix only "i.i.d. N(0,1) bf16, seed s"):
+  * fixed length: ``g = torch.Generator('cpu').manual_seed(seed)``, then
+    ``torch.randn([B, N, H, d], dtype=float32, generator=g).to(bfloat16)``
+    for Q, K, V and (backward only) dO, drawn in that order;
+  * packed variable length: sequence lengths are
+    ``torch.randint(lo, hi + 1, (nseq,), generator=g)`` from the same seeded
+    generator, then Q, K, V (and dO) with shape ``[T, H, d]``,
+    ``T = sum(lengths)``; ``cu_seqlens`` is the int32 prefix sum with a
+    leading 0.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import torch
+
+
+def fixed_inputs(B: int, N: int, H: int, d: int, seed: int, with_dout: bool = False):
+    g = torch.Generator("cpu").manual_seed(seed)
+    names = ["q", "k", "v"] + (["dout"] if with_dout else [])
+    return {n: torch.randn([B, N, H, d], dtype=torch.float32, generator=g).to(torch.bfloat16)
+            for n in names}
+
+
+def varlen_lengths(nseq: int, lo: int, hi: int, g: torch.Generator):
+    return torch.randint(lo, hi + 1, (nseq,), generator=g, dtype=torch.int64)
+
+
+def varlen_inputs(nseq: int, lo: int, hi: int, H: int, d: int, seed: int,
+                  with_dout: bool = False, lengths=None):
+    """Packed inputs.  ``lengths`` overrides the random lengths (the random
+    stream is then used for the tensors only)."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    if lengths is None:
+        lens = varlen_lengths(nseq, lo, hi, g)
+    else:
+        lens = torch.as_tensor(lengths, dtype=torch.int64)
+    cu = torch.zeros(len(lens) + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(lens, 0).to(torch.int32)
+    T = int(cu[-1])
+    names = ["q", "k", "v"] + (["dout"] if with_dout else [])
+    out = {n: torch.randn([T, H, d], dtype=torch.float32, generator=g).to(torch.bfloat16)
+           for n in names}
+    out["cu_seqlens"] = cu
+    out["max_seqlen"] = int(lens.max()) if len(lens) else 0
+    return out
+
+
+@dataclass(frozen=True)
+class Workload:
+    """One named workload: shapes, seed and mask of a parity or bench case."""
+    name: str
+    B: int
+    H: int
+    N: int
+    d: int
+    seed: int
+    causal: bool = False
+    window: int = 0
+    varlen: tuple = field(default=None)   # (nseq, lo, hi) for packed inputs
+    backward: bool = False
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    def make(self):
+        if self.varlen is not None:
+            nseq, lo, hi = self.varlen
+            return varlen_inputs(nseq, lo, hi, self.H, self.d, self.seed, with_dout=self.backward)
+        return fixed_inputs(self.B, self.N, self.H, self.d, self.seed, with_dout=self.backward)
+
+
+# The five workloads of the parity contract.  Shapes and seeds are the ones
+# the long-sequence training and long-prompt prefill scenarios are measured on.
+WORKLOADS = {
+    "tiny": Workload("tiny", B=1, H=1, N=128, d=64, seed=0),
+    "train": Workload("train", B=4, H=16, N=2048, d=128, seed=1),
+    "train_causal": Workload("train_causal", B=4, H=16, N=2048, d=128, seed=1, causal=True),
+    "prefill_b2_causal": Workload("prefill_b2_causal", B=2, H=16, N=8192, d=128, seed=2,
+                                  causal=True),
+    "prefill_b4_causal": Workload("prefill_b4_causal", B=4, H=16, N=8192, d=128, seed=2,
+                                  causal=True),
+    "prefill_b4": Workload("prefill_b4", B=4, H=16, N=8192, d=128, seed=2),
+    "varlen_causal": Workload("varlen_causal", B=16, H=32, N=4096, d=128, seed=3, causal=True,
+                              varlen=(16, 128, 4096)),
+    "varlen_window": Workload("varlen_window", B=16, H=32, N=4096, d=128, seed=3, causal=True,
+                              window=1024, varlen=(16, 128, 4096)),
+    "bwd_causal": Workload("bwd_causal", B=2, H=16, N=4096, d=128, seed=4, causal=True,
+                           backward=True),
+}

@@ -1,0 +1,190 @@
+"""Python face of the float64 CPU oracle (``attn_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, by ``__graft_entry__.smoke``
+and by the CPU-baseline leg of ``bench.py``.  The CUDA library never imports
+it, and it imports nothing from the CUDA package.
+
+The oracle computes, in float64 from exact upcasts of the (bf16) inputs, the
+definition of scaled-dot-product attention, ``O = softmax(scale * Q K^T) V``
+row by row over the keys the mask allows (FlashAttention encyclopedia page,
+section "attention and the memory bottleneck"), with the three-pass safe
+softmax of the blog article "From Online Softmax to FlashAttention", sections
+2.1-2.2, and the gradients that follow from that definition.  See the header
+of ``attn_oracle.c`` for the formulas.
+
+Layouts accepted here:
+  * fixed length: q, k, v, dout are ``[B, N, H, d]``; returned LSE and D are
+    ``[B, H, N]``;
+  * packed variable length: ``[T, H, d]`` plus ``cu_seqlens`` (B+1 int
+    offsets); returned LSE and D are ``[H, T]``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_LIB_DIR = os.path.join(_HERE, "_build")
+_LIB = os.path.join(_LIB_DIR, "libattn_oracle.so")
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``attn_oracle.c`` into ``oracle/_build/libattn_oracle.so``."""
+    os.makedirs(_LIB_DIR, exist_ok=True)
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O3", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        dp = ctypes.POINTER(ctypes.c_double)
+        ip = ctypes.POINTER(ctypes.c_int)
+        common = [dp, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ip, ip,
+                  ctypes.c_double, ctypes.c_int, ctypes.c_int]
+        lib.oracle_fwd.argtypes = common + [dp, dp]
+        lib.oracle_fwd_rows.argtypes = common + [ctypes.c_int, ip, dp, dp]
+        lib.oracle_fwd_online.argtypes = common + [ctypes.c_int, dp, dp]
+        lib.oracle_bwd.argtypes = ([dp, dp, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                    ctypes.c_int, ip, ip, ctypes.c_double, ctypes.c_int,
+                                    ctypes.c_int, ctypes.c_int, ip, dp, dp, dp, dp, dp, dp])
+        for f in (lib.oracle_fwd, lib.oracle_fwd_rows, lib.oracle_fwd_online, lib.oracle_bwd):
+            f.restype = ctypes.c_int
+        lib.oracle_num_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def _f64(x) -> np.ndarray:
+    """Exact upcast to a C-contiguous float64 array (bf16 -> f64 is exact)."""
+    if hasattr(x, "detach"):  # torch tensor
+        import torch
+        x = x.detach().to("cpu", torch.float64).numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _dp(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _ip(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int))
+
+
+class _Packed:
+    """Token-major [T, H, d] view of the inputs plus sequence starts/lengths."""
+
+    def __init__(self, q, cu_seqlens):
+        if cu_seqlens is None:
+            if q.ndim != 4:
+                raise ValueError("fixed-length inputs must be [B, N, H, d]")
+            self.B, self.N, self.H, self.d = q.shape
+            self.T = self.B * self.N
+            self.starts = np.arange(self.B, dtype=np.int32) * self.N
+            self.lens = np.full(self.B, self.N, dtype=np.int32)
+            self.fixed = True
+        else:
+            if q.ndim != 3:
+                raise ValueError("packed inputs must be [T, H, d]")
+            cu = np.asarray(cu_seqlens.cpu() if hasattr(cu_seqlens, "cpu") else cu_seqlens,
+                            dtype=np.int64)
+            self.T, self.H, self.d = q.shape
+            self.B = len(cu) - 1
+            self.starts = np.ascontiguousarray(cu[:-1], dtype=np.int32)
+            self.lens = np.ascontiguousarray(cu[1:] - cu[:-1], dtype=np.int32)
+            self.fixed = False
+
+    def tok(self, x) -> np.ndarray:
+        return _f64(x).reshape(self.T, self.H, self.d)
+
+    def out_shape(self):
+        return (self.B, self.N, self.H, self.d) if self.fixed else (self.T, self.H, self.d)
+
+    def rowstat(self, a_ht: np.ndarray) -> np.ndarray:
+        """[H, T] -> [B, H, N] for fixed length; unchanged for packed."""
+        if self.fixed:
+            return a_ht.reshape(self.H, self.B, self.N).transpose(1, 0, 2).copy()
+        return a_ht
+
+
+def _check(rc: int):
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments (code %d)" % rc)
+
+
+def fwd(q, k, v, scale, causal=False, window=0, cu_seqlens=None):
+    """Three-pass float64 forward.  Returns (O, LSE) as float64 arrays."""
+    pk = _Packed(q, cu_seqlens)
+    Q, K, V = pk.tok(q), pk.tok(k), pk.tok(v)
+    O = np.zeros_like(Q)
+    L = np.zeros((pk.H, pk.T), dtype=np.float64)
+    _check(_load().oracle_fwd(_dp(Q), _dp(K), _dp(V), pk.T, pk.H, pk.d, pk.B, _ip(pk.starts),
+                              _ip(pk.lens), float(scale), int(bool(causal)), int(window),
+                              _dp(O), _dp(L)))
+    return O.reshape(pk.out_shape()), pk.rowstat(L)
+
+
+def fwd_online(q, k, v, scale, block, causal=False, window=0, cu_seqlens=None):
+    """Blocked one-pass forward with the online update; (O, LSE)."""
+    pk = _Packed(q, cu_seqlens)
+    Q, K, V = pk.tok(q), pk.tok(k), pk.tok(v)
+    O = np.zeros_like(Q)
+    L = np.zeros((pk.H, pk.T), dtype=np.float64)
+    _check(_load().oracle_fwd_online(_dp(Q), _dp(K), _dp(V), pk.T, pk.H, pk.d, pk.B,
+                                     _ip(pk.starts), _ip(pk.lens), float(scale),
+                                     int(bool(causal)), int(window), int(block), _dp(O), _dp(L)))
+    return O.reshape(pk.out_shape()), pk.rowstat(L)
+
+
+def fwd_rows(q, k, v, rows, scale, causal=False, window=0, cu_seqlens=None):
+    """Forward for selected rows.  ``rows`` is an int array [R, 3] of
+    (sequence, head, row-within-sequence).  Returns (O_rows [R, d], LSE [R])."""
+    pk = _Packed(q, cu_seqlens)
+    Q, K, V = pk.tok(q), pk.tok(k), pk.tok(v)
+    R = np.ascontiguousarray(np.asarray(rows, dtype=np.int32).reshape(-1, 3))
+    O = np.zeros((len(R), pk.d), dtype=np.float64)
+    L = np.zeros(len(R), dtype=np.float64)
+    _check(_load().oracle_fwd_rows(_dp(Q), _dp(K), _dp(V), pk.T, pk.H, pk.d, pk.B,
+                                   _ip(pk.starts), _ip(pk.lens), float(scale),
+                                   int(bool(causal)), int(window), len(R), _ip(R), _dp(O), _dp(L)))
+    return O, L
+
+
+def bwd(q, k, v, dout, scale, causal=False, window=0, cu_seqlens=None, heads=None):
+    """Float64 backward.  ``heads``: optional list of (sequence, head) pairs;
+    entries of other heads are returned as NaN.  Returns a dict with the
+    oracle's own ``o``, ``lse``, ``D`` and ``dq``, ``dk``, ``dv``."""
+    pk = _Packed(q, cu_seqlens)
+    Q, K, V, dO = pk.tok(q), pk.tok(k), pk.tok(v), pk.tok(dout)
+    out = {name: np.full_like(Q, np.nan) for name in ("o", "dq", "dk", "dv")}
+    L = np.full((pk.H, pk.T), np.nan)
+    Dd = np.full((pk.H, pk.T), np.nan)
+    if heads is None:
+        npairs, P = 0, None
+    else:
+        P = np.ascontiguousarray(np.asarray(heads, dtype=np.int32).reshape(-1, 2))
+        npairs = len(P)
+    _check(_load().oracle_bwd(_dp(Q), _dp(K), _dp(V), _dp(dO), pk.T, pk.H, pk.d, pk.B,
+                              _ip(pk.starts), _ip(pk.lens), float(scale), int(bool(causal)),
+                              int(window), npairs, None if P is None else _ip(P),
+                              _dp(out["dq"]), _dp(out["dk"]), _dp(out["dv"]), _dp(out["o"]),
+                              _dp(L), _dp(Dd)))
+    res = {name: a.reshape(pk.out_shape()) for name, a in out.items()}
+    res["lse"] = pk.rowstat(L)
+    res["D"] = pk.rowstat(Dd)
+    return res
