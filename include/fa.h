@@ -1,0 +1,135 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact IO-aware attention library.
+ *
+ * Operation (FlashAttention encyclopedia page, section "attention and the
+ * memory bottleneck"): for every sequence and head,
+ *     O = softmax(scale * Q K^T) V,
+ * the softmax taken row by row over the keys the mask allows.  The forward
+ * pass is one fused, tiled kernel that streams K/V tiles past an on-chip Q
+ * tile and keeps the online-softmax state of each row on chip (same page,
+ * "tiled computation and online normalisation"); it writes only O and the
+ * per-row log-sum-exp, never the N x N score or probability matrix.  The
+ * backward pass recomputes score tiles from that log-sum-exp instead of
+ * storing probabilities (same page, "training and complexity": compact
+ * normalisation statistics plus recomputation).
+ *
+ * Data layout (all tensors are caller-owned device memory; the library never
+ * allocates, frees or keeps a reference past the call):
+ *   q, k, v, o, dO, dq, dk, dv : bf16, token-major [tokens, H, d], contiguous,
+ *       i.e. element (token t, head h, channel c) at ((t * H) + h) * d + c.
+ *       Fixed length: tokens = B * N, sequence b at rows b*N .. b*N+N-1
+ *       (the usual [B, N, H, d] tensor).  Packed variable length: tokens = T,
+ *       sequence b at rows cu_seqlens[b] .. cu_seqlens[b+1]-1.
+ *   lse : fp32 natural-log log-sum-exp of the scaled scores of each row,
+ *       LSE_i = ln sum_j exp(scale * q_i . k_j) over allowed keys.
+ *       Fixed length: [B, H, N].  Packed: [H, T].
+ *   cu_seqlens : device int32, B + 1 non-decreasing offsets, cu_seqlens[0] = 0,
+ *       cu_seqlens[B] <= T; NULL selects fixed length.
+ *
+ * Shape arguments: B sequences, H heads, d in {64, 128} channels per head.
+ *   N is the sequence length for fixed-length inputs; for packed inputs N is
+ *   the number of token rows T the buffers hold (the per-sequence lengths are
+ *   read from cu_seqlens on the device, so no host synchronisation is needed).
+ *   Packed batches hold at most 4096 sequences.
+ *
+ * Masks (row i, key j local to a sequence of n tokens; query and key sequences
+ * have the same length):
+ *   causal != 0 : key j allowed only if j <= i (top-left aligned).
+ *   window  > 0 : sliding window of exactly `window` keys ending at the
+ *                 query's own position: allowed only if i - window < j <= i.
+ *                 Requires causal != 0.  window >= n equals plain causal.
+ *   window <= 0 : no window.
+ *
+ * scale: must be finite and > 0 (1/sqrt(d) for standard attention).
+ *
+ * Errors: every entry point returns FA_OK (0) or a negative fa_status.
+ *   Argument errors are detected on the host before anything is launched.
+ *   FA_ERR_CUDA means a launch or runtime call failed (cudaGetLastError is
+ *   left set).  Kernels never trap: every wait inside them is bounded, and a
+ *   wait that runs out records FA_ERR_DEVICE_TIMEOUT in a device error word
+ *   that fa_get_device_error() reports.
+ *
+ * Asynchrony: fa_fwd and fa_bwd enqueue kernels on `stream` and return
+ *   without synchronising; outputs are valid once the stream reaches them.
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stddef.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_NULLPTR = -1,        /* a required pointer is NULL */
+    FA_ERR_UNSUPPORTED_D = -2,  /* d not in {64, 128} */
+    FA_ERR_BAD_SHAPE = -3,      /* negative sizes, too many packed sequences, size overflow */
+    FA_ERR_MISALIGNED = -4,     /* a tensor base pointer is not 16-byte aligned */
+    FA_ERR_BAD_MASK = -5,       /* window > 0 without causal */
+    FA_ERR_WORKSPACE = -6,      /* workspace NULL or smaller than fa_bwd_workspace_size */
+    FA_ERR_CUDA = -7,           /* CUDA runtime / launch failure */
+    FA_ERR_DEVICE_TIMEOUT = -8, /* a bounded device-side wait gave up */
+    FA_ERR_BAD_SCALE = -9       /* scale not finite or not > 0 */
+} fa_status;
+
+/*
+ * Forward pass.  Writes o (bf16, layout of q) and lse (fp32, see above).
+ * q, k, v are read only.  Rows of o/lse outside every sequence (packed
+ * buffers with cu_seqlens[B] < T) are left untouched.
+ */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+           int B, int H, int N, int d, float scale, int causal, int window,
+           const int* cu_seqlens, cudaStream_t stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs: one fp32 per (head, token row) for
+ * D_i = rowsum(dO_i * O_i).  For packed inputs pass varlen_total = T (and any
+ * B, N); for fixed length pass varlen_total = 0.
+ */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d, int varlen_total);
+
+/*
+ * Backward pass (gradients of O = softmax(scale Q K^T) V).  Inputs: q, k, v,
+ * the forward's o and lse, and dO (layout of o).  Outputs dq, dk, dv (bf16,
+ * layout of q).  `workspace` is caller-owned device memory of at least
+ * fa_bwd_workspace_size(...) bytes, 16-byte aligned; its contents on entry do
+ * not matter and on exit are unspecified.  Shape and mask arguments as fa_fwd.
+ *
+ * The gradients follow from the definition (the pages print no formulas):
+ *   P_ij = exp(scale s_ij - LSE_i),  D_i = dO_i . O_i,
+ *   dV_j = sum_i P_ij dO_i,  dS_ij = P_ij (dO_i . v_j - D_i),
+ *   dQ_i = scale sum_j dS_ij k_j,  dK_j = scale sum_i dS_ij q_i.
+ */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dO, void* dq, void* dk, void* dv,
+           int B, int H, int N, int d, float scale, int causal, int window,
+           const int* cu_seqlens, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Static, human-readable text for a status code. */
+const char* fa_status_string(int status);
+
+/*
+ * Synchronises `stream`, then returns FA_ERR_DEVICE_TIMEOUT if any kernel of
+ * this library on the current device recorded a bounded-wait timeout since the
+ * last call (and clears the record), FA_ERR_CUDA if the synchronisation
+ * failed, else FA_OK.
+ */
+int fa_get_device_error(cudaStream_t stream);
+
+/*
+ * Test hook for the failure path.  mode 0: normal operation.  mode 1: the
+ * next fa_fwd launches make their load warp skip the first V tile, so the
+ * consumer's bounded wait runs out after timeout_ns nanoseconds (0 keeps the
+ * default of 2 s) and the kernel returns with FA_ERR_DEVICE_TIMEOUT recorded.
+ * Host-side setting, not thread safe; returns the previous mode.
+ */
+int fa_debug_set_fault(int mode, unsigned long long timeout_ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

@@ -1,0 +1,14 @@
+"""B200 (sm_100a) exact IO-aware attention: a C-ABI CUDA library
+(include/fa.h, csrc/) and its thin Python binding.
+
+    from io_aware_exact_21_b200 import forward, backward
+    o, lse = forward(q, k, v, causal=True)
+    dq, dk, dv = backward(q, k, v, o, lse, do, causal=True)
+"""
+from .binding import (FaError, backward, fa_bwd, fa_bwd_workspace_size, fa_debug_set_fault,
+                      fa_fwd, fa_get_device_error, fa_status_string, forward, library_path,
+                      load_library)
+
+__all__ = ["FaError", "backward", "fa_bwd", "fa_bwd_workspace_size", "fa_debug_set_fault",
+           "fa_fwd", "fa_get_device_error", "fa_status_string", "forward", "library_path",
+           "load_library"]

@@ -1,0 +1,169 @@
+"""ctypes binding of the C ABI in include/fa.h.
+
+Argument marshalling only: every step of the attention path runs in the CUDA
+kernels of libfa_b200.so.  Tensors are torch CUDA tensors (torch provides the
+device memory and the stream); nothing here computes attention, and there is
+no fallback: if the library or a GPU is missing, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+from . import build as _build
+
+FA_OK = 0
+STATUS = {
+    0: "FA_OK", -1: "FA_ERR_NULLPTR", -2: "FA_ERR_UNSUPPORTED_D", -3: "FA_ERR_BAD_SHAPE",
+    -4: "FA_ERR_MISALIGNED", -5: "FA_ERR_BAD_MASK", -6: "FA_ERR_WORKSPACE", -7: "FA_ERR_CUDA",
+    -8: "FA_ERR_DEVICE_TIMEOUT", -9: "FA_ERR_BAD_SCALE",
+}
+
+# Exported entry points and their C signatures.
+_VP, _I, _F, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "fa_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _I, _VP, _VP]),
+    "fa_bwd_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "fa_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _I,
+                    _VP, _VP, _SZ, _VP]),
+    "fa_status_string": (ctypes.c_char_p, [_I]),
+    "fa_get_device_error": (_I, [_VP]),
+    "fa_debug_set_fault": (_I, [_I, ctypes.c_ulonglong]),
+}
+
+
+class FaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__("%s failed: %s (%s)" % (where, STATUS.get(code, code),
+                                                 status_string(code)))
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _build.LIB_PATH
+
+
+def load_library():
+    """Load libfa_b200.so (building it first when the sources are newer).
+    Raises if it cannot be built or loaded: there is no other code path."""
+    global _lib
+    if _lib is None:
+        path = _build.LIB_PATH
+        if not os.path.exists(path) or _build.needs_build():
+            _build.build()
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return load_library().fa_status_string(int(code)).decode()
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(code: int, where: str):
+    if code != FA_OK:
+        raise FaError(code, where)
+
+
+# --------------------------------------------------------------- raw ABI ---
+
+def fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, window, cu_seqlens, stream=None) -> int:
+    return load_library().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), int(B), int(H),
+                                 int(N), int(d), float(scale), int(causal), int(window),
+                                 _ptr(cu_seqlens), _stream(stream))
+
+
+def fa_bwd_workspace_size(B, H, N, d, varlen_total=0) -> int:
+    return int(load_library().fa_bwd_workspace_size(int(B), int(H), int(N), int(d),
+                                                    int(varlen_total)))
+
+
+def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, window, cu_seqlens,
+           workspace, workspace_bytes, stream=None) -> int:
+    return load_library().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+                                 _ptr(dq), _ptr(dk), _ptr(dv), int(B), int(H), int(N), int(d),
+                                 float(scale), int(causal), int(window), _ptr(cu_seqlens),
+                                 _ptr(workspace), int(workspace_bytes), _stream(stream))
+
+
+def fa_status_string(code: int) -> str:
+    return status_string(code)
+
+
+def fa_get_device_error(stream=None) -> int:
+    return load_library().fa_get_device_error(_stream(stream))
+
+
+def fa_debug_set_fault(mode: int, timeout_ns: int = 0) -> int:
+    return load_library().fa_debug_set_fault(int(mode), int(timeout_ns))
+
+
+# ------------------------------------------------------ tensor helpers ---
+
+def _shape(q, cu_seqlens):
+    if cu_seqlens is None:
+        B, N, H, d = q.shape
+        return B, H, N, d
+    T, H, d = q.shape
+    return cu_seqlens.numel() - 1, H, T, d
+
+
+def forward(q, k, v, causal=False, window=0, cu_seqlens=None, scale=None, out=None, lse=None,
+            stream=None):
+    """O, LSE for bf16 CUDA tensors [B, N, H, d] (or packed [T, H, d] with
+    int32 ``cu_seqlens``).  Outputs are allocated with torch when not given."""
+    import torch
+    B, H, N, d = _shape(q, cu_seqlens)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N) if cu_seqlens is None else (H, N), dtype=torch.float32,
+                          device=q.device)
+    _check(fa_fwd(q, k, v, out, lse, B, H, N, d, scale, causal, window, cu_seqlens, stream),
+           "fa_fwd")
+    return out, lse
+
+
+def backward(q, k, v, o, lse, dout, causal=False, window=0, cu_seqlens=None, scale=None,
+             grads=None, workspace=None, stream=None):
+    """dQ, dK, dV for the forward's (O, LSE) and the output gradient dO."""
+    import torch
+    B, H, N, d = _shape(q, cu_seqlens)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if grads is None:
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    dq, dk, dv = grads
+    ws_bytes = fa_bwd_workspace_size(B, H, N, d, N if cu_seqlens is not None else 0)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+    _check(fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, window,
+                  cu_seqlens, workspace, workspace.numel(), stream), "fa_bwd")
+    return dq, dk, dv

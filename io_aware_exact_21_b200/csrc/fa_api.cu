@@ -1,0 +1,253 @@
+// fa_api.cu -- the C ABI (include/fa.h): argument validation, TMA tensor-map
+// encoding, per-device set-up and kernel launches on the caller's stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/fa.h"
+#include "bwd_kernels.cuh"
+#include "fwd_kernel.cuh"
+
+namespace {
+
+__device__ int g_error_word;   // bounded-wait timeouts are recorded here
+
+constexpr int kMaxDevices = 64;
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;
+
+int g_fault_mode = 0;
+unsigned long long g_fault_timeout_ns = 0;
+
+struct DeviceState {
+    bool ready = false;
+    int num_sms = 0;
+    int* error_word = nullptr;
+};
+DeviceState g_dev[kMaxDevices];
+std::mutex g_mutex;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+template <typename K>
+cudaError_t allow_smem(K kernel, int bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+// Per-device one-time set-up: SM count, the device address of the error word,
+// the driver's tensor-map encoder and the kernels' shared-memory limits.
+int device_setup(DeviceState** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceState& st = g_dev[dev];
+    if (!st.ready) {
+        if (cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev) !=
+            cudaSuccess)
+            return FA_ERR_CUDA;
+        if (cudaGetSymbolAddress(reinterpret_cast<void**>(&st.error_word), g_error_word) !=
+            cudaSuccess)
+            return FA_ERR_CUDA;
+        if (!g_encode) {
+            void* fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+                    cudaSuccess ||
+                q != cudaDriverEntryPointSuccess || !fn)
+                return FA_ERR_CUDA;
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+        }
+        if (allow_smem(fa::fwd_kernel<64>, fa::FwdCfg<64>::SMEM_BYTES) != cudaSuccess ||
+            allow_smem(fa::fwd_kernel<128>, fa::FwdCfg<128>::SMEM_BYTES) != cudaSuccess ||
+            fa::bwd_set_smem_limits() != cudaSuccess)
+            return FA_ERR_CUDA;
+        st.ready = true;
+    }
+    *out = &st;
+    return FA_OK;
+}
+
+// Tensor map over a token-major [rows, H, d] bf16 tensor; boxes of
+// 64 channels x 1 head x box_rows tokens, 128-byte swizzle, zero fill outside.
+int make_map(CUtensorMap* map, const void* ptr, int64_t rows, int H, int d, int box_rows) {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                          static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                             static_cast<cuuint64_t>(H) * static_cast<cuuint64_t>(d) * 2};
+    cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+bool misaligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+struct Common {
+    fa::Geometry g;
+    int64_t rows;      // token rows of the [rows, H, d] buffers
+};
+
+int validate_common(int B, int H, int N, int d, float scale, int causal, int window,
+                    const int* cu_seqlens, Common* c) {
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED_D;
+    if (B < 0 || H <= 0 || N < 0) return FA_ERR_BAD_SHAPE;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_BAD_SCALE;
+    if (window > 0 && !causal) return FA_ERR_BAD_MASK;
+    if (cu_seqlens && B > fa::kMaxVarlenSeqs) return FA_ERR_BAD_SHAPE;
+    if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return FA_ERR_MISALIGNED;
+    const int64_t rows = cu_seqlens ? static_cast<int64_t>(N) : static_cast<int64_t>(B) * N;
+    if (rows > (int64_t{1} << 31) - 1) return FA_ERR_BAD_SHAPE;
+    if (rows * H * d > (int64_t{1} << 40)) return FA_ERR_BAD_SHAPE;
+    c->rows = rows;
+    c->g.B = B;
+    c->g.H = H;
+    c->g.N = cu_seqlens ? 0 : N;
+    c->g.T = static_cast<int>(rows);
+    c->g.cu_seqlens = cu_seqlens;
+    c->g.causal = causal ? 1 : 0;
+    c->g.window = window > 0 ? window : 0;
+    return FA_OK;
+}
+
+template <int D>
+int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+               const fa::FwdParams& p, int grid, cudaStream_t stream) {
+    fa::fwd_kernel<D><<<grid, fa::FwdCfg<D>::THREADS, fa::FwdCfg<D>::SMEM_BYTES, stream>>>(
+        mq, mk, mv, p);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+           int d, float scale, int causal, int window, const int* cu_seqlens,
+           cudaStream_t stream) {
+    if (!q || !k || !v || !o || !lse) return FA_ERR_NULLPTR;
+    Common c;
+    int rc = validate_common(B, H, N, d, scale, causal, window, cu_seqlens, &c);
+    if (rc != FA_OK) return rc;
+    if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(o) || misaligned(lse))
+        return FA_ERR_MISALIGNED;
+    if (B == 0 || c.rows == 0) return FA_OK;
+    DeviceState* st = nullptr;
+    if ((rc = device_setup(&st)) != FA_OK) return rc;
+
+    CUtensorMap mq, mk, mv;
+    if (make_map(&mq, q, c.rows, H, d, 128) || make_map(&mk, k, c.rows, H, d, 128) ||
+        make_map(&mv, v, c.rows, H, d, 128))
+        return FA_ERR_CUDA;
+
+    fa::FwdParams p;
+    p.g = c.g;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.error_word = st->error_word;
+    p.timeout_ns = g_fault_timeout_ns ? g_fault_timeout_ns : kDefaultTimeoutNs;
+    p.fault_skip_v = g_fault_mode == 1 ? 1 : 0;
+
+    int grid = st->num_sms;
+    if (!cu_seqlens) {
+        const int64_t items = static_cast<int64_t>(B) * H * ((N + 255) / 256);
+        if (items < grid) grid = static_cast<int>(items);
+    }
+    return d == 64 ? launch_fwd<64>(mq, mk, mv, p, grid, stream)
+                   : launch_fwd<128>(mq, mk, mv, p, grid, stream);
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d, int varlen_total) {
+    (void)d;
+    if (H <= 0) return 0;
+    const int64_t rows = varlen_total > 0 ? varlen_total
+                                          : (B > 0 && N > 0 ? static_cast<int64_t>(B) * N : 0);
+    return fa::bwd_workspace_bytes(rows, H);
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale,
+           int causal, int window, const int* cu_seqlens, void* workspace, size_t workspace_bytes,
+           cudaStream_t stream) {
+    if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return FA_ERR_NULLPTR;
+    Common c;
+    int rc = validate_common(B, H, N, d, scale, causal, window, cu_seqlens, &c);
+    if (rc != FA_OK) return rc;
+    if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(o) || misaligned(lse) ||
+        misaligned(dO) || misaligned(dq) || misaligned(dk) || misaligned(dv))
+        return FA_ERR_MISALIGNED;
+    if (B == 0 || c.rows == 0) return FA_OK;
+    const size_t need = fa::bwd_workspace_bytes(c.rows, H);
+    if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
+    if (misaligned(workspace)) return FA_ERR_MISALIGNED;
+    DeviceState* st = nullptr;
+    if ((rc = device_setup(&st)) != FA_OK) return rc;
+
+    fa::BwdArgs a;
+    a.g = c.g;
+    a.d = d;
+    a.q = q; a.k = k; a.v = v; a.o = o; a.dO = dO;
+    a.lse = lse;
+    a.dq = dq; a.dk = dk; a.dv = dv;
+    a.D = static_cast<float*>(workspace);
+    a.scale = scale;
+    a.num_sms = st->num_sms;
+    a.error_word = st->error_word;
+    a.timeout_ns = g_fault_timeout_ns ? g_fault_timeout_ns : kDefaultTimeoutNs;
+    CUtensorMap maps[5];
+    const void* srcs[5] = {q, k, v, dO, o};
+    for (int i = 0; i < 5; ++i)
+        if (make_map(&maps[i], srcs[i], c.rows, H, d, 128)) return FA_ERR_CUDA;
+    return fa::bwd_launch(a, maps, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+const char* fa_status_string(int status) {
+    switch (status) {
+        case FA_OK: return "ok";
+        case FA_ERR_NULLPTR: return "a required pointer is NULL";
+        case FA_ERR_UNSUPPORTED_D: return "head dimension must be 64 or 128";
+        case FA_ERR_BAD_SHAPE: return "invalid shape";
+        case FA_ERR_MISALIGNED: return "a tensor pointer is not 16-byte aligned";
+        case FA_ERR_BAD_MASK: return "a sliding window requires the causal mask";
+        case FA_ERR_WORKSPACE: return "workspace missing or too small";
+        case FA_ERR_CUDA: return "CUDA runtime or launch error";
+        case FA_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait timed out";
+        case FA_ERR_BAD_SCALE: return "scale must be finite and positive";
+        default: return "unknown status";
+    }
+}
+
+int fa_get_device_error(cudaStream_t stream) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return FA_ERR_CUDA;
+    DeviceState* st = nullptr;
+    int rc = device_setup(&st);
+    if (rc != FA_OK) return rc;
+    int word = 0;
+    if (cudaMemcpy(&word, st->error_word, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return FA_ERR_CUDA;
+    if (word != 0) {
+        const int zero = 0;
+        if (cudaMemcpy(st->error_word, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+            return FA_ERR_CUDA;
+        return FA_ERR_DEVICE_TIMEOUT;
+    }
+    return FA_OK;
+}
+
+int fa_debug_set_fault(int mode, unsigned long long timeout_ns) {
+    int prev = g_fault_mode;
+    g_fault_mode = mode;
+    g_fault_timeout_ns = timeout_ns;
+    return prev;
+}
+
+}  // extern "C"

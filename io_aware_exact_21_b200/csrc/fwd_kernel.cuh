@@ -1,0 +1,422 @@
+// fwd_kernel.cuh -- fused, tiled exact attention forward for sm_100a.
+//
+// What it computes: O = softmax(scale * Q K^T) V per (sequence, head), plus
+// the per-row log-sum-exp, without ever writing the score or probability
+// matrix to HBM (FlashAttention encyclopedia page, "attention and the memory
+// bottleneck" and "tiled computation and online normalisation"; the IO-aware
+// essay, "let a block do more work on chip", whose flow chart is: load a Q
+// block, stream K/V blocks, form local scores, update row statistics,
+// accumulate the output, write the final output once).
+//
+// Online update per key tile (encyclopedia page, update equations), here in
+// base 2 with s' = s * scale * log2(e):
+//     m' = max(m, max_j s'_j),  l' = 2^(m-m') l + sum_j 2^(s'_j - m'),
+//     u' = 2^(m-m') u + sum_j 2^(s'_j - m') v_j,   O = u / l,
+//     LSE = ln 2 * (m + log2 l).
+// The rescale is applied only when the running maximum grows by more than
+// kRescaleLog2 (a factor 256): the update is exact for any reference value
+// used consistently in l and u, the maximum only keeps 2^(s'-m) bounded
+// (same page: subtracting the maximum is for numerical stability).
+//
+// CTA = two query tiles of 128 rows (256 rows) of one (sequence, head); both
+// tiles share one stream of K/V tiles of 128 keys.  Roles (384 threads):
+//   warp 0        TMA producer: Q tiles, then K_j, V_j into a ring of smem slots
+//   warp 1        TMEM owner and MMA issuer (one elected thread):
+//                 S_t = Q_t K_j^T (both operands in smem), O_t += P_t V_j
+//                 (P_t read from TMEM, V_j from smem)
+//   warps 2-3     idle
+//   warps 4-7     softmax + correction + epilogue of tile 0 (one thread per row)
+//   warps 8-11    the same for tile 1
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [384,384+D).
+// P_t is written as packed bf16 over the first 64 columns of S_t.
+// The MMA thread issues S_t(j+1) right after O_t += P_t(j) V_j, so while one
+// softmax warpgroup works on its tile the tensor core runs the other's GEMMs.
+#pragma once
+
+#include "schedule.cuh"
+#include "sm100.cuh"
+
+namespace fa {
+
+constexpr float kRescaleLog2 = 8.0f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct FwdParams {
+    Geometry g;
+    __nv_bfloat16* o;
+    float* lse;
+    float scale_log2;       // scale * log2(e)
+    int* error_word;
+    uint64_t timeout_ns;
+    int fault_skip_v;       // test hook: producer skips the first V load
+};
+
+template <int D>
+struct FwdCfg {
+    static constexpr int BM = 128;              // rows per query tile
+    static constexpr int BN = 128;              // keys per key tile
+    static constexpr int ROWS = 2 * BM;         // rows per CTA work item
+    static constexpr int NSLOT = 4;             // K/V ring depth
+    static constexpr int BOX_BYTES = 128 * 128; // one TMA box: 128 rows x 64 bf16
+    static constexpr int TILE_BYTES = BM * D * 2;
+    static constexpr int NBOX = D / 64;
+    static constexpr int THREADS = 384;
+    static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 384;
+    // shared memory carve-up (offsets from a 1024-byte aligned base)
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_KV = OFF_Q + 2 * TILE_BYTES;
+    static constexpr int OFF_BAR = OFF_KV + NSLOT * TILE_BYTES;
+    static constexpr int NBAR = 2 + 2 * NSLOT + 6 + 1;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int OFF_SCRATCH = OFF_MISC + 16;
+    static constexpr int OFF_PREFIX = OFF_SCRATCH + THREADS * 4;
+    static constexpr int SMEM_BYTES = OFF_PREFIX + (kMaxVarlenSeqs + 1) * 4 + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
+fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+           const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+    using C = FwdCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint8_t* sQ = smem + C::OFF_Q;
+    uint8_t* sKV = smem + C::OFF_KV;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* q_full = bars + 0;
+    uint64_t* q_empty = bars + 1;
+    uint64_t* slot_full = bars + 2;
+    uint64_t* slot_empty = bars + 2 + C::NSLOT;
+    uint64_t* s_full = bars + 2 + 2 * C::NSLOT;     // [2]
+    uint64_t* p_full = s_full + 2;                  // [2]
+    uint64_t* o_final = p_full + 2;                 // [2]
+    uint64_t* drain = o_final + 2;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+    int* scratch = reinterpret_cast<int*>(smem + C::OFF_SCRATCH);
+    int* prefix = reinterpret_cast<int*>(smem + C::OFF_PREFIX);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = lane_id();
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
+        for (int s = 0; s < C::NSLOT; ++s) {
+            mbar_init(slot_full + s, 1);
+            mbar_init(slot_empty + s, 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(s_full + t, 1);
+            mbar_init(p_full + t, 4);     // one arrival per softmax warp
+            mbar_init(o_final + t, 1);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_map(&tm_q);
+        tma_prefetch_map(&tm_k);
+        tma_prefetch_map(&tm_v);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, 512);
+        tmem_relinquish();
+    }
+    Schedule sch;
+    sch.g = p.g;
+    sch.rows_per_item = C::ROWS;
+    sch.heavy_first = p.g.causal;
+    sch.prefix = prefix;
+    sch.total_items = build_schedule_prefix(p.g, C::ROWS, prefix, scratch);  // has __syncthreads
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const WaitCtl wc{abort_flag, p.error_word, p.timeout_ns};
+    const int H = p.g.H;
+
+    if (warp < 4) {
+        regs_dealloc<104>();
+        if (warp == 0 && lane == 0) {
+            // ------------------------------------------------ TMA producer --
+            uint32_t cnt = 0, item_it = 0;
+            uint32_t q_issued = 0;
+            bool ok = true;
+            bool skipped = false;
+            uint32_t skipped_at = 0xffffffffu;
+            for (int w = blockIdx.x; w < sch.total_items && ok; w += gridDim.x, ++item_it) {
+                int s, h, blk;
+                sch.item(w, s, h, blk);
+                const SeqSpan sp = sch.span(s);
+                const int r_lo = blk * C::ROWS;
+                const int r_hi = min(sp.len, r_lo + C::ROWS);
+                int jb, je;
+                key_tile_range(r_lo, r_hi, sp.len, p.g.causal, p.g.window, C::BN, jb, je);
+                if (!mbar_wait(q_empty, (item_it & 1) ^ 1, wc)) { ok = false; break; }
+                mbar_arrive_expect_tx(q_full, 2 * C::TILE_BYTES);
+                for (int t = 0; t < 2; ++t)
+                    for (int b = 0; b < C::NBOX; ++b)
+                        tma_load_3d(sQ + t * C::TILE_BYTES + b * C::BOX_BYTES, &tm_q, q_full,
+                                    b * 64, h, sp.start + r_lo + t * C::BM);
+                ++q_issued;
+                for (int j = jb; j < je && ok; ++j) {
+                    for (int kv = 0; kv < 2; ++kv) {
+                        const int slot = cnt % C::NSLOT;
+                        if (!mbar_wait(slot_empty + slot, ((cnt / C::NSLOT) & 1) ^ 1, wc)) {
+                            ok = false;
+                            break;
+                        }
+                        if (kv == 1 && p.fault_skip_v && !skipped) {
+                            skipped = true;   // test hook: this slot never fills
+                            skipped_at = cnt;
+                        } else {
+                            mbar_arrive_expect_tx(slot_full + slot, C::TILE_BYTES);
+                            const CUtensorMap* tm = kv == 0 ? &tm_k : &tm_v;
+                            for (int b = 0; b < C::NBOX; ++b)
+                                tma_load_3d(sKV + slot * C::TILE_BYTES + b * C::BOX_BYTES, tm,
+                                            slot_full + slot, b * 64, h, sp.start + j * C::BN);
+                        }
+                        ++cnt;
+                    }
+                }
+            }
+            if (!ok) {
+                // Let the copies already in flight land before the CTA exits.
+                WaitCtl dw{abort_flag, p.error_word, 200000000ull};
+                volatile int no_abort = 0;
+                dw.abort_flag = &no_abort;
+                // The latest phase of every slot is one of the last NSLOT loads.
+                for (uint32_t x = cnt > C::NSLOT ? cnt - C::NSLOT : 0; x < cnt; ++x)
+                    if (x != skipped_at) mbar_wait(slot_full + x % C::NSLOT, (x / C::NSLOT) & 1, dw);
+                if (q_issued) mbar_wait(q_full, (q_issued - 1) & 1, dw);
+            }
+        } else if (warp == 1 && lane == 0) {
+            // --------------------------------------------------- MMA issuer --
+            constexpr uint32_t IDESC_S = idesc_bf16(128, C::BN, false, false);
+            constexpr uint32_t IDESC_O = idesc_bf16(128, D, false, true);
+            const uint32_t q_addr = smem_u32(sQ);
+            const uint32_t kv_addr = smem_u32(sKV);
+            uint32_t cnt = 0, step = 0, item_it = 0;
+            bool ok = true;
+            auto issue_s = [&](int t, uint32_t kslot) {
+                const uint32_t d_tmem = tmem + (t ? C::COL_S1 : C::COL_S0);
+                const uint32_t a0 = q_addr + t * C::TILE_BYTES;
+                const uint32_t b0 = kv_addr + kslot * C::TILE_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
+                    umma_ss(d_tmem, sw128_desc(a0 + off, 16, 1024), sw128_desc(b0 + off, 16, 1024),
+                            IDESC_S, kk > 0);
+                }
+            };
+            auto issue_pv = [&](int t, uint32_t vslot, uint32_t accumulate) {
+                const uint32_t d_tmem = tmem + (t ? C::COL_O1 : C::COL_O0);
+                const uint32_t a_tmem = tmem + (t ? C::COL_S1 : C::COL_S0);
+                const uint32_t b0 = kv_addr + vslot * C::TILE_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < C::BN / 16; ++kk) {
+                    umma_ts(d_tmem, a_tmem + kk * 8, sw128_desc(b0 + kk * 2048, C::BOX_BYTES, 1024),
+                            IDESC_O, (accumulate | kk) != 0);
+                }
+            };
+            for (int w = blockIdx.x; w < sch.total_items && ok; w += gridDim.x, ++item_it) {
+                int s, h, blk;
+                sch.item(w, s, h, blk);
+                const SeqSpan sp = sch.span(s);
+                const int r_lo = blk * C::ROWS;
+                const int r_hi = min(sp.len, r_lo + C::ROWS);
+                int jb, je;
+                key_tile_range(r_lo, r_hi, sp.len, p.g.causal, p.g.window, C::BN, jb, je);
+                if (!mbar_wait(q_full, item_it & 1, wc)) { ok = false; break; }
+                // first key tile
+                uint32_t kslot = cnt % C::NSLOT;
+                if (!mbar_wait(slot_full + kslot, (cnt / C::NSLOT) & 1, wc)) { ok = false; break; }
+                tc_fence_after();
+                issue_s(0, kslot);
+                umma_commit(s_full + 0);
+                issue_s(1, kslot);
+                umma_commit(s_full + 1);
+                umma_commit(slot_empty + kslot);
+                ++cnt;
+                for (int j = jb; j < je; ++j, ++step) {
+                    const bool last = (j + 1 == je);
+                    const uint32_t vslot = cnt % C::NSLOT;
+                    const uint32_t kslot_n = (cnt + 1) % C::NSLOT;
+                    if (!mbar_wait(slot_full + vslot, (cnt / C::NSLOT) & 1, wc)) { ok = false; break; }
+                    if (!mbar_wait(p_full + 0, step & 1, wc)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_pv(0, vslot, j > jb);
+                    if (last) umma_commit(o_final + 0);
+                    if (!last) {
+                        if (!mbar_wait(slot_full + kslot_n, ((cnt + 1) / C::NSLOT) & 1, wc)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        issue_s(0, kslot_n);
+                        umma_commit(s_full + 0);
+                    }
+                    if (!mbar_wait(p_full + 1, step & 1, wc)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_pv(1, vslot, j > jb);
+                    if (last) umma_commit(o_final + 1);
+                    umma_commit(slot_empty + vslot);
+                    if (!last) {
+                        issue_s(1, kslot_n);
+                        umma_commit(s_full + 1);
+                        umma_commit(slot_empty + kslot_n);
+                        cnt += 2;
+                    } else {
+                        umma_commit(q_empty);
+                        cnt += 1;
+                    }
+                }
+            }
+            if (!ok) {
+                umma_commit(drain);
+                WaitCtl dw{abort_flag, p.error_word, 200000000ull};
+                volatile int no_abort = 0;
+                dw.abort_flag = &no_abort;
+                mbar_wait(drain, 0, dw);
+            }
+        }
+        __syncwarp();
+    } else {
+        // --------------------------------------------- softmax warpgroups --
+        regs_alloc<200>();
+        const int t = (warp >> 2) - 1;               // query tile 0 or 1
+        const int wq = warp & 3;                     // TMEM lane quarter
+        const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+        const uint32_t tS = tmem + lane_base + (t ? C::COL_S1 : C::COL_S0);
+        const uint32_t tO = tmem + lane_base + (t ? C::COL_O1 : C::COL_O0);
+        const int row_in_tile = wq * 32 + lane;
+        const float sl2 = p.scale_log2;
+        uint32_t step = 0, item_it = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; w < sch.total_items && ok; w += gridDim.x, ++item_it) {
+            int s, h, blk;
+            sch.item(w, s, h, blk);
+            const SeqSpan sp = sch.span(s);
+            const int n = sp.len;
+            const int r_lo = blk * C::ROWS;
+            const int r_hi = min(n, r_lo + C::ROWS);
+            int jb, je;
+            key_tile_range(r_lo, r_hi, n, p.g.causal, p.g.window, C::BN, jb, je);
+            const int r0 = r_lo + t * C::BM;            // first row of this tile
+            const int i = r0 + row_in_tile;             // this thread's row
+            float m_ref = -INFINITY;
+            float l = 0.f;
+            for (int j = jb; j < je; ++j, ++step) {
+                if (!mbar_wait(s_full + t, step & 1, wc)) { ok = false; break; }
+                tc_fence_after();
+                float sv[C::BN];
+                {
+                    uint32_t r[32];
+#pragma unroll
+                    for (int c = 0; c < C::BN / 32; ++c) {
+                        tmem_ld32(tS + c * 32, r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(r[e]);
+                    }
+                }
+                const int k0 = j * C::BN;
+                if (tile_needs_mask(r0, C::BM, k0, C::BN, n, p.g.causal, p.g.window)) {
+#pragma unroll
+                    for (int c = 0; c < C::BN; ++c)
+                        if (!key_allowed(i, k0 + c, n, p.g.causal, p.g.window)) sv[c] = -INFINITY;
+                }
+                float mx = sv[0];
+#pragma unroll
+                for (int c = 1; c < C::BN; ++c) mx = fmaxf(mx, sv[c]);
+                const float m_new = fmaxf(m_ref, mx * sl2);
+                const bool resc = m_new > m_ref + kRescaleLog2;
+                float alpha = 1.f;
+                if (resc) {
+                    alpha = ex2(m_ref - m_new);
+                    l *= alpha;
+                    m_ref = m_new;
+                }
+                const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+                float lsum = 0.f;
+#pragma unroll
+                for (int c = 0; c < C::BN / 32; ++c) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float p0 = ex2(fmaf(sv[c * 32 + 2 * e], sl2, neg_m));
+                        const float p1 = ex2(fmaf(sv[c * 32 + 2 * e + 1], sl2, neg_m));
+                        lsum += p0 + p1;
+                        pk[e] = pack_bf16(p0, p1);
+                    }
+                    tmem_st16(tS + c * 16, pk);
+                }
+                l += lsum;
+                if (j > jb && __any_sync(0xffffffffu, resc)) {
+                    // O_t *= alpha.  The previous O_t += P V has completed because
+                    // S_t(j), which the MMA thread issued after it, has; the next
+                    // one waits for this warp's arrival on p_full.
+                    uint32_t r[32];
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        tmem_ld32(tO + c * 32, r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                        tmem_st32(tO + c * 32, r);
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(p_full + t);
+            }
+            if (!ok) break;
+            // ---------------------------------------------------- epilogue --
+            if (!mbar_wait(o_final + t, item_it & 1, wc)) { ok = false; break; }
+            tc_fence_after();
+            const bool valid = i < n;
+            const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            __nv_bfloat16* orow = p.o + (static_cast<size_t>(sp.start) + i) * H * D +
+                                  static_cast<size_t>(h) * D;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tO + c * 32, r);
+                tmem_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    pk[e] = pack_bf16(__uint_as_float(r[2 * e]) * inv_l,
+                                      __uint_as_float(r[2 * e + 1]) * inv_l);
+                if (valid) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                }
+            }
+            if (valid) {
+                const float lse = l > 0.f ? (m_ref + __log2f(l)) * kLn2 : -INFINITY;
+                const size_t idx = p.g.cu_seqlens
+                                       ? static_cast<size_t>(h) * p.g.T + sp.start + i
+                                       : (static_cast<size_t>(s) * H + h) * p.g.N + i;
+                p.lse[idx] = lse;
+            }
+            tc_fence_before();
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace fa

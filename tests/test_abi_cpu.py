@@ -1,0 +1,102 @@
+"""The C-ABI library builds, loads and exports every symbol its header
+declares; argument validation rejects bad calls on the host, with nothing
+launched (these calls never reach a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import io_aware_exact_21_b200 as fa
+from io_aware_exact_21_b200 import binding
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "fa.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = fa.load_library()
+    syms = declared_symbols()
+    assert "fa_fwd" in syms and "fa_bwd" in syms
+    for s in syms:
+        assert hasattr(lib, s), s
+    # the binding wraps every declared entry point under the same name
+    for s in syms:
+        assert s in binding.SIGNATURES, s
+        assert hasattr(fa, s), s
+
+
+def test_status_strings():
+    for code in binding.STATUS:
+        assert fa.fa_status_string(code)
+    assert fa.fa_status_string(12345) == "unknown status"
+
+
+# Fake, 16-byte aligned "device" addresses: validation fails before any use.
+P = 0x10000
+
+
+def fwd(**kw):
+    args = dict(q=P, k=P, v=P, o=P, lse=P, B=1, H=1, N=128, d=128, scale=0.1, causal=0,
+                window=0, cu_seqlens=None, stream=0)
+    args.update(kw)
+    return fa.fa_fwd(**args)
+
+
+def bwd(**kw):
+    args = dict(q=P, k=P, v=P, o=P, lse=P, dout=P, dq=P, dk=P, dv=P, B=1, H=1, N=128, d=128,
+                scale=0.1, causal=0, window=0, cu_seqlens=None, workspace=P,
+                workspace_bytes=1 << 20, stream=0)
+    args.update(kw)
+    return fa.fa_bwd(**args)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), -1), (dict(lse=None), -1),
+    (dict(d=96), -2), (dict(d=256), -2),
+    (dict(H=0), -3), (dict(B=-1), -3), (dict(N=-5), -3),
+    (dict(q=P + 8), -4), (dict(o=P + 2), -4),
+    (dict(window=16), -5),
+    (dict(scale=0.0), -9), (dict(scale=-1.0), -9), (dict(scale=float("inf")), -9),
+    (dict(cu_seqlens=P, B=5000, N=100), -3),
+    (dict(cu_seqlens=P + 2, B=2, N=100), -4),
+])
+def test_fwd_validation(kw, code):
+    assert fwd(**kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dout=None), -1), (dict(dv=None), -1),
+    (dict(d=32), -2),
+    (dict(dq=P + 4), -4),
+    (dict(window=3), -5),
+    (dict(workspace=None), -6), (dict(workspace_bytes=16), -6),
+    (dict(workspace=P + 8), -4),
+])
+def test_bwd_validation(kw, code):
+    assert bwd(**kw) == code
+
+
+def test_empty_problems_are_noops():
+    assert fwd(B=0) == 0
+    assert fwd(N=0) == 0
+    assert bwd(B=0, workspace=None, workspace_bytes=0) == 0
+
+
+def test_workspace_size():
+    # one fp32 D value per (head, token row), rounded up to 256 bytes
+    assert fa.fa_bwd_workspace_size(2, 16, 4096, 128, 0) == 2 * 16 * 4096 * 4
+    assert fa.fa_bwd_workspace_size(16, 32, 0, 128, 1000) == (32 * 1000 * 4 + 255) // 256 * 256
+    assert fa.fa_bwd_workspace_size(1, 1, 1, 64, 0) == 256
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
+def test_valid_call_without_gpu_reports_cuda_error():
+    assert fwd() == -7

@@ -1,0 +1,156 @@
+"""Forward parity on the GPU: fa_fwd (through the C ABI) against the float64
+oracle on the same seeded inputs, plus GPU-side invariants and guard bands."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import io_aware_exact_21_b200 as fa
+from io_aware_exact_21_b200.inputs import WORKLOADS, fixed_inputs, varlen_inputs
+from oracle import oracle as orc
+
+from helpers import (assert_close_bf16, assert_close_lse, gather_rows, sample_rows, to64)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def run_fwd(x, causal, window, cu=None):
+    q, k, v = (x[n].to(DEV) for n in ("q", "k", "v"))
+    cu_d = None if cu is None else cu.to(DEV)
+    o, lse = fa.forward(q, k, v, causal=causal, window=window, cu_seqlens=cu_d)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_error() == 0
+    return o, lse
+
+
+# --------------------------------------------- element-wise, small sizes ---
+
+SMALL = [(1, 1, 128, 64), (1, 2, 1, 128), (1, 2, 17, 128), (2, 2, 129, 64), (2, 3, 1000, 128),
+         (1, 2, 255, 128), (1, 1, 384, 128), (1, 2, 513, 64)]
+MASKS = [(False, 0), (True, 0), (True, 1), (True, 2), (True, 127), (True, 128), (True, 300)]
+
+
+@pytest.mark.parametrize("B,H,N,d", SMALL)
+@pytest.mark.parametrize("causal,window", MASKS)
+def test_fwd_small_elementwise(B, H, N, d, causal, window):
+    x = fixed_inputs(B, N, H, d, seed=100 + N)
+    o, lse = run_fwd(x, causal, window)
+    O, L = orc.fwd(x["q"], x["k"], x["v"], 1 / math.sqrt(d), causal=causal, window=window)
+    assert_close_bf16(o, O, "O")
+    assert_close_lse(lse, L)
+
+
+@pytest.mark.parametrize("lens", [[1, 127, 128, 129, 700], [300], [5, 1, 1000, 64, 257, 3]])
+@pytest.mark.parametrize("causal,window", [(False, 0), (True, 0), (True, 64), (True, 1)])
+def test_fwd_varlen_elementwise(lens, causal, window):
+    x = varlen_inputs(len(lens), 0, 0, 3, 128, seed=7, lengths=lens)
+    cu = x["cu_seqlens"]
+    o, lse = run_fwd(x, causal, window, cu)
+    O, L = orc.fwd(x["q"], x["k"], x["v"], 1 / math.sqrt(128), causal=causal, window=window,
+                   cu_seqlens=cu)
+    assert_close_bf16(o, O, "O")
+    assert_close_lse(lse, L)
+
+
+# --------------------------------------- full-size workloads, sampled rows ---
+
+@pytest.mark.parametrize("name", ["tiny", "train", "train_causal", "prefill_b2_causal",
+                                  "prefill_b4_causal", "prefill_b4", "varlen_causal",
+                                  "varlen_window"])
+def test_fwd_workload_parity(name):
+    wl = WORKLOADS[name]
+    x = wl.make()
+    cu = x.get("cu_seqlens")
+    o, lse = run_fwd(x, wl.causal, wl.window, cu)
+    if name == "tiny":
+        O, L = orc.fwd(x["q"], x["k"], x["v"], wl.scale, causal=wl.causal, window=wl.window)
+        assert_close_bf16(o, O, "O")
+        assert_close_lse(lse, L)
+        return
+    lens = (np.diff(cu.numpy()) if cu is not None else [wl.N] * wl.B)
+    rows = sample_rows(list(lens), wl.H, 160, seed=hash(name) % 1000)
+    Or, Lr = orc.fwd_rows(x["q"], x["k"], x["v"], rows, wl.scale, causal=wl.causal,
+                          window=wl.window, cu_seqlens=cu)
+    og, lg = gather_rows(o, lse, rows, None if cu is None else cu.numpy())
+    assert_close_bf16(og, Or, "O rows")
+    assert_close_lse(lg, Lr)
+    assert torch.isfinite(o).all()
+
+
+# ---------------------------------------------------------- invariants ---
+
+def test_zero_keys_give_column_mean_on_gpu():
+    B, N, H, d = 1, 300, 2, 128
+    x = fixed_inputs(B, N, H, d, seed=11)
+    x["k"] = torch.zeros_like(x["k"])
+    o, lse = run_fwd(x, False, 0)
+    mean = x["v"].double().mean(1, keepdim=True).expand(B, N, H, d).numpy()
+    assert np.abs(to64(o) - mean).max() <= 1e-2
+    assert np.abs(to64(lse) - math.log(N)).max() <= 1e-4
+
+
+def test_causal_row0_and_window1_on_gpu():
+    x = fixed_inputs(2, 257, 2, 128, seed=12)
+    o, _ = run_fwd(x, True, 0)
+    assert torch.equal(o[:, 0].cpu(), x["v"][:, 0])
+    o1, _ = run_fwd(x, True, 1)
+    assert torch.equal(o1.cpu(), x["v"])
+
+
+def test_determinism_and_mask_equivalences():
+    x = fixed_inputs(2, 700, 2, 128, seed=13)
+    o1, l1 = run_fwd(x, True, 0)
+    o2, l2 = run_fwd(x, True, 0)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    ow, lw = run_fwd(x, True, 700)          # window >= N equals causal
+    assert torch.equal(o1, ow) and torch.equal(l1, lw)
+    # uniform packed batch equals the fixed-length call bit for bit
+    B, N, H, d = 2, 700, 2, 128
+    xp = {n: x[n].reshape(B * N, H, d) for n in ("q", "k", "v")}
+    cu = torch.tensor([0, N, 2 * N], dtype=torch.int32)
+    op, lp = run_fwd(xp, True, 0, cu)
+    assert torch.equal(op.reshape(B, N, H, d), o1)
+    assert torch.equal(lp.reshape(H, B, N).permute(1, 0, 2), l1)
+
+
+def test_guard_bands_untouched():
+    """Outputs written only inside the tensors; rows past cu_seqlens[B] untouched."""
+    lens = [129, 300]
+    x = varlen_inputs(2, 0, 0, 2, 128, seed=14, lengths=lens)
+    T = sum(lens)
+    pad = 256
+    q, k, v = (torch.cat([x[n], torch.zeros(pad, 2, 128, dtype=torch.bfloat16)]).to(DEV)
+               for n in ("q", "k", "v"))
+    sentinel = -12345.0
+    guard = 4096
+    o_buf = torch.full(((T + pad) * 2 * 128 + 2 * guard,), sentinel, dtype=torch.bfloat16,
+                       device=DEV)
+    o = o_buf[guard:guard + (T + pad) * 2 * 128].view(T + pad, 2, 128)
+    lse_buf = torch.full((2 * (T + pad) + 2 * guard,), sentinel, dtype=torch.float32, device=DEV)
+    lse = lse_buf[guard:guard + 2 * (T + pad)].view(2, T + pad)
+    cu = x["cu_seqlens"].to(DEV)
+    rc = fa.fa_fwd(q, k, v, o, lse, 2, 2, T + pad, 128, 128 ** -0.5, 1, 0, cu, None)
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert (o_buf[:guard] == sentinel).all() and (o_buf[-guard:] == sentinel).all()
+    assert (lse_buf[:guard] == sentinel).all() and (lse_buf[-guard:] == sentinel).all()
+    assert (o[T:] == sentinel).all() and (lse[:, T:] == sentinel).all()
+    O, L = orc.fwd(x["q"], x["k"], x["v"], 128 ** -0.5, causal=True, cu_seqlens=x["cu_seqlens"])
+    assert_close_bf16(o[:T], O, "O")
+    assert_close_lse(lse[:, :T], L)
+
+
+def test_streams_and_noncontiguous_batch_offsets():
+    """A call on a side stream; outputs valid after that stream is synchronised."""
+    x = fixed_inputs(1, 512, 2, 64, seed=15)
+    s = torch.cuda.Stream()
+    q, k, v = (x[n].to(DEV) for n in ("q", "k", "v"))
+    with torch.cuda.stream(s):
+        o, lse = fa.forward(q, k, v, causal=True, stream=s)
+    s.synchronize()
+    O, L = orc.fwd(x["q"], x["k"], x["v"], 64 ** -0.5, causal=True)
+    assert_close_bf16(o, O, "O")
+    assert_close_lse(lse, L)
