@@ -195,19 +195,24 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
     fa::BwdArgs a;
     a.g = c.g;
     a.d = d;
-    a.q = q; a.k = k; a.v = v; a.o = o; a.dO = dO;
+    a.o = o;
+    a.dO = dO;
     a.lse = lse;
-    a.dq = dq; a.dk = dk; a.dv = dv;
-    a.D = static_cast<float*>(workspace);
+    a.dq = dq;
+    a.dk = dk;
+    a.dv = dv;
+    a.dsum = static_cast<float*>(workspace);
     a.scale = scale;
     a.num_sms = st->num_sms;
     a.error_word = st->error_word;
     a.timeout_ns = g_fault_timeout_ns ? g_fault_timeout_ns : kDefaultTimeoutNs;
-    CUtensorMap maps[5];
-    const void* srcs[5] = {q, k, v, dO, o};
-    for (int i = 0; i < 5; ++i)
-        if (make_map(&maps[i], srcs[i], c.rows, H, d, 128)) return FA_ERR_CUDA;
-    return fa::bwd_launch(a, maps, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+    fa::BwdMaps m;
+    if (make_map(&m.q64, q, c.rows, H, d, 64) || make_map(&m.do64, dO, c.rows, H, d, 64) ||
+        make_map(&m.k128, k, c.rows, H, d, 128) || make_map(&m.v128, v, c.rows, H, d, 128) ||
+        make_map(&m.q128, q, c.rows, H, d, 128) || make_map(&m.do128, dO, c.rows, H, d, 128) ||
+        make_map(&m.k64, k, c.rows, H, d, 64) || make_map(&m.v64, v, c.rows, H, d, 64))
+        return FA_ERR_CUDA;
+    return fa::bwd_launch(a, m, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 const char* fa_status_string(int status) {

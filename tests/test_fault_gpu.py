@@ -1,0 +1,34 @@
+"""Failure path without a GPU fault: the test hook makes the forward's load
+warp skip one V tile, so the consumer's bounded wait runs out; the kernel
+returns, the host reads FA_ERR_DEVICE_TIMEOUT, and the context stays usable."""
+import math
+
+import pytest
+import torch
+
+import io_aware_exact_21_b200 as fa
+from io_aware_exact_21_b200.inputs import fixed_inputs
+from oracle import oracle as orc
+
+from helpers import assert_close_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+def test_bounded_wait_timeout_is_reported_and_recoverable():
+    x = fixed_inputs(1, 512, 2, 128, seed=31)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    assert fa.fa_get_device_error() == 0
+    fa.fa_debug_set_fault(1, 50_000_000)        # skip one V load, 50 ms limit
+    try:
+        fa.forward(q, k, v, causal=False)
+        code = fa.fa_get_device_error()
+    finally:
+        fa.fa_debug_set_fault(0, 0)
+    assert code == -8
+    assert fa.fa_get_device_error() == 0        # the record was cleared
+    o, lse = fa.forward(q, k, v, causal=False)  # the context still works
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_error() == 0
+    O, _ = orc.fwd(x["q"], x["k"], x["v"], 1 / math.sqrt(128))
+    assert_close_bf16(o, O, "O")
