@@ -1,0 +1,380 @@
+"""Benchmark: one training step of exact attention (forward + backward) per
+GPU, through the C ABI, on synthetic inputs shaped like the long-sequence
+workload B=4, H=16, N=8192, d=128 (non-causal), bf16.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  The step is fa_fwd + fa_bwd (forward kernel,
+D pre-pass, dK/dV kernel, dQ kernel).  FLOPs per step are counted as the
+pages' dense attention work: forward 4*B*H*N^2*d, backward 2.5x forward
+(five GEMMs), halved under a causal mask.  Several GPUs run independent
+replicas (no collective: the (sequence, head) units share nothing).
+
+--impl reference times the float64 CPU oracle (the reference arm: there is
+no runnable reference implementation) on a bounded sample of the same
+workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "attention fwd/bwd TFLOPs/s (BF16, d=128) and % of B200 dense BF16 peak"
+UNIT = "TFLOP/s"
+WORKLOAD = dict(B=4, H=16, N=8192, d=128, causal=False, window=0, seed=2)
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+
+
+def flops(B, H, N, d, causal):
+    f = 4.0 * B * H * N * N * d
+    if causal:
+        f *= 0.5
+    return f, 2.5 * f
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_config(extra=None):
+    w = WORKLOAD
+    cfg = {"workload": "B%d H%d N%d d%d %s, forward+backward" % (
+        w["B"], w["H"], w["N"], w["d"], "causal" if w["causal"] else "non-causal"),
+        "B": w["B"], "H": w["H"], "N": w["N"], "d": w["d"], "causal": w["causal"],
+        "window": w["window"], "seed": w["seed"],
+        "l2": "inputs larger than L2 (Q, K, V, dO 128 MiB each); L2 not flushed"}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+# ------------------------------------------------------------ clocks ---
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons every 200 ms."""
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, device):
+        self.proc = None
+        self.lines = []
+        self.t = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            self.sel = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + ",".join(self.FIELDS), "--format=csv,noheader,nounits",
+                 "-lms", "200"] + self.sel, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.t:
+            self.t.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------- our arm ---
+
+def make_inputs(device, seed):
+    from io_aware_exact_21_b200.inputs import fixed_inputs
+    w = WORKLOAD
+    return fixed_inputs(w["B"], w["N"], w["H"], w["d"], seed=seed, with_dout=True)
+
+
+def run_ours(args, rank, world, device):
+    import io_aware_exact_21_b200 as fa
+    w = WORKLOAD
+    B, H, N, d, causal, window = w["B"], w["H"], w["N"], w["d"], w["causal"], w["window"]
+    scale = 1.0 / math.sqrt(d)
+    host = make_inputs(device, w["seed"] + rank)
+    q, k, v, do = (host[n].to(device) for n in ("q", "k", "v", "dout"))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d, 0), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        fa.forward(q, k, v, causal=causal, window=window, scale=scale, out=o, lse=lse, stream=stream)
+        fa.backward(q, k, v, o, lse, do, causal=causal, window=window, scale=scale,
+                    grads=(dq, dk, dv), workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    assert fa.fa_get_device_error() == 0
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    # ---- device-resident timed region
+    clocks = ClockSampler(device)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize(device)
+    fa.fa_profile_begin()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    elapsed = e0.elapsed_time(e1)
+    prof = fa.fa_profile_end()
+    clk = clocks.stop()
+    assert fa.fa_get_device_error() == 0
+
+    # ---- end to end: pinned host inputs in, results back to the host
+    pin = {n: host[n].pin_memory() for n in ("q", "k", "v", "dout")}
+    outs_host = [torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for _ in range(4)]
+    lse_host = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs_host) + lse_host.numel() * 4
+
+    def e2e_step():
+        q.copy_(pin["q"], non_blocking=True)
+        k.copy_(pin["k"], non_blocking=True)
+        v.copy_(pin["v"], non_blocking=True)
+        do.copy_(pin["dout"], non_blocking=True)
+        step()
+        for dst, src in zip(outs_host, (o, dq, dk, dv)):
+            dst.copy_(src, non_blocking=True)
+        lse_host.copy_(lse, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 10))
+    e2e_step()
+    torch.cuda.synchronize(device)
+    barrier()
+    torch.cuda.synchronize(device)
+    e2 = torch.cuda.Event(enable_timing=True)
+    e3 = torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e3.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    e2e_elapsed = e2.elapsed_time(e3)
+
+    times = torch.tensor([elapsed, e2e_elapsed], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
+    elapsed, e2e_elapsed = float(times[0]), float(times[1])
+    if rank != 0:
+        return None
+
+    f_fwd, f_bwd = flops(B, H, N, d, causal)
+    step_flops = f_fwd + f_bwd
+    ms_step = elapsed / args.steps
+    value = step_flops * world * args.steps / (elapsed * 1e-3) / 1e12
+    e2e_value = step_flops * world * e2e_steps / (e2e_elapsed * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    per_kernel = {}
+    for kind, (ms, cnt) in prof.items():
+        per_kernel[kind] = {"ms_per_launch": ms / cnt if cnt else None, "launches": cnt}
+    # dominant kernel by total device time
+    dom = max(prof, key=lambda kk: prof[kk][0])
+    dom_ms = per_kernel[dom]["ms_per_launch"]
+    # algorithmic FLOPs per launch: forward 4BHN^2d; dK/dV kernel = the dV and dK
+    # GEMMs plus the S and dP recomputation it needs (4 x 2BHN^2d, of which the
+    # counted backward work assigns it 2 + 2 ... reported below as executed).
+    kernel_flops = {"fwd": f_fwd, "dkdv": 2.0 * f_fwd, "dq": 1.5 * f_fwd, "dot": 0.0}
+    peak_key = "bf16_tflops_sustained" if peak_src == "measured" else "bf16_tflops"
+    peak = peaks.get(peak_key, FALLBACK_PEAKS["bf16_tflops"])
+    achieved = kernel_flops[dom] / (dom_ms * 1e-3) / 1e12 if dom_ms else None
+    t_fwd = per_kernel["fwd"]["ms_per_launch"]
+    t_bwd = sum(per_kernel[kk]["ms_per_launch"] or 0.0 for kk in ("dot", "dkdv", "dq"))
+    burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: i.i.d. N(0,1) bf16 Q, K, V, dO (seeded), no dataset",
+        "config": workload_config({"parallelism": "replicas" if world > 1 else "single GPU"}),
+        "fwd": {"ms": round(t_fwd, 4), "tflops": round(f_fwd / (t_fwd * 1e-3) / 1e12, 2),
+                "frac_of_measured_burst_peak": round(f_fwd / (t_fwd * 1e-3) / 1e12 / burst, 4)},
+        "bwd": {"ms": round(t_bwd, 4), "tflops": round(f_bwd / (t_bwd * 1e-3) / 1e12, 2),
+                "frac_of_measured_burst_peak": round(f_bwd / (t_bwd * 1e-3) / 1e12 / burst, 4),
+                "kernels_ms": {kk: round(per_kernel[kk]["ms_per_launch"] or 0.0, 4)
+                               for kk in ("dot", "dkdv", "dq")}},
+        "roofline": {"kernel": dom, "bound": "tensor",
+                     "achieved": round(achieved, 2) if achieved else None,
+                     "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4) if achieved else None,
+                     "peak_source": "%s %s" % (peak_src, peak_key),
+                     "traffic": None},
+        "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": sum(c for (_, c) in prof.values()),
+        "clocks": clk,
+    }
+    return out
+
+
+# ------------------------------------------------- CPU oracle (sample) ---
+
+def oracle_sample(n_tokens=None, seed=2):
+    """Time the float64 oracle on a bounded sample of the workload: one
+    (sequence, head) of the B4 H16 N8192 d128 problem -- its forward and
+    backward (the oracle's backward recomputes the forward) -- optionally
+    truncated to `n_tokens` tokens.  Returns (algorithmic TFLOP/s, sample
+    description, threads, seconds)."""
+    from oracle import oracle as orc
+    from io_aware_exact_21_b200.inputs import fixed_inputs
+    w = WORKLOAD
+    d = w["d"]
+    n = n_tokens or w["N"]
+    scale = 1.0 / math.sqrt(d)
+    x = fixed_inputs(1, n, 1, d, seed=seed, with_dout=True)
+    t0 = time.perf_counter()
+    orc.bwd(x["q"], x["k"], x["v"], x["dout"], scale, causal=w["causal"], window=w["window"])
+    secs = time.perf_counter() - t0
+    f_fwd, f_bwd = flops(1, 1, n, d, w["causal"])
+    desc = ("forward + backward of one (sequence, head) of the workload%s: %d tokens, d=%d, "
+            "%.1f s on %d threads" % ("" if n == w["N"] else " truncated", n, d, secs,
+                                      orc.num_threads()))
+    return (f_fwd + f_bwd) / secs / 1e12, desc, orc.num_threads(), secs
+
+
+def run_reference(args):
+    """Reference arm: the float64 CPU oracle as it stands, timed on the host
+    cores, one bounded sample of the workload per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    for _ in range(args.warmup):
+        oracle_sample(n_tokens=256)
+    vals = []
+    t0 = time.perf_counter()
+    desc = threads = None
+    for _ in range(args.steps):
+        val, desc, threads, _ = oracle_sample(n_tokens=2048)
+        vals.append(val)
+    elapsed = time.perf_counter() - t0
+    value = statistics.mean(vals)
+    cfg = workload_config({"parallelism": "host cores"})
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": elapsed * 1e3 / max(1, args.steps),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic: i.i.d. N(0,1) bf16 inputs upcast to float64", "config": cfg,
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the oracle timing (used for profiling runs)")
+    ap.add_argument("--shape", default=None,
+                    help="B,H,N,d override of the workload (profiling of smaller cases)")
+    ap.add_argument("--causal", action="store_true", help="causal mask (profiling)")
+    args = ap.parse_args()
+    if args.shape:
+        B, H, N, d = (int(x) for x in args.shape.split(","))
+        WORKLOAD.update(B=B, H=H, N=N, d=d)
+    if args.causal:
+        WORKLOAD.update(causal=True)
+    if args.warmup < 3:
+        args.warmup = 3
+
+    if args.impl == "reference":
+        out = run_reference(args)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (B200)")
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=device)
+    try:
+        out = run_ours(args, rank, world, device)
+        if out is not None:
+            if not args.no_cpu_baseline and world == 1:
+                val, desc, threads, secs = oracle_sample()
+                out["cpu_baseline"] = {"value": val, "unit": UNIT, "cores": threads,
+                                       "kind": "oracle", "sample": desc}
+            else:
+                out["cpu_baseline"] = None
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

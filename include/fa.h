@@ -120,6 +120,20 @@ const char* fa_status_string(int status);
 int fa_get_device_error(cudaStream_t stream);
 
 /*
+ * Per-kernel device timing.  fa_profile_begin() resets the counters and makes
+ * the following fa_fwd / fa_bwd calls on the calling thread's current device
+ * record a CUDA event pair on the launch stream around each kernel they launch
+ * (up to 1024 launches per kernel kind; later ones are not recorded).
+ * fa_profile_end() waits for the recorded events, stops recording, and writes
+ * for each kind k (0 forward, 1 D pre-pass, 2 dK/dV, 3 dQ) the summed device
+ * milliseconds ms[k] and the number of recorded launches counts[k].
+ * Either output pointer may be NULL.  The events are created once per device
+ * on the first fa_profile_begin() call.
+ */
+int fa_profile_begin(void);
+int fa_profile_end(double* ms, int* counts);
+
+/*
  * Test hook for the failure path.  mode 0: normal operation.  mode 1: the
  * next fa_fwd launches make their load warp skip the first V tile, so the
  * consumer's bounded wait runs out after timeout_ns nanoseconds (0 keeps the

@@ -30,7 +30,11 @@ SIGNATURES = {
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_get_device_error": (_I, [_VP]),
     "fa_debug_set_fault": (_I, [_I, ctypes.c_ulonglong]),
+    "fa_profile_begin": (_I, []),
+    "fa_profile_end": (_I, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]),
 }
+
+PROFILE_KINDS = ("fwd", "dot", "dkdv", "dq")
 
 
 class FaError(RuntimeError):
@@ -121,6 +125,19 @@ def fa_get_device_error(stream=None) -> int:
 
 def fa_debug_set_fault(mode: int, timeout_ns: int = 0) -> int:
     return load_library().fa_debug_set_fault(int(mode), int(timeout_ns))
+
+
+def fa_profile_begin() -> int:
+    return load_library().fa_profile_begin()
+
+
+def fa_profile_end():
+    """Returns {kind: (total_ms, launches)} for the launches recorded since
+    fa_profile_begin()."""
+    ms = (ctypes.c_double * 4)()
+    cnt = (ctypes.c_int * 4)()
+    _check(load_library().fa_profile_end(ms, cnt), "fa_profile_end")
+    return {k: (ms[i], cnt[i]) for i, k in enumerate(PROFILE_KINDS)}
 
 
 # ------------------------------------------------------ tensor helpers ---

@@ -773,10 +773,19 @@ inline cudaError_t bwd_set_smem_limits() {
                                 BwdCfg<128>::SMEM_BYTES);
 }
 
+// Optional timing callbacks around each launch (kind 1 = D pre-pass,
+// 2 = dK/dV, 3 = dQ): start returns a slot that stop closes.
+struct BwdHooks {
+    int (*start)(int kind, cudaStream_t stream);
+    void (*stop)(int kind, int slot, cudaStream_t stream);
+};
+
 template <int D>
-cudaError_t bwd_launch_d(const BwdArgs& a, const BwdMaps& m, cudaStream_t stream) {
+cudaError_t bwd_launch_d(const BwdArgs& a, const BwdMaps& m, cudaStream_t stream,
+                         const BwdHooks& hk) {
     using C = BwdCfg<D>;
     {
+        const int slot = hk.start(1, stream);
         const int64_t rows = static_cast<int64_t>(a.g.T) * a.g.H;
         const int rows_per_block = 8 * (32 / (D / 8));
         int64_t blocks = (rows + rows_per_block - 1) / rows_per_block;
@@ -786,6 +795,7 @@ cudaError_t bwd_launch_d(const BwdArgs& a, const BwdMaps& m, cudaStream_t stream
         dot_kernel<D><<<static_cast<int>(blocks), 256, 0, stream>>>(
             static_cast<const __nv_bfloat16*>(a.dO), static_cast<const __nv_bfloat16*>(a.o),
             a.dsum, a.g);
+        hk.stop(1, slot, stream);
     }
     BwdParams p;
     p.g = a.g;
@@ -802,15 +812,20 @@ cudaError_t bwd_launch_d(const BwdArgs& a, const BwdMaps& m, cudaStream_t stream
     }
     p.out0 = static_cast<__nv_bfloat16*>(a.dk);
     p.out1 = static_cast<__nv_bfloat16*>(a.dv);
+    int slot = hk.start(2, stream);
     dkdv_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(m.k128, m.v128, m.q64, m.do64, p);
+    hk.stop(2, slot, stream);
     p.out0 = static_cast<__nv_bfloat16*>(a.dq);
     p.out1 = nullptr;
+    slot = hk.start(3, stream);
     dq_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(m.q128, m.do128, m.k64, m.v64, p);
+    hk.stop(3, slot, stream);
     return cudaGetLastError();
 }
 
-inline cudaError_t bwd_launch(const BwdArgs& a, const BwdMaps& m, cudaStream_t stream) {
-    return a.d == 64 ? bwd_launch_d<64>(a, m, stream) : bwd_launch_d<128>(a, m, stream);
+inline cudaError_t bwd_launch(const BwdArgs& a, const BwdMaps& m, cudaStream_t stream,
+                              const BwdHooks& hk) {
+    return a.d == 64 ? bwd_launch_d<64>(a, m, stream, hk) : bwd_launch_d<128>(a, m, stream, hk);
 }
 
 }  // namespace fa

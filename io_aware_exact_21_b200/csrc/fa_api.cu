@@ -18,6 +18,31 @@ __device__ int g_error_word;   // bounded-wait timeouts are recorded here
 constexpr int kMaxDevices = 64;
 constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;
 
+// ----------------------------------------------------------- profiling --
+// Event pairs recorded around each launch while profiling is on.
+constexpr int kProfKinds = 4;          // forward, D pre-pass, dK/dV, dQ
+constexpr int kProfCap = 1024;
+struct Profiler {
+    bool created = false;
+    bool on = false;
+    int device = -1;
+    cudaEvent_t ev[kProfKinds][kProfCap][2];
+    int n[kProfKinds] = {0, 0, 0, 0};
+};
+thread_local Profiler g_prof;
+
+// Records the "before" event of a launch of `kind`; returns the slot or -1.
+int prof_start(int kind, cudaStream_t stream) {
+    Profiler& P = g_prof;
+    if (!P.on || P.n[kind] >= kProfCap) return -1;
+    const int slot = P.n[kind]++;
+    cudaEventRecord(P.ev[kind][slot][0], stream);
+    return slot;
+}
+void prof_stop(int kind, int slot, cudaStream_t stream) {
+    if (slot >= 0) cudaEventRecord(g_prof.ev[kind][slot][1], stream);
+}
+
 int g_fault_mode = 0;
 unsigned long long g_fault_timeout_ns = 0;
 
@@ -162,8 +187,11 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
         const int64_t items = static_cast<int64_t>(B) * H * ((N + 255) / 256);
         if (items < grid) grid = static_cast<int>(items);
     }
-    return d == 64 ? launch_fwd<64>(mq, mk, mv, p, grid, stream)
-                   : launch_fwd<128>(mq, mk, mv, p, grid, stream);
+    const int slot = prof_start(0, stream);
+    rc = d == 64 ? launch_fwd<64>(mq, mk, mv, p, grid, stream)
+                 : launch_fwd<128>(mq, mk, mv, p, grid, stream);
+    prof_stop(0, slot, stream);
+    return rc;
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d, int varlen_total) {
@@ -212,7 +240,8 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
         make_map(&m.q128, q, c.rows, H, d, 128) || make_map(&m.do128, dO, c.rows, H, d, 128) ||
         make_map(&m.k64, k, c.rows, H, d, 64) || make_map(&m.v64, v, c.rows, H, d, 64))
         return FA_ERR_CUDA;
-    return fa::bwd_launch(a, m, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+    fa::BwdHooks hooks{prof_start, prof_stop};
+    return fa::bwd_launch(a, m, stream, hooks) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 const char* fa_status_string(int status) {
@@ -244,6 +273,50 @@ int fa_get_device_error(cudaStream_t stream) {
         if (cudaMemcpy(st->error_word, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
             return FA_ERR_CUDA;
         return FA_ERR_DEVICE_TIMEOUT;
+    }
+    return FA_OK;
+}
+
+int fa_profile_begin(void) {
+    Profiler& P = g_prof;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+    if (P.created && P.device != dev) {
+        for (int k = 0; k < kProfKinds; ++k)
+            for (int i = 0; i < kProfCap; ++i) {
+                cudaEventDestroy(P.ev[k][i][0]);
+                cudaEventDestroy(P.ev[k][i][1]);
+            }
+        P.created = false;
+    }
+    if (!P.created) {
+        for (int k = 0; k < kProfKinds; ++k)
+            for (int i = 0; i < kProfCap; ++i)
+                if (cudaEventCreate(&P.ev[k][i][0]) != cudaSuccess ||
+                    cudaEventCreate(&P.ev[k][i][1]) != cudaSuccess)
+                    return FA_ERR_CUDA;
+        P.created = true;
+        P.device = dev;
+    }
+    for (int k = 0; k < kProfKinds; ++k) P.n[k] = 0;
+    P.on = true;
+    return FA_OK;
+}
+
+int fa_profile_end(double* ms, int* counts) {
+    Profiler& P = g_prof;
+    P.on = false;
+    for (int k = 0; k < kProfKinds; ++k) {
+        double total = 0.0;
+        for (int i = 0; i < P.n[k]; ++i) {
+            if (cudaEventSynchronize(P.ev[k][i][1]) != cudaSuccess) return FA_ERR_CUDA;
+            float t = 0.f;
+            if (cudaEventElapsedTime(&t, P.ev[k][i][0], P.ev[k][i][1]) != cudaSuccess)
+                return FA_ERR_CUDA;
+            total += t;
+        }
+        if (ms) ms[k] = total;
+        if (counts) counts[k] = P.n[k];
     }
     return FA_OK;
 }
