@@ -72,7 +72,8 @@ typedef enum {
     FA_ERR_WORKSPACE = -6,      /* workspace NULL or smaller than fa_bwd_workspace_size */
     FA_ERR_CUDA = -7,           /* CUDA runtime / launch failure */
     FA_ERR_DEVICE_TIMEOUT = -8, /* a bounded device-side wait gave up */
-    FA_ERR_BAD_SCALE = -9       /* scale not finite or not > 0 */
+    FA_ERR_BAD_SCALE = -9,      /* scale not finite or not > 0 */
+    FA_ERR_SCRATCH_LIMIT = -10  /* problem larger than fa_bwd_noalloc's built-in scratch */
 } fa_status;
 
 /*
@@ -107,6 +108,34 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
            const void* dO, void* dq, void* dk, void* dv,
            int B, int H, int N, int d, float scale, int causal, int window,
            const int* cu_seqlens, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * fa_bwd_noalloc: the backward pass for callers that cannot allocate device
+ * memory -- for example a plugin inside a framework or runtime that owns every
+ * device allocation and has no way to hand this library a workspace, or a
+ * serving loop that must not allocate once it is running.  It computes exactly
+ * what fa_bwd computes, with the same arguments minus the workspace: the
+ * D = rowsum(dO * O) values live in a fixed device array built into the
+ * library instead (FA_NOALLOC_MAX_ROWS fp32 values, 4 MiB, held on every GPU
+ * that loads the library until the process exits).  The pages have no
+ * counterpart of this entry point; it only changes where the scratch lives.
+ *
+ * - Problems needing more than FA_NOALLOC_MAX_ROWS values (H * token rows)
+ *   return FA_ERR_SCRATCH_LIMIT and launch nothing; use fa_bwd for them.
+ * - It calls no cudaMalloc / cudaFree and no allocating library routine.
+ * - The first call on a device looks up the array's device address (a
+ *   one-time set-up with that device current); make that first call before
+ *   any stream capture.
+ * - All calls share the one array per device and leave their D values in it;
+ *   every call rewrites the part it uses before reading it.  Calls whose
+ *   kernels overlap on the GPU (different streams, or different host threads)
+ *   race on the array: serialise them.
+ */
+#define FA_NOALLOC_MAX_ROWS (1 << 20)
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                   const void* dO, void* dq, void* dk, void* dv,
+                   int B, int H, int N, int d, float scale, int causal, int window,
+                   const int* cu_seqlens, cudaStream_t stream);
 
 /* Static, human-readable text for a status code. */
 const char* fa_status_string(int status);

@@ -17,8 +17,9 @@ FA_OK = 0
 STATUS = {
     0: "FA_OK", -1: "FA_ERR_NULLPTR", -2: "FA_ERR_UNSUPPORTED_D", -3: "FA_ERR_BAD_SHAPE",
     -4: "FA_ERR_MISALIGNED", -5: "FA_ERR_BAD_MASK", -6: "FA_ERR_WORKSPACE", -7: "FA_ERR_CUDA",
-    -8: "FA_ERR_DEVICE_TIMEOUT", -9: "FA_ERR_BAD_SCALE",
+    -8: "FA_ERR_DEVICE_TIMEOUT", -9: "FA_ERR_BAD_SCALE", -10: "FA_ERR_SCRATCH_LIMIT",
 }
+NOALLOC_MAX_ROWS = 1 << 20   # FA_NOALLOC_MAX_ROWS in include/fa.h
 
 # Exported entry points and their C signatures.
 _VP, _I, _F, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
@@ -27,6 +28,8 @@ SIGNATURES = {
     "fa_bwd_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "fa_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _I,
                     _VP, _VP, _SZ, _VP]),
+    "fa_bwd_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I,
+                            _I, _VP, _VP]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_get_device_error": (_I, [_VP]),
     "fa_debug_set_fault": (_I, [_I, ctypes.c_ulonglong]),
@@ -113,6 +116,16 @@ def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, window,
                                  _ptr(dq), _ptr(dk), _ptr(dv), int(B), int(H), int(N), int(d),
                                  float(scale), int(causal), int(window), _ptr(cu_seqlens),
                                  _ptr(workspace), int(workspace_bytes), _stream(stream))
+
+
+def fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, window,
+                   cu_seqlens, stream=None) -> int:
+    """fa_bwd without a workspace argument: for callers that cannot allocate
+    device memory (its scratch is a fixed array inside the library)."""
+    return load_library().fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                         _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), int(B), int(H),
+                                         int(N), int(d), float(scale), int(causal), int(window),
+                                         _ptr(cu_seqlens), _stream(stream))
 
 
 def fa_status_string(code: int) -> str:

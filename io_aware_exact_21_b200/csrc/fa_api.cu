@@ -151,6 +151,36 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+// ------------------------------------------------ allocation-free backward --
+// Built-in scratch for fa_bwd_noalloc: the D values of one backward call.  In
+// host code the symbol is only a host-side stand-in; kernels get the device
+// address looked up once per device below.
+static __device__ __align__(256) float g_noalloc_scratch[FA_NOALLOC_MAX_ROWS];
+
+struct NoAllocState {
+    bool ready = false;
+    float* scratch = nullptr;   // device address of g_noalloc_scratch on this device
+};
+NoAllocState g_noalloc[kMaxDevices];
+
+// One-time, per-device lookup of the scratch array's device address (with
+// that device current).
+int noalloc_setup(float** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    NoAllocState& st = g_noalloc[dev];
+    if (!st.ready) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr)
+            return FA_ERR_CUDA;
+        st.scratch = static_cast<float*>(ptr);
+        st.ready = true;
+    }
+    *out = st.scratch;
+    return FA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -244,6 +274,48 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
     return fa::bwd_launch(a, m, stream, hooks) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                   const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                   float scale, int causal, int window, const int* cu_seqlens,
+                   cudaStream_t stream) {
+    if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return FA_ERR_NULLPTR;
+    Common c;
+    int rc = validate_common(B, H, N, d, scale, causal, window, cu_seqlens, &c);
+    if (rc != FA_OK) return rc;
+    if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(o) || misaligned(lse) ||
+        misaligned(dO) || misaligned(dq) || misaligned(dk) || misaligned(dv))
+        return FA_ERR_MISALIGNED;
+    if (B == 0 || c.rows == 0) return FA_OK;
+    if (c.rows * H > static_cast<int64_t>(FA_NOALLOC_MAX_ROWS)) return FA_ERR_SCRATCH_LIMIT;
+    DeviceState* st = nullptr;
+    if ((rc = device_setup(&st)) != FA_OK) return rc;
+    float* scratch = nullptr;
+    if ((rc = noalloc_setup(&scratch)) != FA_OK) return rc;
+
+    fa::BwdArgs a;
+    a.g = c.g;
+    a.d = d;
+    a.o = o;
+    a.dO = dO;
+    a.lse = lse;
+    a.dq = dq;
+    a.dk = dk;
+    a.dv = dv;
+    a.dsum = scratch;     // every element the kernels read is written first by the D pre-pass
+    a.scale = scale;
+    a.num_sms = st->num_sms;
+    a.error_word = st->error_word;
+    a.timeout_ns = g_fault_timeout_ns ? g_fault_timeout_ns : kDefaultTimeoutNs;
+    fa::BwdMaps m;
+    if (make_map(&m.q64, q, c.rows, H, d, 64) || make_map(&m.do64, dO, c.rows, H, d, 64) ||
+        make_map(&m.k128, k, c.rows, H, d, 128) || make_map(&m.v128, v, c.rows, H, d, 128) ||
+        make_map(&m.q128, q, c.rows, H, d, 128) || make_map(&m.do128, dO, c.rows, H, d, 128) ||
+        make_map(&m.k64, k, c.rows, H, d, 64) || make_map(&m.v64, v, c.rows, H, d, 64))
+        return FA_ERR_CUDA;
+    fa::BwdHooks hooks{prof_start, prof_stop};
+    return fa::bwd_launch(a, m, stream, hooks) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 const char* fa_status_string(int status) {
     switch (status) {
         case FA_OK: return "ok";
@@ -256,6 +328,8 @@ const char* fa_status_string(int status) {
         case FA_ERR_CUDA: return "CUDA runtime or launch error";
         case FA_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait timed out";
         case FA_ERR_BAD_SCALE: return "scale must be finite and positive";
+        case FA_ERR_SCRATCH_LIMIT:
+            return "problem exceeds the built-in scratch of fa_bwd_noalloc (use fa_bwd)";
         default: return "unknown status";
     }
 }

@@ -100,3 +100,24 @@ def test_workspace_size():
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
 def test_valid_call_without_gpu_reports_cuda_error():
     assert fwd() == -7
+
+
+def test_noalloc_validation_on_host():
+    base = dict(q=P, k=P, v=P, o=P, lse=P, dout=P, dq=P, dk=P, dv=P, B=1, H=1, N=128, d=128,
+                scale=0.1, causal=0, window=0, cu_seqlens=None, stream=0)
+
+    def call(**kw):
+        a = dict(base)
+        a.update(kw)
+        return fa.fa_bwd_noalloc(**a)
+
+    assert call(dq=None) == -1
+    assert call(d=80) == -2
+    assert call(window=4) == -5
+    assert call(dv=P + 8) == -4
+    # H * rows above the built-in scratch (FA_NOALLOC_MAX_ROWS) is rejected
+    assert call(H=16, N=binding.NOALLOC_MAX_ROWS // 16 + 1) == -10
+    assert call(B=0) == 0
+    header = open(HEADER).read()
+    assert "#define FA_NOALLOC_MAX_ROWS (1 << 20)" in header
+    assert binding.NOALLOC_MAX_ROWS == 1 << 20
