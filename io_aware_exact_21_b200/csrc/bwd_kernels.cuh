@@ -23,9 +23,9 @@
 //   3. dq_kernel  : a CTA owns 128 queries and streams the key tiles (64 keys):
 //        S = Q K^T, dP = dO V^T, P, dS as above, dQ += dS K.
 // Both big kernels use the forward's role split (TMA warp, MMA warp, two
-// element-wise warpgroups taking alternate tiles) and double-buffer the score
-// tiles in TMEM, so the element-wise work of one tile overlaps the GEMMs of
-// the next.  Deterministic: no atomics.
+// element-wise warpgroups, each taking one 32-column half of every score
+// tile) and double-buffer the score tiles in TMEM, so the element-wise work
+// of one tile overlaps the GEMMs of the next.  Deterministic: no atomics.
 #pragma once
 
 #include "schedule.cuh"
@@ -171,7 +171,7 @@ __device__ __forceinline__ void init_barriers(const BwdBarriers& br, volatile in
     }
     for (int b = 0; b < 2; ++b) {
         mbar_init(br.s_full + b, 1);
-        mbar_init(br.ready + b, 4);     // the four warps of one element-wise warpgroup
+        mbar_init(br.ready + b, 8);     // all eight element-wise warps (both halves of a tile)
     }
     mbar_init(br.acc_final, 1);
     mbar_init(br.acc_empty, 8);         // all eight element-wise warps
@@ -196,6 +196,11 @@ __device__ __forceinline__ void issue_ss_pair(uint32_t d_tmem, uint32_t a_base, 
     }
 }
 
+// Column of the packed bf16 operand for 16-row k-step kk: each element-wise
+// warpgroup packs its 32-column half h of a score tile into the first 16 of
+// that half's columns (h * 32 ... h * 32 + 15), which it has already read.
+__host__ __device__ constexpr uint32_t packed_col(int kk) { return (kk >> 1) * 32 + (kk & 1) * 8; }
+
 // acc[128 x D] (+)= A[tmem, 128 x 64 bf16] * B[smem, 64 x D, MN-major].
 template <int D>
 __device__ __forceinline__ void issue_ts_acc(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base,
@@ -203,8 +208,8 @@ __device__ __forceinline__ void issue_ts_acc(uint32_t d_tmem, uint32_t a_tmem, u
     using C = BwdCfg<D>;
 #pragma unroll
     for (int kk = 0; kk < C::BS / 16; ++kk)
-        umma_ts(d_tmem, a_tmem + kk * 8, sw128_desc(b_base + kk * 2048, C::SBOX, 1024), idesc,
-                (accumulate || kk > 0) ? 1u : 0u);
+        umma_ts(d_tmem, a_tmem + packed_col(kk), sw128_desc(b_base + kk * 2048, C::SBOX, 1024),
+                idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
 // Bounded wait that ignores the abort flag (used to drain in-flight work).
@@ -425,8 +430,8 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             int ib, ie;
             query_tile_range(k0, min(n, k0 + C::BM), n, p.g.causal, p.g.window, C::BS, ib, ie);
             for (int i = ib; i < ie; ++i, ++cnt) {
-                if (static_cast<int>(cnt & 1) != g) continue;
-                if (!mbar_wait(br.s_full + g, (cnt >> 1) & 1, wc)) { ok = false; break; }
+                const int b = cnt & 1;
+                if (!mbar_wait(br.s_full + b, (cnt >> 1) & 1, wc)) { ok = false; break; }
                 // The producer wrote this stage's row statistics with ordinary stores
                 // before arriving on stage_full: wait on it too so they are visible.
                 if (!mbar_wait(br.stage_full + cnt % C::NSTAGE, (cnt / C::NSTAGE) & 1, wc)) {
@@ -434,42 +439,39 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                     break;
                 }
                 tc_fence_after();
-                const float* vs = vec + (cnt % C::NSTAGE) * 2 * C::BS;
-                const int q0 = i * C::BS;
+                // this warpgroup's half of the tile: queries q0 + 32g ... q0 + 32g + 31
+                const float* vs = vec + (cnt % C::NSTAGE) * 2 * C::BS + 32 * g;
+                const int q0 = i * C::BS + 32 * g;
                 const bool need_mask = (k0 + C::BM > n) || (p.g.causal && k0 + C::BM - 1 > q0) ||
-                                       (p.g.window > 0 && q0 + C::BS - 1 - k0 >= p.g.window);
-                const uint32_t tS = tmem + lane_base + C::col_s(g);
-                const uint32_t tP = tmem + lane_base + C::col_dp(g);
+                                       (p.g.window > 0 && q0 + 31 - k0 >= p.g.window);
+                const uint32_t tS = tmem + lane_base + C::col_s(b) + 32 * g;
+                const uint32_t tP = tmem + lane_base + C::col_dp(b) + 32 * g;
+                uint32_t sr[32], dr[32];
+                tmem_ld32(tS, sr);
+                tmem_ld32(tP, dr);
+                tmem_wait_ld();
+                uint32_t pp[16], dd[16];
 #pragma unroll
-                for (int c = 0; c < C::BS / 16; ++c) {
-                    uint32_t sr[16], dr[16];
-                    tmem_ld16(tS + c * 16, sr);
-                    tmem_ld16(tP + c * 16, dr);
-                    tmem_wait_ld();
-                    uint32_t pp[8], dd[8];
+                for (int e = 0; e < 32; e += 2) {
+                    float pv[2], dv[2];
 #pragma unroll
-                    for (int e = 0; e < 16; e += 2) {
-                        float pv[2], dv[2];
-#pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            const int col = c * 16 + e + u;
-                            float pr = ex2(fmaf(__uint_as_float(sr[e + u]), sl2, vs[col]));
-                            if (need_mask &&
-                                !key_allowed(q0 + col, j, n, p.g.causal, p.g.window))
-                                pr = 0.f;
-                            pv[u] = pr;
-                            dv[u] = pr * (__uint_as_float(dr[e + u]) - vs[C::BS + col]);
-                        }
-                        pp[e / 2] = pack_bf16(pv[0], pv[1]);
-                        dd[e / 2] = pack_bf16(dv[0], dv[1]);
+                    for (int u = 0; u < 2; ++u) {
+                        const int col = e + u;
+                        float pr = ex2(fmaf(__uint_as_float(sr[col]), sl2, vs[col]));
+                        if (need_mask && !key_allowed(q0 + col, j, n, p.g.causal, p.g.window))
+                            pr = 0.f;
+                        pv[u] = pr;
+                        dv[u] = pr * (__uint_as_float(dr[col]) - vs[C::BS + col]);
                     }
-                    tmem_st8(tS + c * 8, pp);     // P^T over the first 32 columns of S^T
-                    tmem_st8(tP + c * 8, dd);     // dS^T over the first 32 columns of dP^T
+                    pp[e / 2] = pack_bf16(pv[0], pv[1]);
+                    dd[e / 2] = pack_bf16(dv[0], dv[1]);
                 }
+                tmem_st16(tS, pp);     // P^T packed over the first 16 columns of this half
+                tmem_st16(tP, dd);     // dS^T likewise in the dP^T half
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(br.ready + g);
+                if (lane == 0) mbar_arrive(br.ready + b);
             }
             if (!ok) break;
             // ------------------------------------------------ epilogue --
@@ -676,39 +678,37 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
                 dq_d = p.dsum[idx];
             }
             for (int j = jb; j < je; ++j, ++cnt) {
-                if (static_cast<int>(cnt & 1) != g) continue;
-                if (!mbar_wait(br.s_full + g, (cnt >> 1) & 1, wc)) { ok = false; break; }
+                const int b = cnt & 1;
+                if (!mbar_wait(br.s_full + b, (cnt >> 1) & 1, wc)) { ok = false; break; }
                 tc_fence_after();
-                const int kb = j * C::BS;
-                const bool need_mask = tile_needs_mask(q0, C::BM, kb, C::BS, n, p.g.causal, p.g.window);
-                const uint32_t tS = tmem + lane_base + C::col_s(g);
-                const uint32_t tP = tmem + lane_base + C::col_dp(g);
+                // this warpgroup's half of the tile: keys kb ... kb + 31
+                const int kb = j * C::BS + 32 * g;
+                const bool need_mask = tile_needs_mask(q0, C::BM, kb, 32, n, p.g.causal, p.g.window);
+                const uint32_t tS = tmem + lane_base + C::col_s(b) + 32 * g;
+                const uint32_t tP = tmem + lane_base + C::col_dp(b) + 32 * g;
+                uint32_t sr[32], dr[32];
+                tmem_ld32(tS, sr);
+                tmem_ld32(tP, dr);
+                tmem_wait_ld();
+                uint32_t dd[16];
 #pragma unroll
-                for (int c = 0; c < C::BS / 16; ++c) {
-                    uint32_t sr[16], dr[16];
-                    tmem_ld16(tS + c * 16, sr);
-                    tmem_ld16(tP + c * 16, dr);
-                    tmem_wait_ld();
-                    uint32_t dd[8];
+                for (int e = 0; e < 32; e += 2) {
+                    float dv[2];
 #pragma unroll
-                    for (int e = 0; e < 16; e += 2) {
-                        float dv[2];
-#pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            const int col = c * 16 + e + u;
-                            float pr = ex2(fmaf(__uint_as_float(sr[e + u]), sl2, nl));
-                            if (need_mask && !key_allowed(q, kb + col, n, p.g.causal, p.g.window))
-                                pr = 0.f;
-                            dv[u] = pr * (__uint_as_float(dr[e + u]) - dq_d);
-                        }
-                        dd[e / 2] = pack_bf16(dv[0], dv[1]);
+                    for (int u = 0; u < 2; ++u) {
+                        const int col = e + u;
+                        float pr = ex2(fmaf(__uint_as_float(sr[col]), sl2, nl));
+                        if (need_mask && !key_allowed(q, kb + col, n, p.g.causal, p.g.window))
+                            pr = 0.f;
+                        dv[u] = pr * (__uint_as_float(dr[col]) - dq_d);
                     }
-                    tmem_st8(tP + c * 8, dd);     // dS over the first 32 columns of dP
+                    dd[e / 2] = pack_bf16(dv[0], dv[1]);
                 }
+                tmem_st16(tP, dd);     // dS packed over the first 16 columns of this half
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(br.ready + g);
+                if (lane == 0) mbar_arrive(br.ready + b);
             }
             if (!ok) break;
             // ------------------------------------------------ epilogue --
