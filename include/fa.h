@@ -86,9 +86,12 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
            const int* cu_seqlens, cudaStream_t stream);
 
 /*
- * Bytes of device workspace fa_bwd needs: one fp32 per (head, token row) for
- * D_i = rowsum(dO_i * O_i).  For packed inputs pass varlen_total = T (and any
- * B, N); for fixed length pass varlen_total = 0.
+ * Bytes of device workspace fa_bwd needs: 8 bytes per (head, row) for the
+ * per-row statistics {-LSE_i * log2(e), D_i = rowsum(dO_i * O_i)}, stored with
+ * every sequence padded to a multiple of 128 rows.  Fixed length:
+ * B * H * roundup(N, 128) * 8.  Packed: pass varlen_total = T and the number of
+ * sequences B (N is ignored): H * roundup(T + 127 * B, 128) * 8.  Rounded up
+ * to 256 bytes.  Returns 0 for H <= 0 or B <= 0.
  */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d, int varlen_total);
 
@@ -115,13 +118,14 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
  * device allocation and has no way to hand this library a workspace, or a
  * serving loop that must not allocate once it is running.  It computes exactly
  * what fa_bwd computes, with the same arguments minus the workspace: the
- * D = rowsum(dO * O) values live in a fixed device array built into the
- * library instead (FA_NOALLOC_MAX_ROWS fp32 values, 4 MiB, held on every GPU
+ * per-row statistics live in a fixed device array built into the library
+ * instead (FA_NOALLOC_MAX_ROWS entries of 8 bytes, 8 MiB, held on every GPU
  * that loads the library until the process exits).  The pages have no
  * counterpart of this entry point; it only changes where the scratch lives.
  *
- * - Problems needing more than FA_NOALLOC_MAX_ROWS values (H * token rows)
- *   return FA_ERR_SCRATCH_LIMIT and launch nothing; use fa_bwd for them.
+ * - Problems whose workspace (fa_bwd_workspace_size) exceeds
+ *   8 * FA_NOALLOC_MAX_ROWS bytes return FA_ERR_SCRATCH_LIMIT and launch
+ *   nothing; use fa_bwd for them.
  * - It calls no cudaMalloc / cudaFree and no allocating library routine.
  * - The first call on a device looks up the array's device address (a
  *   one-time set-up with that device current); make that first call before

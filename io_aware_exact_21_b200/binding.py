@@ -19,7 +19,7 @@ STATUS = {
     -4: "FA_ERR_MISALIGNED", -5: "FA_ERR_BAD_MASK", -6: "FA_ERR_WORKSPACE", -7: "FA_ERR_CUDA",
     -8: "FA_ERR_DEVICE_TIMEOUT", -9: "FA_ERR_BAD_SCALE", -10: "FA_ERR_SCRATCH_LIMIT",
 }
-NOALLOC_MAX_ROWS = 1 << 20   # FA_NOALLOC_MAX_ROWS in include/fa.h
+NOALLOC_MAX_ROWS = 1 << 20   # FA_NOALLOC_MAX_ROWS in include/fa.h (8-byte entries)
 
 # Exported entry points and their C signatures.
 _VP, _I, _F, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t

@@ -13,19 +13,25 @@
 //   dQ_i  = scale * sum_j dS_ij k_j
 //
 // Three kernels on the caller's stream:
-//   1. dot_kernel : D_i = rowsum(dO_i * O_i) in fp32, one row per group of
-//      d/8 lanes reading 16-byte vectors, reduced with warp shuffles.
+//   1. stats_kernel: D_i = rowsum(dO_i * O_i) in fp32 (one row per group of
+//      d/8 lanes reading 16-byte vectors, reduced with warp shuffles), stored
+//      with -LSE_i log2(e) in a 128-row padded layout.
 //   2. dkdv_kernel: a CTA owns 128 keys of one (sequence, head) and streams
-//      the query tiles (64 rows) that can see them.  Per query tile:
+//      the 128-row query tiles that can see them.  Per query tile:
 //        S^T = K Q^T and dP^T = V dO^T        (tcgen05, both operands in smem)
 //        P^T = 2^(S^T scale log2e - L log2e), dS^T = P^T (dP^T - D)   (fp32)
 //        dV += P^T dO and dK += dS^T Q        (tcgen05, P^T / dS^T from TMEM)
-//   3. dq_kernel  : a CTA owns 128 queries and streams the key tiles (64 keys):
+//   3. dq_kernel  : a CTA owns 128 queries and streams 128-key tiles:
 //        S = Q K^T, dP = dO V^T, P, dS as above, dQ += dS K.
-// Both big kernels use the forward's role split (TMA warp, MMA warp, two
-// element-wise warpgroups, each taking one 32-column half of every score
-// tile) and double-buffer the score tiles in TMEM, so the element-wise work
-// of one tile overlaps the GEMMs of the next.  Deterministic: no atomics.
+// Every GEMM is 128 x 128 (x 128): on sm_100a an MMA with N = 64 costs as
+// much tensor time as one with N = 128, so 64-wide score tiles would run the
+// tensor core at half rate.  Both big kernels use the forward's role split
+// (TMA warp, MMA warp, two element-wise warpgroups, each taking one 64-column
+// half of every score tile).  The score tiles are single-buffered in TMEM
+// (dK, dV or dQ take the other columns) and the element-wise warps release
+// their results in two steps -- P first (the dV GEMM and the next S^T start),
+// dS second -- so GEMMs and element-wise work overlap.  Deterministic: no
+// atomics.
 #pragma once
 
 #include "schedule.cuh"
@@ -35,10 +41,18 @@ namespace fa {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Per-row statistics the two gradient kernels read, written by the pre-pass
+// into the workspace: {-LSE_i * log2(e), D_i} for each (sequence, head, row),
+// in a layout padded to 128-row blocks so that a streamed tile's statistics
+// are one aligned 1 KB bulk copy:
+//   fixed length: ((s * H + h) * stride) + i,     stride = N rounded up to 128
+//   packed:       h * stride + 128 * blocks(s) + i, blocks(s) = sum over earlier
+//                 sequences of ceil(len / 128), stride >= 128 * blocks(B)
+// Entries of padding rows are never written; readers mask them.
 struct BwdParams {
     Geometry g;
-    const float* lse;       // layout: fixed [B, H, N], packed [H, T]
-    const float* dsum;      // D, same layout
+    const float2* stats;
+    int64_t stats_stride;
     __nv_bfloat16* out0;    // dK (dkdv_kernel) or dQ (dq_kernel)
     __nv_bfloat16* out1;    // dV (dkdv_kernel)
     float scale;
@@ -53,13 +67,34 @@ __device__ __forceinline__ size_t rowstat_index(const Geometry& g, int s, int h,
                         : (static_cast<size_t>(s) * g.H + h) * g.N + i;
 }
 
-// ------------------------------------------------------------ D pre-pass --
+// Index of row i of sequence s, head h in the padded statistics array;
+// `blocks_before` = 128-row blocks of the sequences before s (packed only).
+__device__ __forceinline__ size_t stats_index(const Geometry& g, int64_t stride, int s, int h,
+                                              int blocks_before, int i) {
+    return g.cu_seqlens ? static_cast<size_t>(h) * stride + static_cast<size_t>(blocks_before) * 128 + i
+                        : (static_cast<size_t>(s) * g.H + h) * stride + i;
+}
+
+// ------------------------------------------------------------ pre-pass --
+// stats[row] = {-LSE * log2(e), D = rowsum(dO * O)}: one row per group of d/8
+// lanes reading 16-byte vectors, the dot product reduced with warp shuffles.
+// Packed batches: each CTA first builds the per-sequence block prefix and a
+// copy of cu_seqlens in shared memory to place each token.
 template <int D>
 __global__ void __launch_bounds__(256)
-dot_kernel(const __nv_bfloat16* __restrict__ dO, const __nv_bfloat16* __restrict__ O,
-           float* __restrict__ dsum, Geometry g) {
+stats_kernel(const __nv_bfloat16* __restrict__ dO, const __nv_bfloat16* __restrict__ O,
+             const float* __restrict__ lse, float2* __restrict__ stats, int64_t stride,
+             Geometry g) {
     constexpr int LPR = D / 8;                 // lanes per row (16-byte vectors)
     constexpr int RPW = 32 / LPR;              // rows per warp per iteration
+    extern __shared__ int pre_smem[];
+    int* prefix = pre_smem;                    // B + 1 (packed only)
+    int* cu = pre_smem + kMaxVarlenSeqs + 1;   // B + 1
+    int* scratch = cu + kMaxVarlenSeqs + 1;    // blockDim
+    if (g.cu_seqlens) {
+        for (int i = threadIdx.x; i <= g.B; i += blockDim.x) cu[i] = g.cu_seqlens[i];
+        build_schedule_prefix(g, 128, prefix, scratch);   // __syncthreads inside
+    }
     const int lane = threadIdx.x & 31;
     const int sub = lane / LPR;
     const int part = lane % LPR;
@@ -87,14 +122,23 @@ dot_kernel(const __nv_bfloat16* __restrict__ dO, const __nv_bfloat16* __restrict
         if (r < rows && part == 0) {
             const int64_t token = r / g.H;
             const int h = static_cast<int>(r - token * g.H);
-            size_t idx;
+            int s, i, blocks_before = 0;
             if (g.cu_seqlens) {
-                idx = static_cast<size_t>(h) * g.T + token;
+                if (token >= cu[g.B]) continue;        // a row outside every sequence
+                int lo = 0, hi = g.B - 1;              // last s with cu[s] <= token
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (cu[mid] <= token) lo = mid; else hi = mid - 1;
+                }
+                s = lo;
+                i = static_cast<int>(token - cu[s]);
+                blocks_before = prefix[s];
             } else {
-                const int64_t s = token / g.N;
-                idx = (static_cast<size_t>(s) * g.H + h) * g.N + (token - s * g.N);
+                s = static_cast<int>(token / g.N);
+                i = static_cast<int>(token - static_cast<int64_t>(s) * g.N);
             }
-            dsum[idx] = acc;
+            const float l = lse[rowstat_index(g, s, h, g.cu_seqlens ? cu[s] : 0, i)];
+            stats[stats_index(g, stride, s, h, blocks_before, i)] = make_float2(-l * 1.4426950408889634f, acc);
         }
     }
 }
@@ -103,23 +147,21 @@ dot_kernel(const __nv_bfloat16* __restrict__ dO, const __nv_bfloat16* __restrict
 template <int D>
 struct BwdCfg {
     static constexpr int BM = 128;               // rows the CTA owns (keys or queries)
-    static constexpr int BS = 64;                // rows streamed per step
-    static constexpr int NSTAGE = 4;
+    static constexpr int BS = 128;               // rows streamed per step
+    static constexpr int NSTAGE = 2;
     static constexpr int NBOX = D / 64;
-    static constexpr int FBOX = 128 * 128;       // 128 rows x 128 B
-    static constexpr int SBOX = 64 * 128;        // 64 rows x 128 B
-    static constexpr int FIX_BYTES = BM * D * 2;
-    static constexpr int STR_BYTES = BS * D * 2;
+    static constexpr int BOX = 128 * 128;        // one TMA box: 128 rows x 128 B
+    static constexpr int TILE_BYTES = 128 * D * 2;
     static constexpr int THREADS = 384;
-    static constexpr uint32_t COL_ACC0 = 0, COL_ACC1 = 128;
-    __host__ __device__ static constexpr uint32_t col_s(int b) { return 256 + 128 * b; }
-    __host__ __device__ static constexpr uint32_t col_dp(int b) { return 256 + 128 * b + 64; }
-    static constexpr int OFF_FA = 0;
-    static constexpr int OFF_FB = FIX_BYTES;
-    static constexpr int OFF_ST = 2 * FIX_BYTES;                  // stage: X then Y
-    static constexpr int OFF_VEC = OFF_ST + NSTAGE * 2 * STR_BYTES;  // stage: 64 nl + 64 D
-    static constexpr int OFF_BAR = OFF_VEC + NSTAGE * 2 * BS * 4;
-    static constexpr int NBAR = 2 + 2 * NSTAGE + 2 + 2 + 2 + 1;
+    // TMEM columns: accumulators, then the score tile and its gradient tile
+    static constexpr uint32_t COL_ACC0 = 0, COL_ACC1 = 128, COL_S = 256, COL_DP = 384;
+    static constexpr int OFF_FA = 0;                               // fixed tile A (K or Q)
+    static constexpr int OFF_FB = TILE_BYTES;                      // fixed tile B (V or dO)
+    static constexpr int OFF_ST = 2 * TILE_BYTES;                  // stages: X then Y
+    static constexpr int OFF_VEC = OFF_ST + NSTAGE * 2 * TILE_BYTES;  // stage stats: float2[BS]
+    static constexpr int VEC_BYTES = BS * 8;
+    static constexpr int OFF_BAR = OFF_VEC + NSTAGE * VEC_BYTES;
+    static constexpr int NBAR = 2 + 2 * NSTAGE + 4 + 2 + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int OFF_SCRATCH = OFF_MISC + 16;
     static constexpr int OFF_PREFIX = OFF_SCRATCH + THREADS * 4;
@@ -138,9 +180,13 @@ __device__ __forceinline__ void query_tile_range(int k_lo, int k_hi, int n, int 
     if (ie < ib) ie = ib;
 }
 
+// Barriers.  s_full / dp_full: the score GEMM and the gradient GEMM of a step
+// have completed.  mid: the element-wise warps are done with the first half
+// of their work (dK/dV kernel: P^T written; dQ kernel: S read).  ready: dS
+// written.  Each completes once per step, so its parity is the step count's.
 struct BwdBarriers {
-    uint64_t *fix_full, *fix_empty, *stage_full, *stage_empty, *s_full, *ready, *acc_final,
-        *acc_empty, *drain;
+    uint64_t *fix_full, *fix_empty, *stage_full, *stage_empty, *s_full, *dp_full, *mid, *ready,
+        *acc_final, *acc_empty, *drain;
 };
 
 template <int D>
@@ -153,8 +199,10 @@ __device__ __forceinline__ BwdBarriers carve_barriers(uint8_t* smem) {
     r.stage_full = b + 2;
     r.stage_empty = b + 2 + C::NSTAGE;
     r.s_full = b + 2 + 2 * C::NSTAGE;
-    r.ready = r.s_full + 2;
-    r.acc_final = r.ready + 2;
+    r.dp_full = r.s_full + 1;
+    r.mid = r.dp_full + 1;
+    r.ready = r.mid + 1;
+    r.acc_final = r.ready + 1;
     r.acc_empty = r.acc_final + 1;
     r.drain = r.acc_empty + 1;
     return r;
@@ -169,47 +217,47 @@ __device__ __forceinline__ void init_barriers(const BwdBarriers& br, volatile in
         mbar_init(br.stage_full + s, 1);
         mbar_init(br.stage_empty + s, 1);
     }
-    for (int b = 0; b < 2; ++b) {
-        mbar_init(br.s_full + b, 1);
-        mbar_init(br.ready + b, 8);     // all eight element-wise warps (both halves of a tile)
-    }
+    mbar_init(br.s_full, 1);
+    mbar_init(br.dp_full, 1);
+    mbar_init(br.mid, 8);               // all eight element-wise warps
+    mbar_init(br.ready, 8);
     mbar_init(br.acc_final, 1);
-    mbar_init(br.acc_empty, 8);         // all eight element-wise warps
+    mbar_init(br.acc_empty, 8);
     mbar_init(br.drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
 }
 
-// A-operand (K-major, 128 rows) and B-operand (K-major, 64 rows) descriptors
-// for k-step kk of a d-deep contraction: 16 channels = 32 bytes inside the
-// 128-byte swizzled rows, next 64-channel box after four steps.
+// D[128 x 128] = A[smem 128 x d, K-major] * B[smem 128 x d, K-major]^T.
+// k-step kk covers channels 16kk..16kk+15: 32 bytes inside the 128-byte
+// swizzled rows, the next 64-channel box after four steps.
 template <int D>
-__device__ __forceinline__ void issue_ss_pair(uint32_t d_tmem, uint32_t a_base, uint32_t b_base,
-                                              uint32_t idesc) {
+__device__ __forceinline__ void issue_scores_ss(uint32_t d_tmem, uint32_t a_base, uint32_t b_base) {
     using C = BwdCfg<D>;
+    constexpr uint32_t IDESC = idesc_bf16(128, C::BS, false, false);
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t ka = (kk >> 2) * C::FBOX + (kk & 3) * 32;
-        const uint32_t kb = (kk >> 2) * C::SBOX + (kk & 3) * 32;
-        umma_ss(d_tmem, sw128_desc(a_base + ka, 16, 1024), sw128_desc(b_base + kb, 16, 1024), idesc,
-                kk > 0);
+        const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+        umma_ss(d_tmem, sw128_desc(a_base + off, 16, 1024), sw128_desc(b_base + off, 16, 1024),
+                IDESC, kk > 0);
     }
 }
 
 // Column of the packed bf16 operand for 16-row k-step kk: each element-wise
-// warpgroup packs its 32-column half h of a score tile into the first 16 of
-// that half's columns (h * 32 ... h * 32 + 15), which it has already read.
-__host__ __device__ constexpr uint32_t packed_col(int kk) { return (kk >> 1) * 32 + (kk & 1) * 8; }
+// warpgroup packs its 64-column half h of a score tile into the first 32 of
+// that half's columns (h * 64 ... h * 64 + 31), which it has already read.
+__host__ __device__ constexpr uint32_t packed_col(int kk) { return (kk >> 2) * 64 + (kk & 3) * 8; }
 
-// acc[128 x D] (+)= A[tmem, 128 x 64 bf16] * B[smem, 64 x D, MN-major].
+// acc[128 x D] (+)= A[tmem, 128 x 128 bf16, packed] * B[smem, 128 x D, MN-major].
 template <int D>
-__device__ __forceinline__ void issue_ts_acc(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base,
-                                             uint32_t idesc, bool accumulate) {
+__device__ __forceinline__ void issue_acc_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base,
+                                             bool accumulate) {
     using C = BwdCfg<D>;
+    constexpr uint32_t IDESC = idesc_bf16(128, D, false, true);
 #pragma unroll
     for (int kk = 0; kk < C::BS / 16; ++kk)
-        umma_ts(d_tmem, a_tmem + packed_col(kk), sw128_desc(b_base + kk * 2048, C::SBOX, 1024),
-                idesc, (accumulate || kk > 0) ? 1u : 0u);
+        umma_ts(d_tmem, a_tmem + packed_col(kk), sw128_desc(b_base + kk * 2048, C::BOX, 1024),
+                IDESC, (accumulate || kk > 0) ? 1u : 0u);
 }
 
 // Bounded wait that ignores the abort flag (used to drain in-flight work).
@@ -236,6 +284,58 @@ __device__ __forceinline__ void store_row_chunk(uint32_t taddr, float mul, __nv_
     }
 }
 
+// Load 64 consecutive TMEM columns of this warp's 32 lanes.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+    tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+    tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+}
+
+__device__ __forceinline__ void arrive_warp(uint64_t* bar) {
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane_id() == 0) mbar_arrive(bar);
+}
+
+// Common prologue of both big kernels: barriers, TMEM, schedule.
+template <int D>
+__device__ __forceinline__ uint32_t bwd_prologue(uint8_t* smem, const BwdBarriers& br,
+                                                 volatile int* abort_flag, const BwdParams& p,
+                                                 Schedule& sch, int heavy_first,
+                                                 const CUtensorMap* maps[4]) {
+    using C = BwdCfg<D>;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+    int* scratch = reinterpret_cast<int*>(smem + C::OFF_SCRATCH);
+    int* prefix = reinterpret_cast<int*>(smem + C::OFF_PREFIX);
+    const int warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0) init_barriers<D>(br, abort_flag);
+    if (warp == 0 && lane_id() == 0)
+        for (int i = 0; i < 4; ++i) tma_prefetch_map(maps[i]);
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, 512);
+        tmem_relinquish();
+    }
+    sch.g = p.g;
+    sch.rows_per_item = C::BM;
+    sch.heavy_first = heavy_first;
+    sch.prefix = prefix;
+    sch.total_items = build_schedule_prefix(p.g, C::BM, prefix, scratch);   // __syncthreads inside
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    return *tmem_holder;
+}
+
+template <int D>
+__device__ __forceinline__ void bwd_epilogue_sync(uint32_t tmem) {
+    tc_fence_before();
+    __syncthreads();
+    if ((threadIdx.x >> 5) == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
 // --------------------------------------------------------- dK/dV kernel --
 template <int D>
 __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
@@ -244,38 +344,16 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             const BwdParams p) {
     using C = BwdCfg<D>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                               ~static_cast<uintptr_t>(1023));
+    uint8_t* smem = align_smem_1024(smem_raw);
     const BwdBarriers br = carve_barriers<D>(smem);
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
-    int* scratch = reinterpret_cast<int*>(smem + C::OFF_SCRATCH);
-    int* prefix = reinterpret_cast<int*>(smem + C::OFF_PREFIX);
-    float* vec = reinterpret_cast<float*>(smem + C::OFF_VEC);
+    float2* vec = reinterpret_cast<float2*>(smem + C::OFF_VEC);
+    const CUtensorMap* maps[4] = {&tm_k, &tm_v, &tm_q, &tm_do};
+    Schedule sch;
+    // under a causal mask the first key block sees the most queries: natural order
+    const uint32_t tmem = bwd_prologue<D>(smem, br, abort_flag, p, sch, 0, maps);
     const int warp = threadIdx.x >> 5;
     const int lane = lane_id();
-
-    if (threadIdx.x == 0) init_barriers<D>(br, abort_flag);
-    if (warp == 0 && lane == 0) {
-        tma_prefetch_map(&tm_k);
-        tma_prefetch_map(&tm_v);
-        tma_prefetch_map(&tm_q);
-        tma_prefetch_map(&tm_do);
-    }
-    if (warp == 1) {
-        tmem_alloc(tmem_holder, 512);
-        tmem_relinquish();
-    }
-    Schedule sch;
-    sch.g = p.g;
-    sch.rows_per_item = C::BM;
-    sch.heavy_first = 0;       // under a causal mask the first key block sees the most queries
-    sch.prefix = prefix;
-    sch.total_items = build_schedule_prefix(p.g, C::BM, prefix, scratch);
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_holder;
     const WaitCtl wc{abort_flag, p.error_word, p.timeout_ns};
     const int H = p.g.H;
 
@@ -296,49 +374,40 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                 if (lane == 0) {
                     ok = mbar_wait(br.fix_empty, (item_it & 1) ^ 1, wc);
                     if (ok) {
-                        mbar_arrive_expect_tx(br.fix_full, 2 * C::FIX_BYTES);
+                        mbar_arrive_expect_tx(br.fix_full, 2 * C::TILE_BYTES);
                         for (int b = 0; b < C::NBOX; ++b) {
-                            tma_load_3d(smem + C::OFF_FA + b * C::FBOX, &tm_k, br.fix_full, b * 64, h,
+                            tma_load_3d(smem + C::OFF_FA + b * C::BOX, &tm_k, br.fix_full, b * 64, h,
                                         sp.start + k0);
-                            tma_load_3d(smem + C::OFF_FB + b * C::FBOX, &tm_v, br.fix_full, b * 64, h,
+                            tma_load_3d(smem + C::OFF_FB + b * C::BOX, &tm_v, br.fix_full, b * 64, h,
                                         sp.start + k0);
                         }
                         ++fix_issued;
                     }
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
+                const int blocks_before = p.g.cu_seqlens ? sch.prefix[s] : 0;
                 for (int i = ib; i < ie && ok; ++i, ++cnt) {
                     const int slot = cnt % C::NSTAGE;
-                    if (lane == 0) ok = mbar_wait(br.stage_empty + slot, ((cnt / C::NSTAGE) & 1) ^ 1, wc);
+                    if (lane == 0) {
+                        ok = mbar_wait(br.stage_empty + slot, ((cnt / C::NSTAGE) & 1) ^ 1, wc);
+                        if (ok) {
+                            mbar_arrive_expect_tx(br.stage_full + slot, 2 * C::TILE_BYTES + C::VEC_BYTES);
+                            uint8_t* st = smem + C::OFF_ST + slot * 2 * C::TILE_BYTES;
+                            for (int b = 0; b < C::NBOX; ++b) {
+                                tma_load_3d(st + b * C::BOX, &tm_q, br.stage_full + slot, b * 64, h,
+                                            sp.start + i * C::BS);
+                                tma_load_3d(st + C::TILE_BYTES + b * C::BOX, &tm_do, br.stage_full + slot,
+                                            b * 64, h, sp.start + i * C::BS);
+                            }
+                            // the tile's per-query statistics, one aligned 1 KB copy
+                            bulk_load(vec + slot * C::BS,
+                                      p.stats + stats_index(p.g, p.stats_stride, s, h, blocks_before,
+                                                            i * C::BS),
+                                      C::VEC_BYTES, br.stage_full + slot);
+                        }
+                    }
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (!ok) break;
-                    // per-query statistics of this tile: -L*log2(e) and D (query rows
-                    // outside the sequence get -inf, which zeroes their P)
-                    float* vs = vec + slot * 2 * C::BS;
-#pragma unroll
-                    for (int e = 0; e < C::BS / 32; ++e) {
-                        const int q = i * C::BS + e * 32 + lane;
-                        float nl = -INFINITY, dd = 0.f;
-                        if (q < n) {
-                            const size_t idx = rowstat_index(p.g, s, h, sp.start, q);
-                            nl = -p.lse[idx] * kLog2e;
-                            dd = p.dsum[idx];
-                        }
-                        vs[e * 32 + lane] = nl;
-                        vs[C::BS + e * 32 + lane] = dd;
-                    }
-                    __threadfence_block();
-                    __syncwarp();
-                    if (lane == 0) {
-                        mbar_arrive_expect_tx(br.stage_full + slot, 2 * C::STR_BYTES);
-                        uint8_t* st = smem + C::OFF_ST + slot * 2 * C::STR_BYTES;
-                        for (int b = 0; b < C::NBOX; ++b) {
-                            tma_load_3d(st + b * C::SBOX, &tm_q, br.stage_full + slot, b * 64, h,
-                                        sp.start + i * C::BS);
-                            tma_load_3d(st + C::STR_BYTES + b * C::SBOX, &tm_do, br.stage_full + slot,
-                                        b * 64, h, sp.start + i * C::BS);
-                        }
-                    }
                 }
             }
             if (!ok && lane == 0) {
@@ -348,19 +417,13 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             }
         } else if (warp == 1 && lane == 0) {
             // ---------------------------------------------------- MMA --
-            constexpr uint32_t IDESC_S = idesc_bf16(128, C::BS, false, false);
-            constexpr uint32_t IDESC_ACC = idesc_bf16(128, D, false, true);
+            // per step i:  S^T_i, dP^T_i  ->  [P^T_i written] dV += P^T_i dO_i, S^T_{i+1}
+            //              ->  [dS^T_i written] dK += dS^T_i Q_i, dP^T_{i+1}
             const uint32_t fa_addr = smem_u32(smem + C::OFF_FA);
             const uint32_t fb_addr = smem_u32(smem + C::OFF_FB);
             const uint32_t st_addr = smem_u32(smem + C::OFF_ST);
             uint32_t cnt = 0, item_it = 0;
             bool ok = true;
-            auto issue_scores = [&](int b, uint32_t slot) {
-                const uint32_t x = st_addr + slot * 2 * C::STR_BYTES;
-                issue_ss_pair<D>(tmem + C::col_s(b), fa_addr, x, IDESC_S);              // K Q^T
-                issue_ss_pair<D>(tmem + C::col_dp(b), fb_addr, x + C::STR_BYTES, IDESC_S); // V dO^T
-                umma_commit(br.s_full + b);
-            };
             for (int w = blockIdx.x; w < sch.total_items && ok; w += gridDim.x, ++item_it) {
                 int s, h, blk;
                 sch.item(w, s, h, blk);
@@ -376,29 +439,38 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                     break;
                 }
                 tc_fence_after();
-                issue_scores(cnt & 1, cnt % C::NSTAGE);
+                {
+                    const uint32_t x = st_addr + (cnt % C::NSTAGE) * 2 * C::TILE_BYTES;
+                    issue_scores_ss<D>(tmem + C::COL_S, fa_addr, x);                  // K Q^T
+                    umma_commit(br.s_full);
+                    issue_scores_ss<D>(tmem + C::COL_DP, fb_addr, x + C::TILE_BYTES);  // V dO^T
+                    umma_commit(br.dp_full);
+                }
                 for (int i = ib; i < ie; ++i, ++cnt) {
-                    const int b = cnt & 1;
                     const bool last = (i + 1 == ie);
                     const uint32_t slot = cnt % C::NSTAGE;
+                    const uint32_t x = st_addr + slot * 2 * C::TILE_BYTES;
+                    const uint32_t xn = st_addr + ((cnt + 1) % C::NSTAGE) * 2 * C::TILE_BYTES;
+                    if (!mbar_wait(br.mid, cnt & 1, wc)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_acc_ts<D>(tmem + C::COL_ACC1, tmem + C::COL_S, x + C::TILE_BYTES, i > ib);  // dV
                     if (!last) {
-                        const uint32_t nslot = (cnt + 1) % C::NSTAGE;
-                        if (!mbar_wait(br.stage_full + nslot, ((cnt + 1) / C::NSTAGE) & 1, wc)) {
+                        if (!mbar_wait(br.stage_full + (cnt + 1) % C::NSTAGE, ((cnt + 1) / C::NSTAGE) & 1, wc)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
-                        issue_scores(b ^ 1, nslot);
+                        issue_scores_ss<D>(tmem + C::COL_S, fa_addr, xn);             // next K Q^T
+                        umma_commit(br.s_full);
                     }
-                    if (!mbar_wait(br.ready + b, (cnt >> 1) & 1, wc)) { ok = false; break; }
+                    if (!mbar_wait(br.ready, cnt & 1, wc)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t x = st_addr + slot * 2 * C::STR_BYTES;
-                    issue_ts_acc<D>(tmem + C::COL_ACC1, tmem + C::col_s(b), x + C::STR_BYTES, IDESC_ACC,
-                                    i > ib);                                          // dV += P^T dO
-                    issue_ts_acc<D>(tmem + C::COL_ACC0, tmem + C::col_dp(b), x, IDESC_ACC,
-                                    i > ib);                                          // dK += dS^T Q
+                    issue_acc_ts<D>(tmem + C::COL_ACC0, tmem + C::COL_DP, x, i > ib);     // dK
                     umma_commit(br.stage_empty + slot);
-                    if (last) {
+                    if (!last) {
+                        issue_scores_ss<D>(tmem + C::COL_DP, fb_addr, xn + C::TILE_BYTES);  // next V dO^T
+                        umma_commit(br.dp_full);
+                    } else {
                         umma_commit(br.acc_final);
                         umma_commit(br.fix_empty);
                     }
@@ -413,11 +485,13 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
     } else {
         // ------------------------------------ element-wise warpgroups --
         regs_alloc<200>();
-        const int g = (warp >> 2) - 1;
+        const int g = (warp >> 2) - 1;             // 64-column half of each tile
         const int wq = warp & 3;
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
         const int row = wq * 32 + lane;
         const float sl2 = p.scale_log2;
+        const uint32_t tS = tmem + lane_base + C::COL_S + 64 * g;
+        const uint32_t tP = tmem + lane_base + C::COL_DP + 64 * g;
         uint32_t cnt = 0, item_it = 0;
         bool ok = true;
         for (int w = blockIdx.x; w < sch.total_items && ok; w += gridDim.x, ++item_it) {
@@ -430,8 +504,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             int ib, ie;
             query_tile_range(k0, min(n, k0 + C::BM), n, p.g.causal, p.g.window, C::BS, ib, ie);
             for (int i = ib; i < ie; ++i, ++cnt) {
-                const int b = cnt & 1;
-                if (!mbar_wait(br.s_full + b, (cnt >> 1) & 1, wc)) { ok = false; break; }
+                if (!mbar_wait(br.s_full, cnt & 1, wc)) { ok = false; break; }
                 // The producer wrote this stage's row statistics with ordinary stores
                 // before arriving on stage_full: wait on it too so they are visible.
                 if (!mbar_wait(br.stage_full + cnt % C::NSTAGE, (cnt / C::NSTAGE) & 1, wc)) {
@@ -439,39 +512,57 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                     break;
                 }
                 tc_fence_after();
-                // this warpgroup's half of the tile: queries q0 + 32g ... q0 + 32g + 31
-                const float* vs = vec + (cnt % C::NSTAGE) * 2 * C::BS + 32 * g;
-                const int q0 = i * C::BS + 32 * g;
-                const bool need_mask = (k0 + C::BM > n) || (p.g.causal && k0 + C::BM - 1 > q0) ||
-                                       (p.g.window > 0 && q0 + 31 - k0 >= p.g.window);
-                const uint32_t tS = tmem + lane_base + C::col_s(b) + 32 * g;
-                const uint32_t tP = tmem + lane_base + C::col_dp(b) + 32 * g;
-                uint32_t sr[32], dr[32];
-                tmem_ld32(tS, sr);
-                tmem_ld32(tP, dr);
+                const float2* vs = vec + (cnt % C::NSTAGE) * C::BS + 64 * g;   // {-L log2e, D}
+                const int q0 = i * C::BS + 64 * g;     // this half's first query
+                const bool need_mask = (k0 + C::BM > n) || (q0 + 64 > n) ||
+                                       (p.g.causal && k0 + C::BM - 1 > q0) ||
+                                       (p.g.window > 0 && q0 + 63 - k0 >= p.g.window);
+                uint32_t r[64];
+                tmem_ld64(tS, r);
                 tmem_wait_ld();
-                uint32_t pp[16], dd[16];
+                float pf[64];
+                if (!need_mask) {
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    float pv[2], dv[2];
+                    for (int c = 0; c < 64; ++c) pf[c] = ex2(fmaf(__uint_as_float(r[c]), sl2, vs[c].x));
+                } else {
+                    // masked pairs, and query rows past the sequence end (their
+                    // statistics are padding), get P = 0
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int col = e + u;
-                        float pr = ex2(fmaf(__uint_as_float(sr[col]), sl2, vs[col]));
-                        if (need_mask && !key_allowed(q0 + col, j, n, p.g.causal, p.g.window))
-                            pr = 0.f;
-                        pv[u] = pr;
-                        dv[u] = pr * (__uint_as_float(dr[col]) - vs[C::BS + col]);
+                    for (int c = 0; c < 64; ++c) {
+                        const float x = ex2(fmaf(__uint_as_float(r[c]), sl2, vs[c].x));
+                        pf[c] = (q0 + c < n && key_allowed(q0 + c, j, n, p.g.causal, p.g.window)) ? x : 0.f;
                     }
-                    pp[e / 2] = pack_bf16(pv[0], pv[1]);
-                    dd[e / 2] = pack_bf16(dv[0], dv[1]);
                 }
-                tmem_st16(tS, pp);     // P^T packed over the first 16 columns of this half
-                tmem_st16(tP, dd);     // dS^T likewise in the dP^T half
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(br.ready + b);
+                {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(pf[2 * c], pf[2 * c + 1]);
+                    tmem_st32(tS, pk);           // P^T packed over the first 32 columns of this half
+                }
+                arrive_warp(br.mid);
+                if (!mbar_wait(br.dp_full, cnt & 1, wc)) { ok = false; break; }
+                tc_fence_after();
+                tmem_ld64(tP, r);
+                tmem_wait_ld();
+                {
+                    uint32_t pk[32];
+                    if (!need_mask) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            pk[c] = pack_bf16(pf[2 * c] * (__uint_as_float(r[2 * c]) - vs[2 * c].y),
+                                              pf[2 * c + 1] * (__uint_as_float(r[2 * c + 1]) - vs[2 * c + 1].y));
+                    } else {
+                        // P = 0 must give dS = 0 even where the padding D is not finite
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            const float d0 = pf[2 * c] * (__uint_as_float(r[2 * c]) - vs[2 * c].y);
+                            const float d1 = pf[2 * c + 1] * (__uint_as_float(r[2 * c + 1]) - vs[2 * c + 1].y);
+                            pk[c] = pack_bf16(pf[2 * c] != 0.f ? d0 : 0.f, pf[2 * c + 1] != 0.f ? d1 : 0.f);
+                        }
+                    }
+                    tmem_st32(tP, pk);           // dS^T packed over the first 32 columns of this half
+                }
+                arrive_warp(br.ready);
             }
             if (!ok) break;
             // ------------------------------------------------ epilogue --
@@ -495,13 +586,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             if (lane == 0) mbar_arrive(br.acc_empty);
         }
     }
-
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 512);
-    }
+    bwd_epilogue_sync<D>(tmem);
 }
 
 // ------------------------------------------------------------- dQ kernel --
@@ -512,37 +597,15 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
           const BwdParams p) {
     using C = BwdCfg<D>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                               ~static_cast<uintptr_t>(1023));
+    uint8_t* smem = align_smem_1024(smem_raw);
     const BwdBarriers br = carve_barriers<D>(smem);
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
-    int* scratch = reinterpret_cast<int*>(smem + C::OFF_SCRATCH);
-    int* prefix = reinterpret_cast<int*>(smem + C::OFF_PREFIX);
+    const CUtensorMap* maps[4] = {&tm_q, &tm_do, &tm_k, &tm_v};
+    Schedule sch;
+    // the last query block sees the most keys under a causal mask
+    const uint32_t tmem = bwd_prologue<D>(smem, br, abort_flag, p, sch, p.g.causal, maps);
     const int warp = threadIdx.x >> 5;
     const int lane = lane_id();
-
-    if (threadIdx.x == 0) init_barriers<D>(br, abort_flag);
-    if (warp == 0 && lane == 0) {
-        tma_prefetch_map(&tm_q);
-        tma_prefetch_map(&tm_do);
-        tma_prefetch_map(&tm_k);
-        tma_prefetch_map(&tm_v);
-    }
-    if (warp == 1) {
-        tmem_alloc(tmem_holder, 512);
-        tmem_relinquish();
-    }
-    Schedule sch;
-    sch.g = p.g;
-    sch.rows_per_item = C::BM;
-    sch.heavy_first = p.g.causal;   // the last query block sees the most keys
-    sch.prefix = prefix;
-    sch.total_items = build_schedule_prefix(p.g, C::BM, prefix, scratch);
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_holder;
     const WaitCtl wc{abort_flag, p.error_word, p.timeout_ns};
     const int H = p.g.H;
 
@@ -561,11 +624,11 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
                 int jb, je;
                 key_tile_range(q0, min(n, q0 + C::BM), n, p.g.causal, p.g.window, C::BS, jb, je);
                 if (!mbar_wait(br.fix_empty, (item_it & 1) ^ 1, wc)) { ok = false; break; }
-                mbar_arrive_expect_tx(br.fix_full, 2 * C::FIX_BYTES);
+                mbar_arrive_expect_tx(br.fix_full, 2 * C::TILE_BYTES);
                 for (int b = 0; b < C::NBOX; ++b) {
-                    tma_load_3d(smem + C::OFF_FA + b * C::FBOX, &tm_q, br.fix_full, b * 64, h,
+                    tma_load_3d(smem + C::OFF_FA + b * C::BOX, &tm_q, br.fix_full, b * 64, h,
                                 sp.start + q0);
-                    tma_load_3d(smem + C::OFF_FB + b * C::FBOX, &tm_do, br.fix_full, b * 64, h,
+                    tma_load_3d(smem + C::OFF_FB + b * C::BOX, &tm_do, br.fix_full, b * 64, h,
                                 sp.start + q0);
                 }
                 ++fix_issued;
@@ -575,12 +638,12 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(br.stage_full + slot, 2 * C::STR_BYTES);
-                    uint8_t* st = smem + C::OFF_ST + slot * 2 * C::STR_BYTES;
+                    mbar_arrive_expect_tx(br.stage_full + slot, 2 * C::TILE_BYTES);
+                    uint8_t* st = smem + C::OFF_ST + slot * 2 * C::TILE_BYTES;
                     for (int b = 0; b < C::NBOX; ++b) {
-                        tma_load_3d(st + b * C::SBOX, &tm_k, br.stage_full + slot, b * 64, h,
+                        tma_load_3d(st + b * C::BOX, &tm_k, br.stage_full + slot, b * 64, h,
                                     sp.start + j * C::BS);
-                        tma_load_3d(st + C::STR_BYTES + b * C::SBOX, &tm_v, br.stage_full + slot,
+                        tma_load_3d(st + C::TILE_BYTES + b * C::BOX, &tm_v, br.stage_full + slot,
                                     b * 64, h, sp.start + j * C::BS);
                     }
                 }
@@ -592,19 +655,13 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             }
         } else if (warp == 1 && lane == 0) {
             // ---------------------------------------------------- MMA --
-            constexpr uint32_t IDESC_S = idesc_bf16(128, C::BS, false, false);
-            constexpr uint32_t IDESC_ACC = idesc_bf16(128, D, false, true);
+            // per step j:  S_j, dP_j  ->  [S_j read] S_{j+1}  ->  [dS_j written]
+            //              dQ += dS_j K_j, dP_{j+1}
             const uint32_t fa_addr = smem_u32(smem + C::OFF_FA);
             const uint32_t fb_addr = smem_u32(smem + C::OFF_FB);
             const uint32_t st_addr = smem_u32(smem + C::OFF_ST);
             uint32_t cnt = 0, item_it = 0;
             bool ok = true;
-            auto issue_scores = [&](int b, uint32_t slot) {
-                const uint32_t x = st_addr + slot * 2 * C::STR_BYTES;
-                issue_ss_pair<D>(tmem + C::col_s(b), fa_addr, x, IDESC_S);              // Q K^T
-                issue_ss_pair<D>(tmem + C::col_dp(b), fb_addr, x + C::STR_BYTES, IDESC_S); // dO V^T
-                umma_commit(br.s_full + b);
-            };
             for (int w = blockIdx.x; w < sch.total_items && ok; w += gridDim.x, ++item_it) {
                 int s, h, blk;
                 sch.item(w, s, h, blk);
@@ -620,27 +677,36 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
                     break;
                 }
                 tc_fence_after();
-                issue_scores(cnt & 1, cnt % C::NSTAGE);
+                {
+                    const uint32_t x = st_addr + (cnt % C::NSTAGE) * 2 * C::TILE_BYTES;
+                    issue_scores_ss<D>(tmem + C::COL_S, fa_addr, x);                  // Q K^T
+                    umma_commit(br.s_full);
+                    issue_scores_ss<D>(tmem + C::COL_DP, fb_addr, x + C::TILE_BYTES);  // dO V^T
+                    umma_commit(br.dp_full);
+                }
                 for (int j = jb; j < je; ++j, ++cnt) {
-                    const int b = cnt & 1;
                     const bool last = (j + 1 == je);
                     const uint32_t slot = cnt % C::NSTAGE;
+                    const uint32_t x = st_addr + slot * 2 * C::TILE_BYTES;
+                    const uint32_t xn = st_addr + ((cnt + 1) % C::NSTAGE) * 2 * C::TILE_BYTES;
                     if (!last) {
-                        const uint32_t nslot = (cnt + 1) % C::NSTAGE;
-                        if (!mbar_wait(br.stage_full + nslot, ((cnt + 1) / C::NSTAGE) & 1, wc)) {
+                        if (!mbar_wait(br.stage_full + (cnt + 1) % C::NSTAGE, ((cnt + 1) / C::NSTAGE) & 1, wc)) {
                             ok = false;
                             break;
                         }
+                        if (!mbar_wait(br.mid, cnt & 1, wc)) { ok = false; break; }
                         tc_fence_after();
-                        issue_scores(b ^ 1, nslot);
+                        issue_scores_ss<D>(tmem + C::COL_S, fa_addr, xn);             // next Q K^T
+                        umma_commit(br.s_full);
                     }
-                    if (!mbar_wait(br.ready + b, (cnt >> 1) & 1, wc)) { ok = false; break; }
+                    if (!mbar_wait(br.ready, cnt & 1, wc)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t x = st_addr + slot * 2 * C::STR_BYTES;
-                    issue_ts_acc<D>(tmem + C::COL_ACC0, tmem + C::col_dp(b), x, IDESC_ACC,
-                                    j > jb);                                          // dQ += dS K
+                    issue_acc_ts<D>(tmem + C::COL_ACC0, tmem + C::COL_DP, x, j > jb);     // dQ += dS K
                     umma_commit(br.stage_empty + slot);
-                    if (last) {
+                    if (!last) {
+                        issue_scores_ss<D>(tmem + C::COL_DP, fb_addr, xn + C::TILE_BYTES);  // next dO V^T
+                        umma_commit(br.dp_full);
+                    } else {
                         umma_commit(br.acc_final);
                         umma_commit(br.fix_empty);
                     }
@@ -660,6 +726,8 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
         const int row = wq * 32 + lane;
         const float sl2 = p.scale_log2;
+        const uint32_t tS = tmem + lane_base + C::COL_S + 64 * g;
+        const uint32_t tP = tmem + lane_base + C::COL_DP + 64 * g;
         uint32_t cnt = 0, item_it = 0;
         bool ok = true;
         for (int w = blockIdx.x; w < sch.total_items && ok; w += gridDim.x, ++item_it) {
@@ -673,42 +741,46 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             key_tile_range(q0, min(n, q0 + C::BM), n, p.g.causal, p.g.window, C::BS, jb, je);
             float nl = -INFINITY, dq_d = 0.f;
             if (q < n) {
-                const size_t idx = rowstat_index(p.g, s, h, sp.start, q);
-                nl = -p.lse[idx] * kLog2e;
-                dq_d = p.dsum[idx];
+                const float2 st = p.stats[stats_index(p.g, p.stats_stride, s, h,
+                                                      p.g.cu_seqlens ? sch.prefix[s] : 0, q)];
+                nl = st.x;
+                dq_d = st.y;
             }
             for (int j = jb; j < je; ++j, ++cnt) {
-                const int b = cnt & 1;
-                if (!mbar_wait(br.s_full + b, (cnt >> 1) & 1, wc)) { ok = false; break; }
+                if (!mbar_wait(br.s_full, cnt & 1, wc)) { ok = false; break; }
                 tc_fence_after();
-                // this warpgroup's half of the tile: keys kb ... kb + 31
-                const int kb = j * C::BS + 32 * g;
-                const bool need_mask = tile_needs_mask(q0, C::BM, kb, 32, n, p.g.causal, p.g.window);
-                const uint32_t tS = tmem + lane_base + C::col_s(b) + 32 * g;
-                const uint32_t tP = tmem + lane_base + C::col_dp(b) + 32 * g;
-                uint32_t sr[32], dr[32];
-                tmem_ld32(tS, sr);
-                tmem_ld32(tP, dr);
+                const int kb = j * C::BS + 64 * g;     // this half's first key
+                const bool need_mask = tile_needs_mask(q0, C::BM, kb, 64, n, p.g.causal, p.g.window);
+                uint32_t r[64];
+                tmem_ld64(tS, r);
                 tmem_wait_ld();
-                uint32_t dd[16];
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    float dv[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int col = e + u;
-                        float pr = ex2(fmaf(__uint_as_float(sr[col]), sl2, nl));
-                        if (need_mask && !key_allowed(q, kb + col, n, p.g.causal, p.g.window))
-                            pr = 0.f;
-                        dv[u] = pr * (__uint_as_float(dr[col]) - dq_d);
-                    }
-                    dd[e / 2] = pack_bf16(dv[0], dv[1]);
-                }
-                tmem_st16(tP, dd);     // dS packed over the first 16 columns of this half
-                tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(br.ready + b);
+                if (lane == 0) mbar_arrive(br.mid);     // S read: the next S may overwrite it
+                float pf[64];
+                if (!need_mask) {
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) pf[c] = ex2(fmaf(__uint_as_float(r[c]), sl2, nl));
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) {
+                        const float x = ex2(fmaf(__uint_as_float(r[c]), sl2, nl));
+                        pf[c] = key_allowed(q, kb + c, n, p.g.causal, p.g.window) ? x : 0.f;
+                    }
+                }
+                if (!mbar_wait(br.dp_full, cnt & 1, wc)) { ok = false; break; }
+                tc_fence_after();
+                tmem_ld64(tP, r);
+                tmem_wait_ld();
+                {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        pk[c] = pack_bf16(pf[2 * c] * (__uint_as_float(r[2 * c]) - dq_d),
+                                          pf[2 * c + 1] * (__uint_as_float(r[2 * c + 1]) - dq_d));
+                    tmem_st32(tP, pk);           // dS packed over the first 32 columns of this half
+                }
+                arrive_warp(br.ready);
             }
             if (!ok) break;
             // ------------------------------------------------ epilogue --
@@ -726,19 +798,12 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             if (lane == 0) mbar_arrive(br.acc_empty);
         }
     }
-
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 512);
-    }
+    bwd_epilogue_sync<D>(tmem);
 }
 
 // ------------------------------------------------------------ host side --
 struct BwdMaps {
-    CUtensorMap q64, do64, k128, v128;   // dK/dV kernel
-    CUtensorMap q128, do128, k64, v64;   // dQ kernel
+    CUtensorMap q, k, v, dO;   // 128-row boxes
 };
 
 struct BwdArgs {
@@ -747,19 +812,37 @@ struct BwdArgs {
     const void *o, *dO;
     const float* lse;
     void *dq, *dk, *dv;
-    float* dsum;
+    float2* stats;           // workspace
+    int64_t stats_stride;
     float scale;
     int num_sms;
     int* error_word;
     uint64_t timeout_ns;
 };
 
-inline size_t bwd_workspace_bytes(int64_t rows, int H) {
-    return static_cast<size_t>((rows * H * 4 + 255) / 256 * 256);
+// Row stride of the padded statistics array (see BwdParams).
+inline int64_t bwd_stats_stride(int B, int N, int64_t packed_rows, bool packed) {
+    if (!packed) return (static_cast<int64_t>(N) + 127) / 128 * 128;
+    return (packed_rows + 127 * static_cast<int64_t>(B) + 127) / 128 * 128;
 }
+
+// Workspace bytes: the padded statistics array, 8 bytes per entry.
+inline size_t bwd_workspace_bytes(int B, int H, int64_t stride, bool packed) {
+    const int64_t entries = packed ? static_cast<int64_t>(H) * stride
+                                   : static_cast<int64_t>(B) * H * stride;
+    return static_cast<size_t>((entries * 8 + 255) / 256 * 256);
+}
+
+constexpr int kStatsSmem = (2 * (kMaxVarlenSeqs + 1) + 256) * 4;
 
 inline cudaError_t bwd_set_smem_limits() {
     cudaError_t e;
+    if ((e = cudaFuncSetAttribute(stats_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  kStatsSmem)) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(stats_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  kStatsSmem)) != cudaSuccess)
+        return e;
     if ((e = cudaFuncSetAttribute(dkdv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   BwdCfg<64>::SMEM_BYTES)) != cudaSuccess)
         return e;
@@ -792,15 +875,15 @@ cudaError_t bwd_launch_d(const BwdArgs& a, const BwdMaps& m, cudaStream_t stream
         const int64_t cap = static_cast<int64_t>(a.num_sms) * 8;
         if (blocks > cap) blocks = cap;
         if (blocks < 1) blocks = 1;
-        dot_kernel<D><<<static_cast<int>(blocks), 256, 0, stream>>>(
-            static_cast<const __nv_bfloat16*>(a.dO), static_cast<const __nv_bfloat16*>(a.o),
-            a.dsum, a.g);
+        stats_kernel<D><<<static_cast<int>(blocks), 256, a.g.cu_seqlens ? kStatsSmem : 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(a.dO), static_cast<const __nv_bfloat16*>(a.o), a.lse,
+            a.stats, a.stats_stride, a.g);
         hk.stop(1, slot, stream);
     }
     BwdParams p;
     p.g = a.g;
-    p.lse = a.lse;
-    p.dsum = a.dsum;
+    p.stats = a.stats;
+    p.stats_stride = a.stats_stride;
     p.scale = a.scale;
     p.scale_log2 = a.scale * kLog2e;
     p.error_word = a.error_word;
@@ -813,12 +896,12 @@ cudaError_t bwd_launch_d(const BwdArgs& a, const BwdMaps& m, cudaStream_t stream
     p.out0 = static_cast<__nv_bfloat16*>(a.dk);
     p.out1 = static_cast<__nv_bfloat16*>(a.dv);
     int slot = hk.start(2, stream);
-    dkdv_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(m.k128, m.v128, m.q64, m.do64, p);
+    dkdv_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(m.k, m.v, m.q, m.dO, p);
     hk.stop(2, slot, stream);
     p.out0 = static_cast<__nv_bfloat16*>(a.dq);
     p.out1 = nullptr;
     slot = hk.start(3, stream);
-    dq_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(m.q128, m.do128, m.k64, m.v64, p);
+    dq_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(m.q, m.dO, m.k, m.v, p);
     hk.stop(3, slot, stream);
     return cudaGetLastError();
 }

@@ -155,17 +155,17 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
 // Built-in scratch for fa_bwd_noalloc: the D values of one backward call.  In
 // host code the symbol is only a host-side stand-in; kernels get the device
 // address looked up once per device below.
-static __device__ __align__(256) float g_noalloc_scratch[FA_NOALLOC_MAX_ROWS];
+static __device__ __align__(256) float2 g_noalloc_scratch[FA_NOALLOC_MAX_ROWS];
 
 struct NoAllocState {
     bool ready = false;
-    float* scratch = nullptr;   // device address of g_noalloc_scratch on this device
+    float2* scratch = nullptr;  // device address of g_noalloc_scratch on this device
 };
 NoAllocState g_noalloc[kMaxDevices];
 
 // One-time, per-device lookup of the scratch array's device address (with
 // that device current).
-int noalloc_setup(float** out) {
+int noalloc_setup(float2** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_mutex);
@@ -174,7 +174,7 @@ int noalloc_setup(float** out) {
         void* ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr)
             return FA_ERR_CUDA;
-        st.scratch = static_cast<float*>(ptr);
+        st.scratch = static_cast<float2*>(ptr);
         st.ready = true;
     }
     *out = st.scratch;
@@ -226,10 +226,10 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d, int varlen_total) {
     (void)d;
-    if (H <= 0) return 0;
-    const int64_t rows = varlen_total > 0 ? varlen_total
-                                          : (B > 0 && N > 0 ? static_cast<int64_t>(B) * N : 0);
-    return fa::bwd_workspace_bytes(rows, H);
+    if (H <= 0 || B <= 0) return 0;
+    const bool packed = varlen_total > 0;
+    if (!packed && N <= 0) return 0;
+    return fa::bwd_workspace_bytes(B, H, fa::bwd_stats_stride(B, N, varlen_total, packed), packed);
 }
 
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -244,7 +244,9 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
         misaligned(dO) || misaligned(dq) || misaligned(dk) || misaligned(dv))
         return FA_ERR_MISALIGNED;
     if (B == 0 || c.rows == 0) return FA_OK;
-    const size_t need = fa::bwd_workspace_bytes(c.rows, H);
+    const bool packed = cu_seqlens != nullptr;
+    const int64_t stride = fa::bwd_stats_stride(B, N, c.rows, packed);
+    const size_t need = fa::bwd_workspace_bytes(B, H, stride, packed);
     if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
     if (misaligned(workspace)) return FA_ERR_MISALIGNED;
     DeviceState* st = nullptr;
@@ -259,16 +261,15 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
     a.dq = dq;
     a.dk = dk;
     a.dv = dv;
-    a.dsum = static_cast<float*>(workspace);
+    a.stats = static_cast<float2*>(workspace);
+    a.stats_stride = stride;
     a.scale = scale;
     a.num_sms = st->num_sms;
     a.error_word = st->error_word;
     a.timeout_ns = g_fault_timeout_ns ? g_fault_timeout_ns : kDefaultTimeoutNs;
     fa::BwdMaps m;
-    if (make_map(&m.q64, q, c.rows, H, d, 64) || make_map(&m.do64, dO, c.rows, H, d, 64) ||
-        make_map(&m.k128, k, c.rows, H, d, 128) || make_map(&m.v128, v, c.rows, H, d, 128) ||
-        make_map(&m.q128, q, c.rows, H, d, 128) || make_map(&m.do128, dO, c.rows, H, d, 128) ||
-        make_map(&m.k64, k, c.rows, H, d, 64) || make_map(&m.v64, v, c.rows, H, d, 64))
+    if (make_map(&m.q, q, c.rows, H, d, 128) || make_map(&m.k, k, c.rows, H, d, 128) ||
+        make_map(&m.v, v, c.rows, H, d, 128) || make_map(&m.dO, dO, c.rows, H, d, 128))
         return FA_ERR_CUDA;
     fa::BwdHooks hooks{prof_start, prof_stop};
     return fa::bwd_launch(a, m, stream, hooks) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -286,10 +287,13 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
         misaligned(dO) || misaligned(dq) || misaligned(dk) || misaligned(dv))
         return FA_ERR_MISALIGNED;
     if (B == 0 || c.rows == 0) return FA_OK;
-    if (c.rows * H > static_cast<int64_t>(FA_NOALLOC_MAX_ROWS)) return FA_ERR_SCRATCH_LIMIT;
+    const bool packed = cu_seqlens != nullptr;
+    const int64_t stride = fa::bwd_stats_stride(B, N, c.rows, packed);
+    if (fa::bwd_workspace_bytes(B, H, stride, packed) > sizeof(float2) * FA_NOALLOC_MAX_ROWS)
+        return FA_ERR_SCRATCH_LIMIT;
     DeviceState* st = nullptr;
     if ((rc = device_setup(&st)) != FA_OK) return rc;
-    float* scratch = nullptr;
+    float2* scratch = nullptr;
     if ((rc = noalloc_setup(&scratch)) != FA_OK) return rc;
 
     fa::BwdArgs a;
@@ -301,16 +305,15 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
     a.dq = dq;
     a.dk = dk;
     a.dv = dv;
-    a.dsum = scratch;     // every element the kernels read is written first by the D pre-pass
+    a.stats = scratch;    // every entry the kernels use is written first by the pre-pass
+    a.stats_stride = stride;
     a.scale = scale;
     a.num_sms = st->num_sms;
     a.error_word = st->error_word;
     a.timeout_ns = g_fault_timeout_ns ? g_fault_timeout_ns : kDefaultTimeoutNs;
     fa::BwdMaps m;
-    if (make_map(&m.q64, q, c.rows, H, d, 64) || make_map(&m.do64, dO, c.rows, H, d, 64) ||
-        make_map(&m.k128, k, c.rows, H, d, 128) || make_map(&m.v128, v, c.rows, H, d, 128) ||
-        make_map(&m.q128, q, c.rows, H, d, 128) || make_map(&m.do128, dO, c.rows, H, d, 128) ||
-        make_map(&m.k64, k, c.rows, H, d, 64) || make_map(&m.v64, v, c.rows, H, d, 64))
+    if (make_map(&m.q, q, c.rows, H, d, 128) || make_map(&m.k, k, c.rows, H, d, 128) ||
+        make_map(&m.v, v, c.rows, H, d, 128) || make_map(&m.dO, dO, c.rows, H, d, 128))
         return FA_ERR_CUDA;
     fa::BwdHooks hooks{prof_start, prof_stop};
     return fa::bwd_launch(a, m, stream, hooks) == cudaSuccess ? FA_OK : FA_ERR_CUDA;

@@ -79,8 +79,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
            const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
     using C = FwdCfg<D>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                               ~static_cast<uintptr_t>(1023));
+    uint8_t* smem = align_smem_1024(smem_raw);
     uint8_t* sQ = smem + C::OFF_Q;
     uint8_t* sKV = smem + C::OFF_KV;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);

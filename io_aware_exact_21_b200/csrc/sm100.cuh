@@ -28,6 +28,16 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
+// First 1024-byte aligned byte of the dynamic shared memory (swizzled TMA
+// tiles need 1024-byte alignment).  Offsetting the __shared__ array itself,
+// rather than rebuilding a pointer from an integer, keeps the shared address
+// space visible to the compiler, so accesses through it stay shared-memory
+// instructions instead of generic ones.
+__device__ __forceinline__ uint8_t* align_smem_1024(uint8_t* smem_raw) {
+    const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    return smem_raw + pad;
+}
+
 // --------------------------------------------------------------- mbarrier --
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
@@ -102,6 +112,18 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
         " [%0], [%1, {%3, %4, %5}], [%2];"
         ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)),
           "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+// Contiguous global -> shared copy of `bytes` (multiple of 16, both
+// addresses 16-byte aligned), completion on `bar` through its transaction
+// count.  No multicast.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes,
+                                          uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes),
+          "r"(smem_u32(bar))
         : "memory");
 }
 

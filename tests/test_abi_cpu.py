@@ -91,10 +91,13 @@ def test_empty_problems_are_noops():
 
 
 def test_workspace_size():
-    # one fp32 D value per (head, token row), rounded up to 256 bytes
-    assert fa.fa_bwd_workspace_size(2, 16, 4096, 128, 0) == 2 * 16 * 4096 * 4
-    assert fa.fa_bwd_workspace_size(16, 32, 0, 128, 1000) == (32 * 1000 * 4 + 255) // 256 * 256
-    assert fa.fa_bwd_workspace_size(1, 1, 1, 64, 0) == 256
+    # 8 bytes per (head, row), each sequence padded to 128 rows
+    assert fa.fa_bwd_workspace_size(2, 16, 4096, 128, 0) == 2 * 16 * 4096 * 8
+    assert fa.fa_bwd_workspace_size(2, 16, 4000, 128, 0) == 2 * 16 * 4096 * 8
+    # packed: H * roundup(T + 127 B, 128) * 8
+    assert fa.fa_bwd_workspace_size(16, 32, 0, 128, 1000) == 32 * 3072 * 8
+    assert fa.fa_bwd_workspace_size(1, 1, 1, 64, 0) == 128 * 8
+    assert fa.fa_bwd_workspace_size(0, 1, 1, 64, 0) == 0
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
@@ -115,8 +118,9 @@ def test_noalloc_validation_on_host():
     assert call(d=80) == -2
     assert call(window=4) == -5
     assert call(dv=P + 8) == -4
-    # H * rows above the built-in scratch (FA_NOALLOC_MAX_ROWS) is rejected
+    # a workspace above the built-in scratch (8 * FA_NOALLOC_MAX_ROWS bytes) is rejected
     assert call(H=16, N=binding.NOALLOC_MAX_ROWS // 16 + 1) == -10
+    assert call(H=16, N=binding.NOALLOC_MAX_ROWS // 16) == -7 or torch.cuda.is_available()
     assert call(B=0) == 0
     header = open(HEADER).read()
     assert "#define FA_NOALLOC_MAX_ROWS (1 << 20)" in header
