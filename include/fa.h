@@ -30,7 +30,7 @@
  *   N is the sequence length for fixed-length inputs; for packed inputs N is
  *   the number of token rows T the buffers hold (the per-sequence lengths are
  *   read from cu_seqlens on the device, so no host synchronisation is needed).
- *   Packed batches hold at most 4096 sequences.
+ *   Packed batches hold at most 2048 sequences.
  *
  * Masks (row i, key j local to a sequence of n tokens; query and key sequences
  * have the same length):

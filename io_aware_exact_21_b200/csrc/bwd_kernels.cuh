@@ -88,12 +88,13 @@ stats_kernel(const __nv_bfloat16* __restrict__ dO, const __nv_bfloat16* __restri
     constexpr int LPR = D / 8;                 // lanes per row (16-byte vectors)
     constexpr int RPW = 32 / LPR;              // rows per warp per iteration
     extern __shared__ int pre_smem[];
-    int* prefix = pre_smem;                    // B + 1 (packed only)
-    int* cu = pre_smem + kMaxVarlenSeqs + 1;   // B + 1
-    int* scratch = cu + kMaxVarlenSeqs + 1;    // blockDim
+    int* prefix = pre_smem;                    // B + 1 block prefix (packed only)
+    int* uprefix = prefix + kMaxVarlenSeqs + 1;
+    int* cu = uprefix + kMaxVarlenSeqs + 1;    // B + 1
+    int* scratch = cu + kMaxVarlenSeqs + 1;    // 2 * blockDim
     if (g.cu_seqlens) {
         for (int i = threadIdx.x; i <= g.B; i += blockDim.x) cu[i] = g.cu_seqlens[i];
-        build_schedule_prefix(g, 128, prefix, scratch);   // __syncthreads inside
+        build_schedule_prefix(g, 128, prefix, uprefix, scratch);   // __syncthreads inside
     }
     const int lane = threadIdx.x & 31;
     const int sub = lane / LPR;
@@ -164,8 +165,8 @@ struct BwdCfg {
     static constexpr int NBAR = 2 + 2 * NSTAGE + 4 + 2 + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int OFF_SCRATCH = OFF_MISC + 16;
-    static constexpr int OFF_PREFIX = OFF_SCRATCH + THREADS * 4;
-    static constexpr int SMEM_BYTES = OFF_PREFIX + (kMaxVarlenSeqs + 1) * 4 + 1024;
+    static constexpr int OFF_PREFIX = OFF_SCRATCH + 2 * THREADS * 4;   // block and unit prefixes
+    static constexpr int SMEM_BYTES = OFF_PREFIX + 2 * (kMaxVarlenSeqs + 1) * 4 + 1024;
 };
 
 // Query-tile range [ib, ie) (tiles of BS rows) whose rows can see some key of
@@ -301,7 +302,7 @@ __device__ __forceinline__ void arrive_warp(uint64_t* bar) {
 template <int D>
 __device__ __forceinline__ uint32_t bwd_prologue(uint8_t* smem, const BwdBarriers& br,
                                                  volatile int* abort_flag, const BwdParams& p,
-                                                 Schedule& sch, int heavy_first,
+                                                 Schedule& sch,
                                                  const CUtensorMap* maps[4]) {
     using C = BwdCfg<D>;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
@@ -317,9 +318,10 @@ __device__ __forceinline__ uint32_t bwd_prologue(uint8_t* smem, const BwdBarrier
     }
     sch.g = p.g;
     sch.rows_per_item = C::BM;
-    sch.heavy_first = heavy_first;
-    sch.prefix = prefix;
-    sch.total_items = build_schedule_prefix(p.g, C::BM, prefix, scratch);   // __syncthreads inside
+    sch.bprefix = prefix;
+    sch.uprefix = prefix + kMaxVarlenSeqs + 1;
+    sch.total_units = build_schedule_prefix(p.g, C::BM, prefix, prefix + kMaxVarlenSeqs + 1,
+                                            scratch);   // __syncthreads inside
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -350,8 +352,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
     float2* vec = reinterpret_cast<float2*>(smem + C::OFF_VEC);
     const CUtensorMap* maps[4] = {&tm_k, &tm_v, &tm_q, &tm_do};
     Schedule sch;
-    // under a causal mask the first key block sees the most queries: natural order
-    const uint32_t tmem = bwd_prologue<D>(smem, br, abort_flag, p, sch, 0, maps);
+    const uint32_t tmem = bwd_prologue<D>(smem, br, abort_flag, p, sch, maps);
     const int warp = threadIdx.x >> 5;
     const int lane = lane_id();
     const WaitCtl wc{abort_flag, p.error_word, p.timeout_ns};
@@ -363,9 +364,9 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             // ---------------------------------- producer (whole warp) --
             uint32_t cnt = 0, item_it = 0, fix_issued = 0;
             bool ok = true;
-            for (int w = blockIdx.x; w < sch.total_items && ok; w += gridDim.x, ++item_it) {
-                int s, h, blk;
-                sch.item(w, s, h, blk);
+            ItemIter it;
+            int s, h, blk;
+            for (; ok && it.next(sch, s, h, blk); ++item_it) {
                 const SeqSpan sp = sch.span(s);
                 const int n = sp.len;
                 const int k0 = blk * C::BM;
@@ -385,7 +386,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                     }
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
-                const int blocks_before = p.g.cu_seqlens ? sch.prefix[s] : 0;
+                const int blocks_before = sch.blocks_before(s);
                 for (int i = ib; i < ie && ok; ++i, ++cnt) {
                     const int slot = cnt % C::NSTAGE;
                     if (lane == 0) {
@@ -424,9 +425,9 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             const uint32_t st_addr = smem_u32(smem + C::OFF_ST);
             uint32_t cnt = 0, item_it = 0;
             bool ok = true;
-            for (int w = blockIdx.x; w < sch.total_items && ok; w += gridDim.x, ++item_it) {
-                int s, h, blk;
-                sch.item(w, s, h, blk);
+            ItemIter it;
+            int s, h, blk;
+            for (; ok && it.next(sch, s, h, blk); ++item_it) {
                 const SeqSpan sp = sch.span(s);
                 const int n = sp.len;
                 const int k0 = blk * C::BM;
@@ -494,9 +495,9 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
         const uint32_t tP = tmem + lane_base + C::COL_DP + 64 * g;
         uint32_t cnt = 0, item_it = 0;
         bool ok = true;
-        for (int w = blockIdx.x; w < sch.total_items && ok; w += gridDim.x, ++item_it) {
-            int s, h, blk;
-            sch.item(w, s, h, blk);
+        ItemIter it;
+        int s, h, blk;
+        for (; ok && it.next(sch, s, h, blk); ++item_it) {
             const SeqSpan sp = sch.span(s);
             const int n = sp.len;
             const int k0 = blk * C::BM;
@@ -602,8 +603,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
     const CUtensorMap* maps[4] = {&tm_q, &tm_do, &tm_k, &tm_v};
     Schedule sch;
-    // the last query block sees the most keys under a causal mask
-    const uint32_t tmem = bwd_prologue<D>(smem, br, abort_flag, p, sch, p.g.causal, maps);
+    const uint32_t tmem = bwd_prologue<D>(smem, br, abort_flag, p, sch, maps);
     const int warp = threadIdx.x >> 5;
     const int lane = lane_id();
     const WaitCtl wc{abort_flag, p.error_word, p.timeout_ns};
@@ -615,9 +615,9 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             // -------------------------------------------------- producer --
             uint32_t cnt = 0, item_it = 0, fix_issued = 0;
             bool ok = true;
-            for (int w = blockIdx.x; w < sch.total_items && ok; w += gridDim.x, ++item_it) {
-                int s, h, blk;
-                sch.item(w, s, h, blk);
+            ItemIter it;
+            int s, h, blk;
+            for (; ok && it.next(sch, s, h, blk); ++item_it) {
                 const SeqSpan sp = sch.span(s);
                 const int n = sp.len;
                 const int q0 = blk * C::BM;
@@ -662,9 +662,9 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             const uint32_t st_addr = smem_u32(smem + C::OFF_ST);
             uint32_t cnt = 0, item_it = 0;
             bool ok = true;
-            for (int w = blockIdx.x; w < sch.total_items && ok; w += gridDim.x, ++item_it) {
-                int s, h, blk;
-                sch.item(w, s, h, blk);
+            ItemIter it;
+            int s, h, blk;
+            for (; ok && it.next(sch, s, h, blk); ++item_it) {
                 const SeqSpan sp = sch.span(s);
                 const int n = sp.len;
                 const int q0 = blk * C::BM;
@@ -730,9 +730,9 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         const uint32_t tP = tmem + lane_base + C::COL_DP + 64 * g;
         uint32_t cnt = 0, item_it = 0;
         bool ok = true;
-        for (int w = blockIdx.x; w < sch.total_items && ok; w += gridDim.x, ++item_it) {
-            int s, h, blk;
-            sch.item(w, s, h, blk);
+        ItemIter it;
+        int s, h, blk;
+        for (; ok && it.next(sch, s, h, blk); ++item_it) {
             const SeqSpan sp = sch.span(s);
             const int n = sp.len;
             const int q0 = blk * C::BM;
@@ -742,7 +742,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             float nl = -INFINITY, dq_d = 0.f;
             if (q < n) {
                 const float2 st = p.stats[stats_index(p.g, p.stats_stride, s, h,
-                                                      p.g.cu_seqlens ? sch.prefix[s] : 0, q)];
+                                                      sch.blocks_before(s), q)];
                 nl = st.x;
                 dq_d = st.y;
             }
@@ -833,7 +833,7 @@ inline size_t bwd_workspace_bytes(int B, int H, int64_t stride, bool packed) {
     return static_cast<size_t>((entries * 8 + 255) / 256 * 256);
 }
 
-constexpr int kStatsSmem = (2 * (kMaxVarlenSeqs + 1) + 256) * 4;
+constexpr int kStatsSmem = (3 * (kMaxVarlenSeqs + 1) + 2 * 256) * 4;
 
 inline cudaError_t bwd_set_smem_limits() {
     cudaError_t e;

@@ -69,8 +69,8 @@ struct FwdCfg {
     static constexpr int NBAR = 2 + 2 * NSLOT + 6 + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int OFF_SCRATCH = OFF_MISC + 16;
-    static constexpr int OFF_PREFIX = OFF_SCRATCH + THREADS * 4;
-    static constexpr int SMEM_BYTES = OFF_PREFIX + (kMaxVarlenSeqs + 1) * 4 + 1024;
+    static constexpr int OFF_PREFIX = OFF_SCRATCH + 2 * THREADS * 4;   // block and unit prefixes
+    static constexpr int SMEM_BYTES = OFF_PREFIX + 2 * (kMaxVarlenSeqs + 1) * 4 + 1024;
 };
 
 template <int D>
@@ -127,9 +127,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     Schedule sch;
     sch.g = p.g;
     sch.rows_per_item = C::ROWS;
-    sch.heavy_first = p.g.causal;
-    sch.prefix = prefix;
-    sch.total_items = build_schedule_prefix(p.g, C::ROWS, prefix, scratch);  // has __syncthreads
+    sch.bprefix = prefix;
+    sch.uprefix = prefix + kMaxVarlenSeqs + 1;
+    sch.total_units = build_schedule_prefix(p.g, C::ROWS, prefix, prefix + kMaxVarlenSeqs + 1,
+                                            scratch);  // has __syncthreads
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -146,9 +147,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             bool ok = true;
             bool skipped = false;
             uint32_t skipped_at = 0xffffffffu;
-            for (int w = blockIdx.x; w < sch.total_items && ok; w += gridDim.x, ++item_it) {
-                int s, h, blk;
-                sch.item(w, s, h, blk);
+            ItemIter it;
+            int s, h, blk;
+            for (; ok && it.next(sch, s, h, blk); ++item_it) {
                 const SeqSpan sp = sch.span(s);
                 const int r_lo = blk * C::ROWS;
                 const int r_hi = min(sp.len, r_lo + C::ROWS);
@@ -221,9 +222,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                             IDESC_O, (accumulate | kk) != 0);
                 }
             };
-            for (int w = blockIdx.x; w < sch.total_items && ok; w += gridDim.x, ++item_it) {
-                int s, h, blk;
-                sch.item(w, s, h, blk);
+            ItemIter it;
+            int s, h, blk;
+            for (; ok && it.next(sch, s, h, blk); ++item_it) {
                 const SeqSpan sp = sch.span(s);
                 const int r_lo = blk * C::ROWS;
                 const int r_hi = min(sp.len, r_lo + C::ROWS);
@@ -295,9 +296,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         const float sl2 = p.scale_log2;
         uint32_t step = 0, item_it = 0;
         bool ok = true;
-        for (int w = blockIdx.x; w < sch.total_items && ok; w += gridDim.x, ++item_it) {
-            int s, h, blk;
-            sch.item(w, s, h, blk);
+        ItemIter it;
+        int s, h, blk;
+        for (; ok && it.next(sch, s, h, blk); ++item_it) {
             const SeqSpan sp = sch.span(s);
             const int n = sp.len;
             const int r_lo = blk * C::ROWS;
@@ -313,14 +314,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 tc_fence_after();
                 float sv[C::BN];
                 {
-                    uint32_t r[32];
+                    uint32_t r[C::BN];
 #pragma unroll
-                    for (int c = 0; c < C::BN / 32; ++c) {
-                        tmem_ld32(tS + c * 32, r);
-                        tmem_wait_ld();
+                    for (int c = 0; c < C::BN / 32; ++c)
+                        tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(r[e]);
-                    }
+                    for (int e = 0; e < C::BN; ++e) sv[e] = __uint_as_float(r[e]);
                 }
                 const int k0 = j * C::BN;
                 if (tile_needs_mask(r0, C::BM, k0, C::BN, n, p.g.causal, p.g.window)) {
@@ -328,9 +328,20 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     for (int c = 0; c < C::BN; ++c)
                         if (!key_allowed(i, k0 + c, n, p.g.causal, p.g.window)) sv[c] = -INFINITY;
                 }
-                float mx = sv[0];
+                // row maximum as a tree (the max is exact in any order), so the
+                // 127 compares are not one dependent chain
+                float mx;
+                {
+                    float m8[8];
 #pragma unroll
-                for (int c = 1; c < C::BN; ++c) mx = fmaxf(mx, sv[c]);
+                    for (int e = 0; e < 8; ++e) m8[e] = sv[e];
+#pragma unroll
+                    for (int c = 8; c < C::BN; c += 8)
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) m8[e] = fmaxf(m8[e], sv[c + e]);
+                    mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+                }
                 const float m_new = fmaxf(m_ref, mx * sl2);
                 const bool resc = m_new > m_ref + kRescaleLog2;
                 float alpha = 1.f;

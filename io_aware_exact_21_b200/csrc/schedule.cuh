@@ -14,7 +14,7 @@
 
 namespace fa {
 
-constexpr int kMaxVarlenSeqs = 4096;   // sequences a packed batch may hold
+constexpr int kMaxVarlenSeqs = 2048;   // sequences a packed batch may hold
 
 struct Geometry {
     int B;                  // sequences
@@ -59,17 +59,19 @@ __device__ __forceinline__ bool tile_needs_mask(int r0, int BM, int k0, int BN, 
     return false;
 }
 
-// Static persistent schedule.  Work items are (sequence, head, block of
-// `rows_per_item` rows); item w goes to CTA w % gridDim.x.  Items are ordered
-// sequence-major, then head, then block, so the CTAs running at the same time
-// share K/V of few heads in L2; with `heavy_first` the blocks of a head are
-// visited from the last (most keys under a causal mask) to the first.
+// Static persistent schedule.  The rows of a (sequence, head) are cut into
+// blocks of `rows_per_item` rows; a work unit is the pair of blocks p and
+// nb-1-p of one (sequence, head) (the middle block alone when nb is odd), so
+// that under a causal mask -- where a block's cost grows or shrinks linearly
+// with its index -- every unit costs the same.  Units are ordered sequence-
+// major, then head, then p, so the CTAs running at the same time share K/V of
+// few heads in L2; unit w goes to CTA w % gridDim.x.
 struct Schedule {
     Geometry g;
     int rows_per_item;
-    int heavy_first;
-    const int* prefix;      // shared memory: prefix[s] = sum of blocks of sequences < s
-    int total_items;
+    const int* bprefix;     // shared memory: blocks of the sequences before s (packed only)
+    const int* uprefix;     // shared memory: units of the sequences before s (packed only)
+    int total_units;
 
     __device__ __forceinline__ int blocks_of(int len) const {
         return (len + rows_per_item - 1) / rows_per_item;
@@ -83,60 +85,106 @@ struct Schedule {
         return SeqSpan{s * g.N, g.N};
     }
 
-    // Decode item w into (sequence, head, block).
-    __device__ __forceinline__ void item(int w, int& s, int& h, int& blk) const {
-        int nb;
-        int local;
+    // Blocks of the sequences before s (packed batches; 0 for fixed length).
+    __device__ __forceinline__ int blocks_before(int s) const {
+        return g.cu_seqlens ? bprefix[s] : 0;
+    }
+
+    // Decode unit w into (sequence, head, first block p, blocks of the sequence nb).
+    __device__ __forceinline__ void unit(int w, int& s, int& h, int& p, int& nb) const {
+        int nu, local;
         if (!g.cu_seqlens) {
             nb = blocks_of(g.N);
-            s = w / (g.H * nb);
-            local = w - s * g.H * nb;
+            nu = (nb + 1) >> 1;
+            s = w / (g.H * nu);
+            local = w - s * g.H * nu;
         } else {
-            // binary search: largest s with prefix[s] * H <= w
+            // binary search: largest s with uprefix[s] * H <= w
             int lo = 0, hi = g.B - 1;
             while (lo < hi) {
                 int mid = (lo + hi + 1) >> 1;
-                if (prefix[mid] * g.H <= w) lo = mid; else hi = mid - 1;
+                if (uprefix[mid] * g.H <= w) lo = mid; else hi = mid - 1;
             }
             s = lo;
-            nb = prefix[s + 1] - prefix[s];
-            local = w - prefix[s] * g.H;
+            nu = uprefix[s + 1] - uprefix[s];
+            nb = bprefix[s + 1] - bprefix[s];
+            local = w - uprefix[s] * g.H;
         }
-        h = local / nb;
-        blk = local - h * nb;
-        if (heavy_first) blk = nb - 1 - blk;
+        h = local / nu;
+        p = local - h * nu;
     }
 };
 
-// Build the per-sequence block prefix in shared memory (packed batches only)
-// and return the number of work items.  All threads of the CTA call it.
+// Walks the blocks one CTA processes: its units in order, both blocks of each.
+struct ItemIter {
+    int w;
+    int half;
+    __device__ __forceinline__ ItemIter() : w(blockIdx.x), half(0) {}
+    __device__ __forceinline__ bool next(const Schedule& sch, int& s, int& h, int& blk) {
+        while (w < sch.total_units) {
+            int p, nb;
+            sch.unit(w, s, h, p, nb);
+            if (half == 0) {
+                half = 1;
+                blk = p;
+                return true;
+            }
+            half = 0;
+            w += gridDim.x;
+            if (nb - 1 - p != p) {
+                blk = nb - 1 - p;
+                return true;
+            }
+        }
+        return false;
+    }
+};
+
+// Build the per-sequence block and unit prefixes in shared memory (packed
+// batches only) and return the number of work units.  All threads of the CTA
+// call it.
 __device__ __forceinline__ int build_schedule_prefix(const Geometry& g, int rows_per_item,
-                                                     int* prefix, int* scratch /* blockDim */) {
+                                                     int* bprefix, int* uprefix,
+                                                     int* scratch /* 2 * blockDim */) {
     if (!g.cu_seqlens) {
-        int nb = (g.N + rows_per_item - 1) / rows_per_item;
-        return g.B * g.H * nb;
+        const int nb = (g.N + rows_per_item - 1) / rows_per_item;
+        return g.B * g.H * ((nb + 1) >> 1);
     }
     const int tid = threadIdx.x, nt = blockDim.x;
     const int per = (g.B + nt - 1) / nt;
     const int s0 = min(g.B, tid * per), s1 = min(g.B, s0 + per);
-    int run = 0;
+    int runb = 0, runu = 0;
     for (int s = s0; s < s1; ++s) {
-        int len = g.cu_seqlens[s + 1] - g.cu_seqlens[s];
-        run += (len + rows_per_item - 1) / rows_per_item;
-        prefix[s + 1] = run;          // local inclusive prefix for now
+        const int len = g.cu_seqlens[s + 1] - g.cu_seqlens[s];
+        const int nb = (len + rows_per_item - 1) / rows_per_item;
+        runb += nb;
+        runu += (nb + 1) >> 1;
+        bprefix[s + 1] = runb;          // local inclusive prefixes for now
+        uprefix[s + 1] = runu;
     }
-    scratch[tid] = run;
+    scratch[tid] = runb;
+    scratch[nt + tid] = runu;
     __syncthreads();
     if (tid == 0) {
-        int acc = 0;
-        for (int t = 0; t < nt; ++t) { int v = scratch[t]; scratch[t] = acc; acc += v; }
-        prefix[0] = 0;
+        int ab = 0, au = 0;
+        for (int t = 0; t < nt; ++t) {
+            const int vb = scratch[t], vu = scratch[nt + t];
+            scratch[t] = ab;
+            scratch[nt + t] = au;
+            ab += vb;
+            au += vu;
+        }
+        bprefix[0] = 0;
+        uprefix[0] = 0;
     }
     __syncthreads();
-    const int off = scratch[tid];
-    for (int s = s0; s < s1; ++s) prefix[s + 1] += off;
+    const int ob = scratch[tid], ou = scratch[nt + tid];
+    for (int s = s0; s < s1; ++s) {
+        bprefix[s + 1] += ob;
+        uprefix[s + 1] += ou;
+    }
     __syncthreads();
-    return prefix[g.B] * g.H;
+    return uprefix[g.B] * g.H;
 }
 
 }  // namespace fa
