@@ -37,6 +37,42 @@ UNIT = "TFLOP/s"
 WORKLOAD = dict(B=4, H=16, N=8192, d=128, causal=False, window=0, seed=2)
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
+# one ncu capture of the B=2 H=16 N=8192 d=128 non-causal case, scaled by 2 to
+# the B=4 workload (each kernel's traffic grows with the number of heads it
+# processes).  Valid only for the kernel sources it was taken on: the entry
+# carries a hash of them and is reported as null once they change.
+# Summaries and commands: profiles/*_kernel_B2H16N8192d128.md.
+TRAFFIC = {
+    "fwd": {"bytes_per_launch": 2 * (207.27e6 + 50.36e6), "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh"),
+            "sha": "f46501df6dc6d3e3"},
+    "dkdv": {"bytes_per_launch": 2 * (273.03e6 + 107.20e6),
+             "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "5fe302c77f19a617"},
+    "dq": {"bytes_per_launch": 2 * (271.28e6 + 52.17e6),
+           "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "5fe302c77f19a617"},
+}
+
+
+def traffic_for(kernel):
+    """ncu traffic per launch if the kernel's sources still match the capture."""
+    import hashlib
+    t = TRAFFIC.get(kernel)
+    if not t:
+        return None
+    h = hashlib.sha256()
+    try:
+        for f in t["sources"]:
+            with open(os.path.join(ROOT, "io_aware_exact_21_b200", "csrc", f), "rb") as fh:
+                h.update(fh.read())
+    except OSError:
+        return None
+    if h.hexdigest()[:16] != t["sha"]:
+        return None
+    w = WORKLOAD
+    if (w["B"], w["H"], w["N"], w["d"], w["causal"]) != (4, 16, 8192, 128, False):
+        return None
+    return t["bytes_per_launch"]
+
 
 def flops(B, H, N, d, causal):
     f = 4.0 * B * H * N * N * d
@@ -263,7 +299,8 @@ def run_ours(args, rank, world, device):
                      "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4) if achieved else None,
                      "peak_source": "%s %s" % (peak_src, peak_key),
-                     "traffic": None},
+                     "traffic": traffic_for(dom),
+                     "traffic_unit": "bytes per launch (ncu dram read + write)"},
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": sum(c for (_, c) in prof.values()),
