@@ -323,7 +323,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     for (int e = 0; e < C::BN; ++e) sv[e] = __uint_as_float(r[e]);
                 }
                 const int k0 = j * C::BN;
-                if (tile_needs_mask(r0, C::BM, k0, C::BN, n, p.g.causal, p.g.window)) {
+                const bool masked = tile_needs_mask(r0, C::BM, k0, C::BN, n, p.g.causal, p.g.window);
+                if (masked) {
 #pragma unroll
                     for (int c = 0; c < C::BN; ++c)
                         if (!key_allowed(i, k0 + c, n, p.g.causal, p.g.window)) sv[c] = -INFINITY;
@@ -352,6 +353,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 }
                 const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
                 float lsum = 0.f;
+                // masked keys hold -inf: ex2 returns exactly 0 for them
 #pragma unroll
                 for (int c = 0; c < C::BN / 32; ++c) {
                     uint32_t pk[16];

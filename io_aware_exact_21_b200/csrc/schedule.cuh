@@ -49,13 +49,16 @@ __device__ __forceinline__ void key_tile_range(int r_lo, int r_hi, int n, int ca
     if (je < jb) je = jb;
 }
 
-// True when some pair of (rows [r0, r0+BM), keys [k0, k0+BN)) is masked out,
-// so the tile needs the element-wise mask.
+// True when some pair of (rows [r0, r0+BM) inside the sequence, keys
+// [k0, k0+BN)) is masked out, so the tile needs the element-wise mask.  Rows
+// past the sequence end are not considered: their results are never stored,
+// and ignoring them makes the decision depend only on the mask's meaning (a
+// window of n or more keys classifies every tile exactly like plain causal).
 __device__ __forceinline__ bool tile_needs_mask(int r0, int BM, int k0, int BN, int n, int causal,
                                                 int window) {
     if (k0 + BN > n) return true;
     if (causal && k0 + BN - 1 > r0) return true;
-    if (window > 0 && k0 <= r0 + BM - 1 - window) return true;
+    if (window > 0 && k0 <= min(r0 + BM, n) - 1 - window) return true;
     return false;
 }
 
