@@ -28,7 +28,8 @@
 //   warps 4-7     softmax + correction + epilogue of tile 0 (one thread per row)
 //   warps 8-11    the same for tile 1
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [384,384+D).
-// P_t is written as packed bf16 over the first 64 columns of S_t.
+// P_t is written as packed bf16 over the first 64 columns of S_t, in two
+// halves of 64 keys that are released to the MMA warp one at a time.
 // The MMA thread issues S_t(j+1) right after O_t += P_t(j) V_j, so while one
 // softmax warpgroup works on its tile the tensor core runs the other's GEMMs.
 #pragma once
@@ -66,7 +67,7 @@ struct FwdCfg {
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_KV = OFF_Q + 2 * TILE_BYTES;
     static constexpr int OFF_BAR = OFF_KV + NSLOT * TILE_BYTES;
-    static constexpr int NBAR = 2 + 2 * NSLOT + 6 + 1;
+    static constexpr int NBAR = 2 + 2 * NSLOT + 8 + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int OFF_SCRATCH = OFF_MISC + 16;
     static constexpr int OFF_PREFIX = OFF_SCRATCH + 2 * THREADS * 4;   // block and unit prefixes
@@ -88,8 +89,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     uint64_t* slot_full = bars + 2;
     uint64_t* slot_empty = bars + 2 + C::NSLOT;
     uint64_t* s_full = bars + 2 + 2 * C::NSLOT;     // [2]
-    uint64_t* p_full = s_full + 2;                  // [2]
-    uint64_t* o_final = p_full + 2;                 // [2]
+    uint64_t* p_full = s_full + 2;                  // [2 tiles x 2 halves]
+    uint64_t* o_final = p_full + 4;                 // [2]
     uint64_t* drain = o_final + 2;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
@@ -108,7 +109,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(s_full + t, 1);
-            mbar_init(p_full + t, 4);     // one arrival per softmax warp
+            mbar_init(p_full + 2 * t, 4);       // one arrival per softmax warp, per half
+            mbar_init(p_full + 2 * t + 1, 4);
             mbar_init(o_final + t, 1);
         }
         mbar_init(drain, 1);
@@ -212,12 +214,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                             IDESC_S, kk > 0);
                 }
             };
-            auto issue_pv = [&](int t, uint32_t vslot, uint32_t accumulate) {
+            // O_t (+)= P_t[:, keys of half] V_j[keys of half, :]  (half = 64 keys)
+            auto issue_pv = [&](int t, uint32_t vslot, uint32_t accumulate, int half) {
                 const uint32_t d_tmem = tmem + (t ? C::COL_O1 : C::COL_O0);
                 const uint32_t a_tmem = tmem + (t ? C::COL_S1 : C::COL_S0);
                 const uint32_t b0 = kv_addr + vslot * C::TILE_BYTES;
 #pragma unroll
-                for (int kk = 0; kk < C::BN / 16; ++kk) {
+                for (int k = 0; k < C::BN / 32; ++k) {
+                    const int kk = half * (C::BN / 32) + k;
                     umma_ts(d_tmem, a_tmem + kk * 8, sw128_desc(b0 + kk * 2048, C::BOX_BYTES, 1024),
                             IDESC_O, (accumulate | kk) != 0);
                 }
@@ -248,7 +252,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     if (!mbar_wait(slot_full + vslot, (cnt / C::NSLOT) & 1, wc)) { ok = false; break; }
                     if (!mbar_wait(p_full + 0, step & 1, wc)) { ok = false; break; }
                     tc_fence_after();
-                    issue_pv(0, vslot, j > jb);
+                    issue_pv(0, vslot, j > jb, 0);
+                    if (!mbar_wait(p_full + 1, step & 1, wc)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_pv(0, vslot, 1, 1);
                     if (last) umma_commit(o_final + 0);
                     if (!last) {
                         if (!mbar_wait(slot_full + kslot_n, ((cnt + 1) / C::NSLOT) & 1, wc)) {
@@ -259,9 +266,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                         issue_s(0, kslot_n);
                         umma_commit(s_full + 0);
                     }
-                    if (!mbar_wait(p_full + 1, step & 1, wc)) { ok = false; break; }
+                    if (!mbar_wait(p_full + 2, step & 1, wc)) { ok = false; break; }
                     tc_fence_after();
-                    issue_pv(1, vslot, j > jb);
+                    issue_pv(1, vslot, j > jb, 0);
+                    if (!mbar_wait(p_full + 3, step & 1, wc)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_pv(1, vslot, 1, 1);
                     if (last) umma_commit(o_final + 1);
                     umma_commit(slot_empty + vslot);
                     if (!last) {
@@ -353,39 +363,44 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 }
                 const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
                 float lsum = 0.f;
-                // masked keys hold -inf: ex2 returns exactly 0 for them
+                // P in two halves of 64 keys, each released to the MMA warp as soon
+                // as it is in TMEM, so O += P V for the first half overlaps the
+                // exponentials of the second.  Masked keys hold -inf: ex2 gives 0.
 #pragma unroll
-                for (int c = 0; c < C::BN / 32; ++c) {
-                    uint32_t pk[16];
+                for (int half = 0; half < 2; ++half) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float p0 = ex2(fmaf(sv[c * 32 + 2 * e], sl2, neg_m));
-                        const float p1 = ex2(fmaf(sv[c * 32 + 2 * e + 1], sl2, neg_m));
-                        lsum += p0 + p1;
-                        pk[e] = pack_bf16(p0, p1);
+                    for (int c = half * (C::BN / 64); c < (half + 1) * (C::BN / 64); ++c) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const float p0 = ex2(fmaf(sv[c * 32 + 2 * e], sl2, neg_m));
+                            const float p1 = ex2(fmaf(sv[c * 32 + 2 * e + 1], sl2, neg_m));
+                            lsum += p0 + p1;
+                            pk[e] = pack_bf16(p0, p1);
+                        }
+                        tmem_st16(tS + c * 16, pk);
                     }
-                    tmem_st16(tS + c * 16, pk);
+                    if (half == 0 && j > jb && __any_sync(0xffffffffu, resc)) {
+                        // O_t *= alpha before the first O_t += P V of this step.  The
+                        // previous one has completed because S_t(j), which the MMA
+                        // thread issued after it, has.
+                        uint32_t r[32];
+#pragma unroll
+                        for (int c = 0; c < D / 32; ++c) {
+                            tmem_ld32(tO + c * 32, r);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 32; ++e)
+                                r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                            tmem_st32(tO + c * 32, r);
+                        }
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(p_full + 2 * t + half);
                 }
                 l += lsum;
-                if (j > jb && __any_sync(0xffffffffu, resc)) {
-                    // O_t *= alpha.  The previous O_t += P V has completed because
-                    // S_t(j), which the MMA thread issued after it, has; the next
-                    // one waits for this warp's arrival on p_full.
-                    uint32_t r[32];
-#pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        tmem_ld32(tO + c * 32, r);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-                        tmem_st32(tO + c * 32, r);
-                    }
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(p_full + t);
             }
             if (!ok) break;
             // ---------------------------------------------------- epilogue --
