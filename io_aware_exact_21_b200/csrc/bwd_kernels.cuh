@@ -162,7 +162,7 @@ struct BwdCfg {
     static constexpr int OFF_VEC = OFF_ST + NSTAGE * 2 * TILE_BYTES;  // stage stats: float2[BS]
     static constexpr int VEC_BYTES = BS * 8;
     static constexpr int OFF_BAR = OFF_VEC + NSTAGE * VEC_BYTES;
-    static constexpr int NBAR = 2 + 2 * NSTAGE + 4 + 2 + 1;
+    static constexpr int NBAR = 2 + 2 * NSTAGE + 6 + 2 + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int OFF_SCRATCH = OFF_MISC + 16;
     static constexpr int OFF_PREFIX = OFF_SCRATCH + 2 * THREADS * 4;   // block and unit prefixes
@@ -183,8 +183,11 @@ __device__ __forceinline__ void query_tile_range(int k_lo, int k_hi, int n, int 
 
 // Barriers.  s_full / dp_full: the score GEMM and the gradient GEMM of a step
 // have completed.  mid: the element-wise warps are done with the first half
-// of their work (dK/dV kernel: P^T written; dQ kernel: S read).  ready: dS
-// written.  Each completes once per step, so its parity is the step count's.
+// of their work (dK/dV kernel: P^T written, in two parts; dQ kernel: S read,
+// part 0 only).  ready: dS written, in two parts.  A part is the first or the
+// second 32 columns of each warpgroup's 64-column half, so the accumulating
+// GEMM can start on part 0 while part 1 is computed.  Each barrier completes
+// once per step, so its parity is the step count's.
 struct BwdBarriers {
     uint64_t *fix_full, *fix_empty, *stage_full, *stage_empty, *s_full, *dp_full, *mid, *ready,
         *acc_final, *acc_empty, *drain;
@@ -201,9 +204,9 @@ __device__ __forceinline__ BwdBarriers carve_barriers(uint8_t* smem) {
     r.stage_empty = b + 2 + C::NSTAGE;
     r.s_full = b + 2 + 2 * C::NSTAGE;
     r.dp_full = r.s_full + 1;
-    r.mid = r.dp_full + 1;
-    r.ready = r.mid + 1;
-    r.acc_final = r.ready + 1;
+    r.mid = r.dp_full + 1;          // [2 parts]
+    r.ready = r.mid + 2;            // [2 parts]
+    r.acc_final = r.ready + 2;
     r.acc_empty = r.acc_final + 1;
     r.drain = r.acc_empty + 1;
     return r;
@@ -220,8 +223,10 @@ __device__ __forceinline__ void init_barriers(const BwdBarriers& br, volatile in
     }
     mbar_init(br.s_full, 1);
     mbar_init(br.dp_full, 1);
-    mbar_init(br.mid, 8);               // all eight element-wise warps
-    mbar_init(br.ready, 8);
+    for (int part = 0; part < 2; ++part) {
+        mbar_init(br.mid + part, 8);    // all eight element-wise warps
+        mbar_init(br.ready + part, 8);
+    }
     mbar_init(br.acc_final, 1);
     mbar_init(br.acc_empty, 8);
     mbar_init(br.drain, 1);
@@ -249,16 +254,20 @@ __device__ __forceinline__ void issue_scores_ss(uint32_t d_tmem, uint32_t a_base
 // that half's columns (h * 64 ... h * 64 + 31), which it has already read.
 __host__ __device__ constexpr uint32_t packed_col(int kk) { return (kk >> 2) * 64 + (kk & 3) * 8; }
 
-// acc[128 x D] (+)= A[tmem, 128 x 128 bf16, packed] * B[smem, 128 x D, MN-major].
+// acc[128 x D] (+)= A[tmem, rows of `part`, bf16 packed] * B[smem, same rows, MN-major]:
+// part 0 covers k-steps {0, 1, 4, 5} (streamed rows 0-31 and 64-95), part 1
+// covers {2, 3, 6, 7}.  `accumulate` false only for the first part of a tile's
+// first step.
 template <int D>
 __device__ __forceinline__ void issue_acc_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base,
-                                             bool accumulate) {
-    using C = BwdCfg<D>;
+                                             bool accumulate, int part) {
     constexpr uint32_t IDESC = idesc_bf16(128, D, false, true);
 #pragma unroll
-    for (int kk = 0; kk < C::BS / 16; ++kk)
-        umma_ts(d_tmem, a_tmem + packed_col(kk), sw128_desc(b_base + kk * 2048, C::BOX, 1024),
-                IDESC, (accumulate || kk > 0) ? 1u : 0u);
+    for (int i = 0; i < 4; ++i) {
+        const int kk = (i >> 1) * 4 + part * 2 + (i & 1);
+        umma_ts(d_tmem, a_tmem + packed_col(kk), sw128_desc(b_base + kk * 2048, BwdCfg<D>::BOX, 1024),
+                IDESC, (accumulate || i > 0) ? 1u : 0u);
+    }
 }
 
 // Bounded wait that ignores the abort flag (used to drain in-flight work).
@@ -452,9 +461,14 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                     const uint32_t slot = cnt % C::NSTAGE;
                     const uint32_t x = st_addr + slot * 2 * C::TILE_BYTES;
                     const uint32_t xn = st_addr + ((cnt + 1) % C::NSTAGE) * 2 * C::TILE_BYTES;
-                    if (!mbar_wait(br.mid, cnt & 1, wc)) { ok = false; break; }
-                    tc_fence_after();
-                    issue_acc_ts<D>(tmem + C::COL_ACC1, tmem + C::COL_S, x + C::TILE_BYTES, i > ib);  // dV
+                    bool mok = true;
+                    for (int part = 0; part < 2 && mok; ++part) {
+                        if (!mbar_wait(br.mid + part, cnt & 1, wc)) { mok = false; break; }
+                        tc_fence_after();
+                        issue_acc_ts<D>(tmem + C::COL_ACC1, tmem + C::COL_S, x + C::TILE_BYTES,
+                                        i > ib || part > 0, part);                      // dV
+                    }
+                    if (!mok) { ok = false; break; }
                     if (!last) {
                         if (!mbar_wait(br.stage_full + (cnt + 1) % C::NSTAGE, ((cnt + 1) / C::NSTAGE) & 1, wc)) {
                             ok = false;
@@ -464,9 +478,13 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                         issue_scores_ss<D>(tmem + C::COL_S, fa_addr, xn);             // next K Q^T
                         umma_commit(br.s_full);
                     }
-                    if (!mbar_wait(br.ready, cnt & 1, wc)) { ok = false; break; }
-                    tc_fence_after();
-                    issue_acc_ts<D>(tmem + C::COL_ACC0, tmem + C::COL_DP, x, i > ib);     // dK
+                    for (int part = 0; part < 2 && mok; ++part) {
+                        if (!mbar_wait(br.ready + part, cnt & 1, wc)) { mok = false; break; }
+                        tc_fence_after();
+                        issue_acc_ts<D>(tmem + C::COL_ACC0, tmem + C::COL_DP, x, i > ib || part > 0,
+                                        part);                                          // dK
+                    }
+                    if (!mok) { ok = false; break; }
                     umma_commit(br.stage_empty + slot);
                     if (!last) {
                         issue_scores_ss<D>(tmem + C::COL_DP, fb_addr, xn + C::TILE_BYTES);  // next V dO^T
@@ -522,48 +540,55 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                 tmem_ld64(tS, r);
                 tmem_wait_ld();
                 float pf[64];
-                if (!need_mask) {
 #pragma unroll
-                    for (int c = 0; c < 64; ++c) pf[c] = ex2(fmaf(__uint_as_float(r[c]), sl2, vs[c].x));
-                } else {
-                    // masked pairs, and query rows past the sequence end (their
-                    // statistics are padding), get P = 0
+                for (int part = 0; part < 2; ++part) {
+                    if (!need_mask) {
 #pragma unroll
-                    for (int c = 0; c < 64; ++c) {
-                        const float x = ex2(fmaf(__uint_as_float(r[c]), sl2, vs[c].x));
-                        pf[c] = (q0 + c < n && key_allowed(q0 + c, j, n, p.g.causal, p.g.window)) ? x : 0.f;
+                        for (int c = 32 * part; c < 32 * part + 32; ++c)
+                            pf[c] = ex2(fmaf(__uint_as_float(r[c]), sl2, vs[c].x));
+                    } else {
+                        // masked pairs, and query rows past the sequence end (their
+                        // statistics are padding), get P = 0
+#pragma unroll
+                        for (int c = 32 * part; c < 32 * part + 32; ++c) {
+                            const float x = ex2(fmaf(__uint_as_float(r[c]), sl2, vs[c].x));
+                            pf[c] = (q0 + c < n && key_allowed(q0 + c, j, n, p.g.causal, p.g.window)) ? x : 0.f;
+                        }
                     }
-                }
-                {
-                    uint32_t pk[32];
+                    uint32_t pk[16];
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(pf[2 * c], pf[2 * c + 1]);
-                    tmem_st32(tS, pk);           // P^T packed over the first 32 columns of this half
+                    for (int c = 0; c < 16; ++c)
+                        pk[c] = pack_bf16(pf[32 * part + 2 * c], pf[32 * part + 2 * c + 1]);
+                    tmem_st16(tS + 16 * part, pk);   // P^T packed over the first 32 columns of this half
+                    arrive_warp(br.mid + part);
                 }
-                arrive_warp(br.mid);
                 if (!mbar_wait(br.dp_full, cnt & 1, wc)) { ok = false; break; }
                 tc_fence_after();
                 tmem_ld64(tP, r);
                 tmem_wait_ld();
-                {
-                    uint32_t pk[32];
+#pragma unroll
+                for (int part = 0; part < 2; ++part) {
+                    uint32_t pk[16];
                     if (!need_mask) {
 #pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            pk[c] = pack_bf16(pf[2 * c] * (__uint_as_float(r[2 * c]) - vs[2 * c].y),
-                                              pf[2 * c + 1] * (__uint_as_float(r[2 * c + 1]) - vs[2 * c + 1].y));
+                        for (int c = 0; c < 16; ++c) {
+                            const int k = 32 * part + 2 * c;
+                            pk[c] = pack_bf16(pf[k] * (__uint_as_float(r[k]) - vs[k].y),
+                                              pf[k + 1] * (__uint_as_float(r[k + 1]) - vs[k + 1].y));
+                        }
                     } else {
                         // P = 0 must give dS = 0 even where the padding D is not finite
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) {
-                            const float d0 = pf[2 * c] * (__uint_as_float(r[2 * c]) - vs[2 * c].y);
-                            const float d1 = pf[2 * c + 1] * (__uint_as_float(r[2 * c + 1]) - vs[2 * c + 1].y);
-                            pk[c] = pack_bf16(pf[2 * c] != 0.f ? d0 : 0.f, pf[2 * c + 1] != 0.f ? d1 : 0.f);
+                        for (int c = 0; c < 16; ++c) {
+                            const int k = 32 * part + 2 * c;
+                            const float d0 = pf[k] * (__uint_as_float(r[k]) - vs[k].y);
+                            const float d1 = pf[k + 1] * (__uint_as_float(r[k + 1]) - vs[k + 1].y);
+                            pk[c] = pack_bf16(pf[k] != 0.f ? d0 : 0.f, pf[k + 1] != 0.f ? d1 : 0.f);
                         }
                     }
-                    tmem_st32(tP, pk);           // dS^T packed over the first 32 columns of this half
+                    tmem_st16(tP + 16 * part, pk);   // dS^T packed over the first 32 columns of this half
+                    arrive_warp(br.ready + part);
                 }
-                arrive_warp(br.ready);
             }
             if (!ok) break;
             // ------------------------------------------------ epilogue --
@@ -699,9 +724,14 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
                         issue_scores_ss<D>(tmem + C::COL_S, fa_addr, xn);             // next Q K^T
                         umma_commit(br.s_full);
                     }
-                    if (!mbar_wait(br.ready, cnt & 1, wc)) { ok = false; break; }
-                    tc_fence_after();
-                    issue_acc_ts<D>(tmem + C::COL_ACC0, tmem + C::COL_DP, x, j > jb);     // dQ += dS K
+                    bool mok = true;
+                    for (int part = 0; part < 2 && mok; ++part) {
+                        if (!mbar_wait(br.ready + part, cnt & 1, wc)) { mok = false; break; }
+                        tc_fence_after();
+                        issue_acc_ts<D>(tmem + C::COL_ACC0, tmem + C::COL_DP, x, j > jb || part > 0,
+                                        part);                                          // dQ += dS K
+                    }
+                    if (!mok) { ok = false; break; }
                     umma_commit(br.stage_empty + slot);
                     if (!last) {
                         issue_scores_ss<D>(tmem + C::COL_DP, fb_addr, xn + C::TILE_BYTES);  // next dO V^T
@@ -772,15 +802,18 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
                 tc_fence_after();
                 tmem_ld64(tP, r);
                 tmem_wait_ld();
-                {
-                    uint32_t pk[32];
 #pragma unroll
-                    for (int c = 0; c < 32; ++c)
-                        pk[c] = pack_bf16(pf[2 * c] * (__uint_as_float(r[2 * c]) - dq_d),
-                                          pf[2 * c + 1] * (__uint_as_float(r[2 * c + 1]) - dq_d));
-                    tmem_st32(tP, pk);           // dS packed over the first 32 columns of this half
+                for (int part = 0; part < 2; ++part) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const int k = 32 * part + 2 * c;
+                        pk[c] = pack_bf16(pf[k] * (__uint_as_float(r[k]) - dq_d),
+                                          pf[k + 1] * (__uint_as_float(r[k + 1]) - dq_d));
+                    }
+                    tmem_st16(tP + 16 * part, pk);   // dS packed over the first 32 columns of this half
+                    arrive_warp(br.ready + part);
                 }
-                arrive_warp(br.ready);
             }
             if (!ok) break;
             // ------------------------------------------------ epilogue --
