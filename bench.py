@@ -103,10 +103,27 @@ def workload_config(extra=None):
     return cfg
 
 
+# ------------------------------------------------- multi-rank helpers ---
+
+def max_over_ranks(values, world, device=None):
+    """Element-wise maximum of per-rank timings (every rank gets the result);
+    the job is as slow as its slowest rank."""
+    if world <= 1:
+        return [float(v) for v in values]
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(step_flops, world, steps, elapsed_ms):
+    """Whole-job TFLOP/s: the FLOPs all ranks processed over the max-over-ranks time."""
+    return step_flops * world * steps / (elapsed_ms * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------ clocks ---
 
 class ClockSampler:
-    """Samples nvidia-smi clocks and throttle reasons every 200 ms."""
+    """Samples nvidia-smi clocks and throttle reasons every 100 ms."""
     FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
               "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
               "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
@@ -126,7 +143,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "--query-gpu=" + ",".join(self.FIELDS), "--format=csv,noheader,nounits",
-                 "-lms", "200"] + self.sel, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "100"] + self.sel, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
             return
@@ -253,18 +270,15 @@ def run_ours(args, rank, world, device):
     barrier()
     e2e_elapsed = e2.elapsed_time(e3)
 
-    times = torch.tensor([elapsed, e2e_elapsed], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
-    elapsed, e2e_elapsed = float(times[0]), float(times[1])
+    elapsed, e2e_elapsed = max_over_ranks([elapsed, e2e_elapsed], world, device)
     if rank != 0:
         return None
 
     f_fwd, f_bwd = flops(B, H, N, d, causal)
     step_flops = f_fwd + f_bwd
     ms_step = elapsed / args.steps
-    value = step_flops * world * args.steps / (elapsed * 1e-3) / 1e12
-    e2e_value = step_flops * world * e2e_steps / (e2e_elapsed * 1e-3) / 1e12
+    value = job_throughput(step_flops, world, args.steps, elapsed)
+    e2e_value = job_throughput(step_flops, world, e2e_steps, e2e_elapsed)
     peaks, peak_src = load_peaks()
     per_kernel = {}
     for kind, (ms, cnt) in prof.items():
