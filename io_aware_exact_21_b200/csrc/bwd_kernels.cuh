@@ -53,6 +53,8 @@ struct BwdParams {
     Geometry g;
     const float2* stats;
     int64_t stats_stride;
+    const __nv_bfloat16* qrows;   // Q and dO (the dQ kernel reads its own rows directly)
+    const __nv_bfloat16* dorows;
     __nv_bfloat16* out0;    // dK (dkdv_kernel) or dQ (dq_kernel)
     __nv_bfloat16* out1;    // dV (dkdv_kernel)
     float scale;
@@ -616,21 +618,108 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
 }
 
 // ------------------------------------------------------------- dQ kernel --
+// The CTA's own operands Q and dO live in TMEM (packed bf16, written by the
+// element-wise warps straight from global memory), so the score GEMMs read
+// their A operand from TMEM and all shared memory goes to a 3-deep ring of
+// K/V tiles: a tile's refill then starts a step earlier than with two stages.
 template <int D>
-__global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
-dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
-          const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+struct DqCfg {
+    static constexpr int BM = 128;               // queries the CTA owns
+    static constexpr int BS = 128;               // keys streamed per step
+    static constexpr int NSTAGE = 3;
+    static constexpr int NBOX = D / 64;
+    static constexpr int BOX = 128 * 128;
+    static constexpr int TILE_BYTES = 128 * D * 2;
+    static constexpr int THREADS = 384;
+    // TMEM columns: dQ, Q (packed), dO (packed), S, dP
+    static constexpr uint32_t COL_DQ = 0, COL_Q = 128, COL_DO = 192, COL_S = 256, COL_DP = 384;
+    static constexpr int OFF_ST = 0;                                  // stages: K then V
+    static constexpr int OFF_BAR = NSTAGE * 2 * TILE_BYTES;
+    static constexpr int NBAR = 2 * NSTAGE + 1 + 2 + 1 + 2 + 2 + 1;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int OFF_SCRATCH = OFF_MISC + 16;
+    static constexpr int OFF_PREFIX = OFF_SCRATCH + 2 * THREADS * 4;
+    static constexpr int SMEM_BYTES = OFF_PREFIX + 2 * (kMaxVarlenSeqs + 1) * 4 + 1024;
+};
+
+struct DqBarriers {
+    uint64_t *stage_full, *stage_empty, *fix_ready, *s_full, *dp_full, *mid, *ready, *acc_final,
+        *acc_empty, *drain;
+};
+
+// D[128 x 128] = A[tmem 128 x d, packed bf16] * B[smem 128 x d, K-major]^T.
+template <int D>
+__device__ __forceinline__ void issue_scores_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base) {
+    constexpr uint32_t IDESC = idesc_bf16(128, DqCfg<D>::BS, false, false);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * DqCfg<D>::BOX + (kk & 3) * 32;
+        umma_ts(d_tmem, a_tmem + kk * 8, sw128_desc(b_base + off, 16, 1024), IDESC, kk > 0);
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
+dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
           const BwdParams p) {
-    using C = BwdCfg<D>;
+    using C = DqCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align_smem_1024(smem_raw);
-    const BwdBarriers br = carve_barriers<D>(smem);
+    uint64_t* bb = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    DqBarriers br;
+    br.stage_full = bb;
+    br.stage_empty = bb + C::NSTAGE;
+    br.fix_ready = bb + 2 * C::NSTAGE;
+    br.s_full = br.fix_ready + 1;
+    br.dp_full = br.s_full + 1;
+    br.mid = br.dp_full + 1;
+    br.ready = br.mid + 2;          // [2 parts]
+    br.acc_final = br.ready + 2;
+    br.acc_empty = br.acc_final + 1;
+    br.drain = br.acc_empty + 1;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
-    const CUtensorMap* maps[4] = {&tm_q, &tm_do, &tm_k, &tm_v};
-    Schedule sch;
-    const uint32_t tmem = bwd_prologue<D>(smem, br, abort_flag, p, sch, maps);
+    int* scratch = reinterpret_cast<int*>(smem + C::OFF_SCRATCH);
+    int* prefix = reinterpret_cast<int*>(smem + C::OFF_PREFIX);
     const int warp = threadIdx.x >> 5;
     const int lane = lane_id();
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < C::NSTAGE; ++i) {
+            mbar_init(br.stage_full + i, 1);
+            mbar_init(br.stage_empty + i, 1);
+        }
+        mbar_init(br.fix_ready, 8);      // all eight element-wise warps
+        mbar_init(br.s_full, 1);
+        mbar_init(br.dp_full, 1);
+        mbar_init(br.mid, 8);
+        mbar_init(br.ready, 8);
+        mbar_init(br.ready + 1, 8);
+        mbar_init(br.acc_final, 1);
+        mbar_init(br.acc_empty, 8);
+        mbar_init(br.drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_map(&tm_k);
+        tma_prefetch_map(&tm_v);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, 512);
+        tmem_relinquish();
+    }
+    Schedule sch;
+    sch.g = p.g;
+    sch.rows_per_item = C::BM;
+    sch.bprefix = prefix;
+    sch.uprefix = prefix + kMaxVarlenSeqs + 1;
+    sch.total_units = build_schedule_prefix(p.g, C::BM, prefix, prefix + kMaxVarlenSeqs + 1,
+                                            scratch);   // __syncthreads inside
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
     const WaitCtl wc{abort_flag, p.error_word, p.timeout_ns};
     const int H = p.g.H;
 
@@ -638,25 +727,16 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         regs_dealloc<104>();
         if (warp == 0 && lane == 0) {
             // -------------------------------------------------- producer --
-            uint32_t cnt = 0, item_it = 0, fix_issued = 0;
+            uint32_t cnt = 0;
             bool ok = true;
             ItemIter it;
             int s, h, blk;
-            for (; ok && it.next(sch, s, h, blk); ++item_it) {
+            while (ok && it.next(sch, s, h, blk)) {
                 const SeqSpan sp = sch.span(s);
                 const int n = sp.len;
                 const int q0 = blk * C::BM;
                 int jb, je;
                 key_tile_range(q0, min(n, q0 + C::BM), n, p.g.causal, p.g.window, C::BS, jb, je);
-                if (!mbar_wait(br.fix_empty, (item_it & 1) ^ 1, wc)) { ok = false; break; }
-                mbar_arrive_expect_tx(br.fix_full, 2 * C::TILE_BYTES);
-                for (int b = 0; b < C::NBOX; ++b) {
-                    tma_load_3d(smem + C::OFF_FA + b * C::BOX, &tm_q, br.fix_full, b * 64, h,
-                                sp.start + q0);
-                    tma_load_3d(smem + C::OFF_FB + b * C::BOX, &tm_do, br.fix_full, b * 64, h,
-                                sp.start + q0);
-                }
-                ++fix_issued;
                 for (int j = jb; j < je; ++j, ++cnt) {
                     const int slot = cnt % C::NSTAGE;
                     if (!mbar_wait(br.stage_empty + slot, ((cnt / C::NSTAGE) & 1) ^ 1, wc)) {
@@ -676,14 +756,11 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             if (!ok) {
                 for (uint32_t x = cnt > C::NSTAGE ? cnt - C::NSTAGE : 0; x < cnt; ++x)
                     drain_wait(br.stage_full + x % C::NSTAGE, (x / C::NSTAGE) & 1, p.error_word);
-                if (fix_issued) drain_wait(br.fix_full, (fix_issued - 1) & 1, p.error_word);
             }
         } else if (warp == 1 && lane == 0) {
             // ---------------------------------------------------- MMA --
             // per step j:  S_j, dP_j  ->  [S_j read] S_{j+1}  ->  [dS_j written]
             //              dQ += dS_j K_j, dP_{j+1}
-            const uint32_t fa_addr = smem_u32(smem + C::OFF_FA);
-            const uint32_t fb_addr = smem_u32(smem + C::OFF_FB);
             const uint32_t st_addr = smem_u32(smem + C::OFF_ST);
             uint32_t cnt = 0, item_it = 0;
             bool ok = true;
@@ -695,7 +772,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
                 const int q0 = blk * C::BM;
                 int jb, je;
                 key_tile_range(q0, min(n, q0 + C::BM), n, p.g.causal, p.g.window, C::BS, jb, je);
-                if (!mbar_wait(br.fix_full, item_it & 1, wc)) { ok = false; break; }
+                if (!mbar_wait(br.fix_ready, item_it & 1, wc)) { ok = false; break; }
                 if (!mbar_wait(br.acc_empty, (item_it & 1) ^ 1, wc)) { ok = false; break; }
                 if (!mbar_wait(br.stage_full + cnt % C::NSTAGE, (cnt / C::NSTAGE) & 1, wc)) {
                     ok = false;
@@ -704,9 +781,9 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
                 tc_fence_after();
                 {
                     const uint32_t x = st_addr + (cnt % C::NSTAGE) * 2 * C::TILE_BYTES;
-                    issue_scores_ss<D>(tmem + C::COL_S, fa_addr, x);                  // Q K^T
+                    issue_scores_ts<D>(tmem + C::COL_S, tmem + C::COL_Q, x);                // Q K^T
                     umma_commit(br.s_full);
-                    issue_scores_ss<D>(tmem + C::COL_DP, fb_addr, x + C::TILE_BYTES);  // dO V^T
+                    issue_scores_ts<D>(tmem + C::COL_DP, tmem + C::COL_DO, x + C::TILE_BYTES);  // dO V^T
                     umma_commit(br.dp_full);
                 }
                 for (int j = jb; j < je; ++j, ++cnt) {
@@ -721,24 +798,23 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
                         }
                         if (!mbar_wait(br.mid, cnt & 1, wc)) { ok = false; break; }
                         tc_fence_after();
-                        issue_scores_ss<D>(tmem + C::COL_S, fa_addr, xn);             // next Q K^T
+                        issue_scores_ts<D>(tmem + C::COL_S, tmem + C::COL_Q, xn);           // next Q K^T
                         umma_commit(br.s_full);
                     }
                     bool mok = true;
                     for (int part = 0; part < 2 && mok; ++part) {
                         if (!mbar_wait(br.ready + part, cnt & 1, wc)) { mok = false; break; }
                         tc_fence_after();
-                        issue_acc_ts<D>(tmem + C::COL_ACC0, tmem + C::COL_DP, x, j > jb || part > 0,
+                        issue_acc_ts<D>(tmem + C::COL_DQ, tmem + C::COL_DP, x, j > jb || part > 0,
                                         part);                                          // dQ += dS K
                     }
                     if (!mok) { ok = false; break; }
                     umma_commit(br.stage_empty + slot);
                     if (!last) {
-                        issue_scores_ss<D>(tmem + C::COL_DP, fb_addr, xn + C::TILE_BYTES);  // next dO V^T
+                        issue_scores_ts<D>(tmem + C::COL_DP, tmem + C::COL_DO, xn + C::TILE_BYTES);  // next dO V^T
                         umma_commit(br.dp_full);
                     } else {
                         umma_commit(br.acc_final);
-                        umma_commit(br.fix_empty);
                     }
                 }
             }
@@ -769,6 +845,29 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             const int q = q0 + row;               // this thread's query row
             int jb, je;
             key_tile_range(q0, min(n, q0 + C::BM), n, p.g.causal, p.g.window, C::BS, jb, je);
+            {
+                // this row of Q (warpgroup 0) or dO (warpgroup 1) into TMEM as
+                // packed bf16 pairs; rows past the sequence end are zero.  The
+                // previous block's GEMMs have all completed (its epilogue waited
+                // for the last one), so the columns are free.
+                const __nv_bfloat16* src = (g == 0 ? p.qrows : p.dorows) +
+                                           ((static_cast<size_t>(sp.start) + q) * H + h) * D;
+                uint32_t r[D / 2];
+#pragma unroll
+                for (int v = 0; v < D / 8; ++v) {
+                    uint4 x4 = make_uint4(0, 0, 0, 0);
+                    if (q < n) x4 = __ldg(reinterpret_cast<const uint4*>(src) + v);
+                    r[4 * v] = x4.x;
+                    r[4 * v + 1] = x4.y;
+                    r[4 * v + 2] = x4.z;
+                    r[4 * v + 3] = x4.w;
+                }
+                const uint32_t dst = tmem + lane_base + (g == 0 ? C::COL_Q : C::COL_DO);
+#pragma unroll
+                for (int c = 0; c < D / 64; ++c)
+                    tmem_st32(dst + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+                arrive_warp(br.fix_ready);
+            }
             float nl = -INFINITY, dq_d = 0.f;
             if (q < n) {
                 const float2 st = p.stats[stats_index(p.g, p.stats_stride, s, h,
@@ -824,14 +923,19 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
 #pragma unroll
             for (int c = 0; c < D / 64; ++c) {
                 const int col = g * (D / 2) + c * 32;
-                store_row_chunk(tmem + lane_base + C::COL_ACC0 + col, p.scale, p.out0 + off + col, valid);
+                store_row_chunk(tmem + lane_base + C::COL_DQ + col, p.scale, p.out0 + off + col, valid);
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(br.acc_empty);
         }
     }
-    bwd_epilogue_sync<D>(tmem);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
 }
 
 // ------------------------------------------------------------ host side --
@@ -842,7 +946,7 @@ struct BwdMaps {
 struct BwdArgs {
     Geometry g;
     int d;
-    const void *o, *dO;
+    const void *q, *o, *dO;
     const float* lse;
     void *dq, *dk, *dv;
     float2* stats;           // workspace
@@ -883,10 +987,10 @@ inline cudaError_t bwd_set_smem_limits() {
                                   BwdCfg<128>::SMEM_BYTES)) != cudaSuccess)
         return e;
     if ((e = cudaFuncSetAttribute(dq_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  BwdCfg<64>::SMEM_BYTES)) != cudaSuccess)
+                                  DqCfg<64>::SMEM_BYTES)) != cudaSuccess)
         return e;
     return cudaFuncSetAttribute(dq_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                BwdCfg<128>::SMEM_BYTES);
+                                DqCfg<128>::SMEM_BYTES);
 }
 
 // Optional timing callbacks around each launch (kind 1 = D pre-pass,
@@ -917,6 +1021,8 @@ cudaError_t bwd_launch_d(const BwdArgs& a, const BwdMaps& m, cudaStream_t stream
     p.g = a.g;
     p.stats = a.stats;
     p.stats_stride = a.stats_stride;
+    p.qrows = static_cast<const __nv_bfloat16*>(a.q);
+    p.dorows = static_cast<const __nv_bfloat16*>(a.dO);
     p.scale = a.scale;
     p.scale_log2 = a.scale * kLog2e;
     p.error_word = a.error_word;
@@ -934,7 +1040,7 @@ cudaError_t bwd_launch_d(const BwdArgs& a, const BwdMaps& m, cudaStream_t stream
     p.out0 = static_cast<__nv_bfloat16*>(a.dq);
     p.out1 = nullptr;
     slot = hk.start(3, stream);
-    dq_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(m.q, m.dO, m.k, m.v, p);
+    dq_kernel<D><<<grid, DqCfg<D>::THREADS, DqCfg<D>::SMEM_BYTES, stream>>>(m.k, m.v, p);
     hk.stop(3, slot, stream);
     return cudaGetLastError();
 }

@@ -255,6 +255,7 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
     fa::BwdArgs a;
     a.g = c.g;
     a.d = d;
+    a.q = q;
     a.o = o;
     a.dO = dO;
     a.lse = lse;
@@ -299,6 +300,7 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
     fa::BwdArgs a;
     a.g = c.g;
     a.d = d;
+    a.q = q;
     a.o = o;
     a.dO = dO;
     a.lse = lse;
