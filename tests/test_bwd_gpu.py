@@ -152,3 +152,18 @@ def test_bwd_packed_batch_sampled_sequences(window):
             assert_close_bf16(t[a:b, h], ref[name][a:b, h], "%s[seq %d, head %d]" % (name, s, h))
     for t in (dq, dk, dv):
         assert torch.isfinite(t).all()
+
+
+def test_bwd_bench_configuration_sampled_head():
+    """The launch configuration bench.py times: B=4, H=16, N=8192, d=128,
+    non-causal (seed 2, the prefill inputs plus dO); one head in full."""
+    wl = WORKLOADS["prefill_b4"]
+    x = fixed_inputs(wl.B, wl.N, wl.H, wl.d, seed=wl.seed, with_dout=True)
+    o, lse, dq, dk, dv = run(x, False, 0)
+    heads = [(2, 9)]
+    ref = orc.bwd(x["q"], x["k"], x["v"], x["dout"], wl.scale, causal=False, heads=heads)
+    for s, h in heads:
+        for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+            assert_close_bf16(t[s, :, h], ref[name][s, :, h], "%s[%d,:,%d]" % (name, s, h))
+    for t in (dq, dk, dv):
+        assert torch.isfinite(t).all()
