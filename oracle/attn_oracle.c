@@ -62,19 +62,24 @@ static double dot(const double *a, const double *b, int d)
     return acc;
 }
 
-/* One query row, three passes.  Writes o_row[d] and returns the LSE. */
-static double three_pass_row(const double *q, const double *k, const double *v,
-                             int H, int d, int start, int n, int h, int i,
-                             double scale, int causal, int window, double *o_row)
+/* One query row, three passes.  The query row is qstart + i of q; its keys
+ * and values are rows kstart .. kstart + nk - 1 of k and v, and the mask sees
+ * the query at position i + off of the key sequence (off = 0 for
+ * self-attention).  Writes o_row[d] and returns the LSE. */
+static double three_pass_row_kv(const double *q, const double *k, const double *v,
+                                int H, int d, int qstart, int kstart, int nk, int off,
+                                int h, int i, double scale, int causal, int window,
+                                double *o_row)
 {
     const size_t rs = (size_t)H * d;               /* token row stride */
-    const double *qi = q + (size_t)(start + i) * rs + (size_t)h * d;
+    const double *qi = q + (size_t)(qstart + i) * rs + (size_t)h * d;
+    const int pos = i + off;
 
     /* pass 1: row maximum of the scaled scores over allowed keys */
     double m = -INFINITY;
-    for (int j = 0; j < n; ++j) {
-        if (!key_allowed(i, j, causal, window)) continue;
-        double s = scale * dot(qi, k + (size_t)(start + j) * rs + (size_t)h * d, d);
+    for (int j = 0; j < nk; ++j) {
+        if (!key_allowed(pos, j, causal, window)) continue;
+        double s = scale * dot(qi, k + (size_t)(kstart + j) * rs + (size_t)h * d, d);
         if (s > m) m = s;
     }
     for (int c = 0; c < d; ++c) o_row[c] = 0.0;
@@ -82,21 +87,30 @@ static double three_pass_row(const double *q, const double *k, const double *v,
 
     /* pass 2: normaliser l = sum_j exp(s_j - m) */
     double l = 0.0;
-    for (int j = 0; j < n; ++j) {
-        if (!key_allowed(i, j, causal, window)) continue;
-        double s = scale * dot(qi, k + (size_t)(start + j) * rs + (size_t)h * d, d);
+    for (int j = 0; j < nk; ++j) {
+        if (!key_allowed(pos, j, causal, window)) continue;
+        double s = scale * dot(qi, k + (size_t)(kstart + j) * rs + (size_t)h * d, d);
         l += exp(s - m);
     }
 
     /* pass 3: o = sum_j (exp(s_j - m) / l) v_j */
-    for (int j = 0; j < n; ++j) {
-        if (!key_allowed(i, j, causal, window)) continue;
-        const double *vj = v + (size_t)(start + j) * rs + (size_t)h * d;
-        double s = scale * dot(qi, k + (size_t)(start + j) * rs + (size_t)h * d, d);
+    for (int j = 0; j < nk; ++j) {
+        if (!key_allowed(pos, j, causal, window)) continue;
+        const double *vj = v + (size_t)(kstart + j) * rs + (size_t)h * d;
+        double s = scale * dot(qi, k + (size_t)(kstart + j) * rs + (size_t)h * d, d);
         double p = exp(s - m) / l;
         for (int c = 0; c < d; ++c) o_row[c] += p * vj[c];
     }
     return m + log(l);
+}
+
+/* Self-attention row: queries and keys are the same sequence. */
+static double three_pass_row(const double *q, const double *k, const double *v,
+                             int H, int d, int start, int n, int h, int i,
+                             double scale, int causal, int window, double *o_row)
+{
+    return three_pass_row_kv(q, k, v, H, d, start, start, n, 0, h, i, scale, causal, window,
+                             o_row);
 }
 
 /* Full forward over every (sequence, head, row). */
@@ -139,6 +153,42 @@ int oracle_fwd_rows(const double *q, const double *k, const double *v,
         int s = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
         lse_rows[r] = three_pass_row(q, k, v, H, d, starts[s], lens[s], h, i,
                                      scale, causal, window, o_rows + (size_t)r * d);
+    }
+    return 0;
+}
+
+/*
+ * Forward with a key/value sequence that may be longer than the query
+ * sequence (prefill against cached keys and values): sequence s has nq =
+ * qlens[s] query rows starting at qstarts[s] of q and nk = klens[s] key/value
+ * rows starting at kstarts[s] of k and v.  The queries are the LAST nq
+ * positions of the key sequence, so query row i sits at position
+ * i + (nk - nq): under the causal mask it sees keys j <= i + nk - nq
+ * (bottom-right alignment), under a window W also only j > i + nk - nq - W.
+ * With nq = nk this is oracle_fwd.  A query that sees no key gets O = 0 and
+ * LSE = -inf.  o is [Tq, H, d]; lse is [H, Tq].
+ */
+int oracle_fwd_kv(const double *q, const double *k, const double *v,
+                  int Tq, int Tk, int H, int d, int nseq,
+                  const int *qstarts, const int *qlens, const int *kstarts, const int *klens,
+                  double scale, int causal, int window, double *o, double *lse)
+{
+    if (window > 0 && !causal) return -5;
+    if (Tq < 0 || Tk < 0 || H <= 0 || d <= 0 || nseq < 0) return -3;
+    for (int s = 0; s < nseq; ++s)
+        if (qlens[s] < 0 || klens[s] < 0 || qstarts[s] < 0 || kstarts[s] < 0 ||
+            qstarts[s] + qlens[s] > Tq || kstarts[s] + klens[s] > Tk) return -3;
+    const size_t rs = (size_t)H * d;
+    for (int s = 0; s < nseq; ++s) {
+        const int nq = qlens[s], nk = klens[s];
+        #pragma omp parallel for collapse(2) schedule(dynamic, 8)
+        for (int h = 0; h < H; ++h)
+            for (int i = 0; i < nq; ++i) {
+                double *orow = o + (size_t)(qstarts[s] + i) * rs + (size_t)h * d;
+                lse[(size_t)h * Tq + qstarts[s] + i] =
+                    three_pass_row_kv(q, k, v, H, d, qstarts[s], kstarts[s], nk, nk - nq, h, i,
+                                      scale, causal, window, orow);
+            }
     }
     return 0;
 }

@@ -56,6 +56,10 @@ def _load():
         lib.oracle_fwd.argtypes = common + [dp, dp]
         lib.oracle_fwd_rows.argtypes = common + [ctypes.c_int, ip, dp, dp]
         lib.oracle_fwd_online.argtypes = common + [ctypes.c_int, dp, dp]
+        lib.oracle_fwd_kv.argtypes = [dp, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_int, ctypes.c_int, ip, ip, ip, ip, ctypes.c_double,
+                                      ctypes.c_int, ctypes.c_int, dp, dp]
+        lib.oracle_fwd_kv.restype = ctypes.c_int
         lib.oracle_bwd.argtypes = ([dp, dp, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                     ctypes.c_int, ip, ip, ctypes.c_double, ctypes.c_int,
                                     ctypes.c_int, ctypes.c_int, ip, dp, dp, dp, dp, dp, dp])
@@ -188,3 +192,40 @@ def bwd(q, k, v, dout, scale, causal=False, window=0, cu_seqlens=None, heads=Non
     res["lse"] = pk.rowstat(L)
     res["D"] = pk.rowstat(Dd)
     return res
+
+
+def fwd_kv(q, k, v, scale, causal=False, window=0, cu_seqlens_q=None, cu_seqlens_k=None):
+    """Forward of queries against a key/value sequence that may be longer
+    (prefill with cached keys and values; causal masks bottom-right aligned).
+    Fixed length: q [B, Nq, H, d], k/v [B, Nk, H, d] -> O [B, Nq, H, d],
+    LSE [B, H, Nq].  Packed: q [Tq, H, d], k/v [Tk, H, d] with cu_seqlens_q/_k
+    -> O [Tq, H, d], LSE [H, Tq]."""
+    if cu_seqlens_q is None:
+        B, Nq, H, d = q.shape
+        Nk = k.shape[1]
+        Q, K, V = (_f64(x).reshape(-1, H, d) for x in (q, k, v))
+        qs = np.ascontiguousarray(np.arange(B, dtype=np.int32) * Nq)
+        ks = np.ascontiguousarray(np.arange(B, dtype=np.int32) * Nk)
+        ql = np.full(B, Nq, dtype=np.int32)
+        kl = np.full(B, Nk, dtype=np.int32)
+    else:
+        cq = np.asarray(cu_seqlens_q.cpu() if hasattr(cu_seqlens_q, "cpu") else cu_seqlens_q,
+                        dtype=np.int64)
+        ck = np.asarray(cu_seqlens_k.cpu() if hasattr(cu_seqlens_k, "cpu") else cu_seqlens_k,
+                        dtype=np.int64)
+        H, d = q.shape[1], q.shape[2]
+        B = len(cq) - 1
+        Q, K, V = (_f64(x).reshape(-1, H, d) for x in (q, k, v))
+        qs = np.ascontiguousarray(cq[:-1], dtype=np.int32)
+        ks = np.ascontiguousarray(ck[:-1], dtype=np.int32)
+        ql = np.ascontiguousarray(np.diff(cq), dtype=np.int32)
+        kl = np.ascontiguousarray(np.diff(ck), dtype=np.int32)
+    Tq, Tk = Q.shape[0], K.shape[0]
+    O = np.zeros_like(Q)
+    L = np.zeros((H, Tq), dtype=np.float64)
+    _check(_load().oracle_fwd_kv(_dp(Q), _dp(K), _dp(V), Tq, Tk, H, d, B, _ip(qs), _ip(ql),
+                                 _ip(ks), _ip(kl), float(scale), int(bool(causal)), int(window),
+                                 _dp(O), _dp(L)))
+    if cu_seqlens_q is None:
+        return O.reshape(B, Nq, H, d), L.reshape(H, B, Nq).transpose(1, 0, 2).copy()
+    return O, L
