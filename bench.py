@@ -13,6 +13,10 @@ replicas (no collective: the (sequence, head) units share nothing).
 --impl reference times the float64 CPU oracle (the reference arm: there is
 no runnable reference implementation) on a bounded sample of the same
 workload on the host cores.
+
+--workload prefill_kv measures the cached-KV prefill forward instead
+(fa_fwd_kv: B=4, H=16, 2048 new query tokens after 6144 cached ones, so
+Nk=8192, d=128, causal aligned bottom-right), with its own oracle sample.
 """
 from __future__ import annotations
 
@@ -72,6 +76,17 @@ def traffic_for(kernel):
     if (w["B"], w["H"], w["N"], w["d"], w["causal"]) != (4, 16, 8192, 128, False):
         return None
     return t["bytes_per_launch"]
+
+
+PREFILL_KV = dict(B=4, H=16, Nq=2048, Nk=8192, d=128, causal=True, window=0, seed=5)
+
+
+def flops_kv(B, H, Nq, Nk, d, causal):
+    """Forward FLOPs of Nq queries against Nk keys: 4*d per (query, key) pair
+    the mask keeps, with the causal triangle of the last Nq positions halved
+    as in the self-attention count."""
+    pairs = Nq * Nk - (0.5 * Nq * Nq if causal else 0.0)
+    return 4.0 * B * H * pairs * d
 
 
 def flops(B, H, N, d, causal):
@@ -356,6 +371,144 @@ def run_ours(args, rank, world, device):
     return out
 
 
+# ------------------------------------------- cached-KV prefill arm ---
+
+def prefill_kv_config(extra=None):
+    w = PREFILL_KV
+    cfg = {"workload": "cached-KV prefill B%d H%d Nq%d Nk%d d%d %s (bottom-right), forward only"
+           % (w["B"], w["H"], w["Nq"], w["Nk"], w["d"], "causal" if w["causal"] else "non-causal"),
+           "B": w["B"], "H": w["H"], "Nq": w["Nq"], "Nk": w["Nk"], "d": w["d"],
+           "causal": w["causal"], "window": w["window"], "seed": w["seed"],
+           "l2": "inputs larger than L2 (K, V 128 MiB each); L2 not flushed"}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+def run_prefill_kv(args, rank, world, device):
+    import io_aware_exact_21_b200 as fa
+    from io_aware_exact_21_b200.inputs import kv_inputs
+    w = PREFILL_KV
+    B, H, Nq, Nk, d = w["B"], w["H"], w["Nq"], w["Nk"], w["d"]
+    causal, window = w["causal"], w["window"]
+    scale = 1.0 / math.sqrt(d)
+    host = kv_inputs(B, Nq, Nk, H, d, seed=w["seed"] + rank)
+    q, k, v = (host[n].to(device) for n in ("q", "k", "v"))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(qq, kk, vv, oo, ll):
+        fa.forward_kv(qq, kk, vv, causal=causal, window=window, scale=scale, out=oo, lse=ll,
+                      stream=stream)
+
+    for _ in range(args.warmup):
+        step(q, k, v, o, lse)
+    torch.cuda.synchronize(device)
+    assert fa.fa_get_device_error() == 0
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    clocks = ClockSampler(device)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize(device)
+    fa.fa_profile_begin()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step(q, k, v, o, lse)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    elapsed = e0.elapsed_time(e1)
+    prof = fa.fa_profile_end()
+    clk = clocks.stop()
+    assert fa.fa_get_device_error() == 0
+
+    # end to end: each step copies Q, K, V in from pinned host memory and O,
+    # LSE back, in order on one stream (no overlap between steps).
+    pin = {n: host[n].pin_memory() for n in ("q", "k", "v")}
+    dev_in = {n: torch.empty_like(t, device=device) for n, t in pin.items()}
+    host_o = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    host_l = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = host_o.numel() * host_o.element_size() + host_l.numel() * host_l.element_size()
+
+    def e2e_step():
+        for n in ("q", "k", "v"):
+            dev_in[n].copy_(pin[n], non_blocking=True)
+        step(dev_in["q"], dev_in["k"], dev_in["v"], o, lse)
+        host_o.copy_(o, non_blocking=True)
+        host_l.copy_(lse, non_blocking=True)
+
+    e2e_steps = max(2, min(args.steps, 10))
+    e2e_step()
+    torch.cuda.synchronize(device)
+    barrier()
+    e2 = torch.cuda.Event(enable_timing=True)
+    e3 = torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e3.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    e2e_elapsed = e2.elapsed_time(e3)
+    assert fa.fa_get_device_error() == 0
+
+    elapsed, e2e_elapsed = max_over_ranks([elapsed, e2e_elapsed], world, device)
+    if rank != 0:
+        return None
+    f = flops_kv(B, H, Nq, Nk, d, causal)
+    value = job_throughput(f, world, args.steps, elapsed)
+    ms, cnt = prof["fwd"]
+    kernel_ms = ms / cnt
+    peaks, peak_src = load_peaks()
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    achieved = f / (kernel_ms * 1e-3) / 1e12
+    return {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(elapsed / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: i.i.d. N(0,1) bf16 Q, K, V (seeded), no dataset",
+        "config": prefill_kv_config({"parallelism": "replicas" if world > 1 else "single GPU"}),
+        "roofline": {"kernel": "fwd", "bound": "tensor", "achieved": round(achieved, 2),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "peak_source": "%s bf16_tflops (burst: the kernel is timed alone)" % peak_src,
+                     "traffic": None,
+                     "traffic_unit": "bytes per launch (ncu dram read + write)"},
+        "e2e": {"value": round(job_throughput(f, world, e2e_steps, e2e_elapsed), 2), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "how": "pinned host -> device copy of Q, K, V and device -> host copy of O, LSE "
+                       "every step, in order on the compute stream"},
+        "gpu_launches": sum(c for (_, c) in prof.values()),
+        "clocks": clk,
+    }
+
+
+def oracle_sample_kv(n_q=None, seed=5):
+    """Time the float64 oracle's cached-KV forward on one (sequence, head) of
+    the prefill workload, optionally with fewer queries (the key length and
+    the queries' positions at its end are kept)."""
+    from oracle import oracle as orc
+    from io_aware_exact_21_b200.inputs import kv_inputs
+    w = PREFILL_KV
+    nq = n_q or w["Nq"]
+    x = kv_inputs(1, nq, w["Nk"], 1, w["d"], seed=seed)
+    t0 = time.perf_counter()
+    orc.fwd_kv(x["q"], x["k"], x["v"], 1.0 / math.sqrt(w["d"]), causal=w["causal"],
+               window=w["window"])
+    secs = time.perf_counter() - t0
+    f = flops_kv(1, 1, nq, w["Nk"], w["d"], w["causal"])
+    desc = ("cached-KV forward of one (sequence, head) of the prefill workload: %d queries, "
+            "%d keys, d=%d, %.1f s on %d threads" % (nq, w["Nk"], w["d"], secs, orc.num_threads()))
+    return f / secs / 1e12, desc, orc.num_threads(), secs
+
+
 # ------------------------------------------------- CPU oracle (sample) ---
 
 def oracle_sample(n_tokens=None, seed=2):
@@ -387,17 +540,21 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return None
+    kv = args.workload == "prefill_kv"
     for _ in range(args.warmup):
-        oracle_sample(n_tokens=256)
+        if kv:
+            oracle_sample_kv(n_q=16)
+        else:
+            oracle_sample(n_tokens=256)
     vals = []
     t0 = time.perf_counter()
     desc = threads = None
     for _ in range(args.steps):
-        val, desc, threads, _ = oracle_sample(n_tokens=2048)
+        val, desc, threads, _ = oracle_sample_kv(n_q=256) if kv else oracle_sample(n_tokens=2048)
         vals.append(val)
     elapsed = time.perf_counter() - t0
     value = statistics.mean(vals)
-    cfg = workload_config({"parallelism": "host cores"})
+    cfg = (prefill_kv_config if kv else workload_config)({"parallelism": "host cores"})
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": elapsed * 1e3 / max(1, args.steps),
@@ -419,6 +576,9 @@ def main():
     ap.add_argument("--shape", default=None,
                     help="B,H,N,d override of the workload (profiling of smaller cases)")
     ap.add_argument("--causal", action="store_true", help="causal mask (profiling)")
+    ap.add_argument("--workload", choices=["train", "prefill_kv"], default="train",
+                    help="train: forward+backward step (default); prefill_kv: cached-KV "
+                         "prefill forward")
     args = ap.parse_args()
     if args.shape:
         B, H, N, d = (int(x) for x in args.shape.split(","))
@@ -445,11 +605,12 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                              device_id=device)
+    kv = args.workload == "prefill_kv"
     try:
-        out = run_ours(args, rank, world, device)
+        out = (run_prefill_kv if kv else run_ours)(args, rank, world, device)
         if out is not None:
             if not args.no_cpu_baseline and world == 1:
-                val, desc, threads, secs = oracle_sample()
+                val, desc, threads, secs = oracle_sample_kv() if kv else oracle_sample()
                 out["cpu_baseline"] = {"value": val, "unit": UNIT, "cores": threads,
                                        "kind": "oracle", "sample": desc}
             else:

@@ -33,7 +33,7 @@
  *   Packed batches hold at most 2048 sequences.
  *
  * Masks (row i, key j local to a sequence of n tokens; query and key sequences
- * have the same length):
+ * have the same length except in fa_fwd_kv, below):
  *   causal != 0 : key j allowed only if j <= i (top-left aligned).
  *   window  > 0 : sliding window of exactly `window` keys ending at the
  *                 query's own position: allowed only if i - window < j <= i.
@@ -49,8 +49,9 @@
  *   wait that runs out records FA_ERR_DEVICE_TIMEOUT in a device error word
  *   that fa_get_device_error() reports.
  *
- * Asynchrony: fa_fwd and fa_bwd enqueue kernels on `stream` and return
- *   without synchronising; outputs are valid once the stream reaches them.
+ * Asynchrony: the forward and backward entry points enqueue kernels on
+ *   `stream` and return without synchronising; outputs are valid once the
+ *   stream reaches them.
  */
 #ifndef FA_B200_H
 #define FA_B200_H
@@ -84,6 +85,40 @@ typedef enum {
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
            int B, int H, int N, int d, float scale, int causal, int window,
            const int* cu_seqlens, cudaStream_t stream);
+
+/*
+ * Forward pass of queries against a longer cached key/value sequence
+ * (prefill of a chunk of new tokens after earlier ones whose keys and values
+ * are already computed).  Same operation as fa_fwd, with key/value sequences
+ * that may differ in length from the query sequences; fa_fwd(..., N, ...) is
+ * fa_fwd_kv(..., N, N, ..., cu_seqlens, cu_seqlens, ...).  The pages define
+ * attention for any number of keys per query and name cached keys and values
+ * as an interface (FlashAttention encyclopedia page, "software integration");
+ * where the queries sit inside the key sequence they leave open, and this
+ * library takes the reading that follows from prefill: the nq queries of a
+ * sequence are its LAST nq positions, so query row i is at key position
+ * i + nk - nq (bottom-right alignment) and the causal and window rules apply
+ * to that position:
+ *   causal : key j allowed only if j <= i + nk - nq,
+ *   window : also only if j > i + nk - nq - window.
+ * A query without any allowed key (nk = 0, or causal with i + nk - nq < 0)
+ * gets O = 0 and LSE = -inf.
+ *
+ * q, o : [tokens_q, H, d]; k, v : [tokens_k, H, d]; lse as fa_fwd over the
+ *   query rows ([B, H, Nq] fixed, [H, Tq] packed).
+ * Fixed length (both cu_seqlens NULL): Nq queries and Nk keys per sequence,
+ *   tokens_q = B * Nq, tokens_k = B * Nk.
+ * Packed (both non-NULL; one NULL and one not is FA_ERR_BAD_SHAPE):
+ *   cu_seqlens_q / cu_seqlens_k are device int32 arrays of B + 1 offsets into
+ *   the query and key buffers; Nq and Nk are the token rows those buffers
+ *   hold.  Per-sequence lengths may differ in either direction.
+ * k and v may be NULL when the key buffers hold no rows (tokens_k = 0).
+ * Errors as fa_fwd.  The backward entry points take equal query and key
+ * lengths only.
+ */
+int fa_fwd_kv(const void* q, const void* k, const void* v, void* o, float* lse,
+              int B, int H, int Nq, int Nk, int d, float scale, int causal, int window,
+              const int* cu_seqlens_q, const int* cu_seqlens_k, cudaStream_t stream);
 
 /*
  * Bytes of device workspace fa_bwd needs: 8 bytes per (head, row) for the

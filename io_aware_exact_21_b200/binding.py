@@ -25,6 +25,7 @@ NOALLOC_MAX_ROWS = 1 << 20   # FA_NOALLOC_MAX_ROWS in include/fa.h (8-byte entri
 _VP, _I, _F, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 SIGNATURES = {
     "fa_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _I, _VP, _VP]),
+    "fa_fwd_kv": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _I, _VP, _VP, _VP]),
     "fa_bwd_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "fa_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _I,
                     _VP, _VP, _SZ, _VP]),
@@ -105,6 +106,14 @@ def fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, window, cu_seqlens, strea
                                  _ptr(cu_seqlens), _stream(stream))
 
 
+def fa_fwd_kv(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, window, cu_seqlens_q,
+              cu_seqlens_k, stream=None) -> int:
+    return load_library().fa_fwd_kv(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), int(B),
+                                    int(H), int(Nq), int(Nk), int(d), float(scale), int(causal),
+                                    int(window), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
+                                    _stream(stream))
+
+
 def fa_bwd_workspace_size(B, H, N, d, varlen_total=0) -> int:
     return int(load_library().fa_bwd_workspace_size(int(B), int(H), int(N), int(d),
                                                     int(varlen_total)))
@@ -178,6 +187,29 @@ def forward(q, k, v, causal=False, window=0, cu_seqlens=None, scale=None, out=No
                           device=q.device)
     _check(fa_fwd(q, k, v, out, lse, B, H, N, d, scale, causal, window, cu_seqlens, stream),
            "fa_fwd")
+    return out, lse
+
+
+def forward_kv(q, k, v, causal=False, window=0, cu_seqlens_q=None, cu_seqlens_k=None,
+               scale=None, out=None, lse=None, stream=None):
+    """O, LSE of queries q [B, Nq, H, d] against cached keys/values k, v
+    [B, Nk, H, d] (or packed [Tq, H, d] / [Tk, H, d] with int32 cu_seqlens_q
+    and cu_seqlens_k); queries are the last positions of their key sequence."""
+    import torch
+    B, H, Nq, d = _shape(q, cu_seqlens_q)
+    if cu_seqlens_q is None:
+        Nk = k.shape[1]
+    else:
+        Nk = k.shape[0]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Nq) if cu_seqlens_q is None else (H, Nq), dtype=torch.float32,
+                          device=q.device)
+    _check(fa_fwd_kv(q, k, v, out, lse, B, H, Nq, Nk, d, scale, causal, window, cu_seqlens_q,
+                     cu_seqlens_k, stream), "fa_fwd_kv")
     return out, lse
 
 

@@ -140,6 +140,10 @@ int validate_common(int B, int H, int N, int d, float scale, int causal, int win
     c->g.cu_seqlens = cu_seqlens;
     c->g.causal = causal ? 1 : 0;
     c->g.window = window > 0 ? window : 0;
+    // self-attention: the key/value sequences are the query sequences
+    c->g.Nk = c->g.N;
+    c->g.Tk = c->g.T;
+    c->g.cu_seqlens_k = cu_seqlens;
     return FA_OK;
 }
 
@@ -188,19 +192,42 @@ extern "C" {
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
            int d, float scale, int causal, int window, const int* cu_seqlens,
            cudaStream_t stream) {
-    if (!q || !k || !v || !o || !lse) return FA_ERR_NULLPTR;
+    return fa_fwd_kv(q, k, v, o, lse, B, H, N, N, d, scale, causal, window, cu_seqlens,
+                     cu_seqlens, stream);
+}
+
+int fa_fwd_kv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+              int Nq, int Nk, int d, float scale, int causal, int window,
+              const int* cu_seqlens_q, const int* cu_seqlens_k, cudaStream_t stream) {
+    if (!q || !o || !lse) return FA_ERR_NULLPTR;
     Common c;
-    int rc = validate_common(B, H, N, d, scale, causal, window, cu_seqlens, &c);
+    int rc = validate_common(B, H, Nq, d, scale, causal, window, cu_seqlens_q, &c);
     if (rc != FA_OK) return rc;
+    if (Nk < 0 || (cu_seqlens_q == nullptr) != (cu_seqlens_k == nullptr)) return FA_ERR_BAD_SHAPE;
+    if (cu_seqlens_k && (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u)) return FA_ERR_MISALIGNED;
+    const bool packed = cu_seqlens_q != nullptr;
+    const int64_t rows_k = packed ? static_cast<int64_t>(Nk) : static_cast<int64_t>(B) * Nk;
+    if (rows_k > (int64_t{1} << 31) - 1 || rows_k * H * d > (int64_t{1} << 40))
+        return FA_ERR_BAD_SHAPE;
+    if (rows_k > 0 && (!k || !v)) return FA_ERR_NULLPTR;   // k, v may be NULL without key rows
+    c.g.Nk = packed ? 0 : Nk;
+    c.g.Tk = static_cast<int>(rows_k);
+    c.g.cu_seqlens_k = cu_seqlens_k;
     if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(o) || misaligned(lse))
         return FA_ERR_MISALIGNED;
     if (B == 0 || c.rows == 0) return FA_OK;
     DeviceState* st = nullptr;
     if ((rc = device_setup(&st)) != FA_OK) return rc;
 
+    // With no key rows at all every key tile is fully masked (each sequence
+    // has nk = 0), but a tensor map cannot be empty: point the K/V maps at q,
+    // whose tiles are then loaded, masked and contribute nothing.
+    const void* kk = rows_k > 0 ? k : q;
+    const void* vv = rows_k > 0 ? v : q;
+    const int64_t map_rows_k = rows_k > 0 ? rows_k : c.rows;
     CUtensorMap mq, mk, mv;
-    if (make_map(&mq, q, c.rows, H, d, 128) || make_map(&mk, k, c.rows, H, d, 128) ||
-        make_map(&mv, v, c.rows, H, d, 128))
+    if (make_map(&mq, q, c.rows, H, d, 128) || make_map(&mk, kk, map_rows_k, H, d, 128) ||
+        make_map(&mv, vv, map_rows_k, H, d, 128))
         return FA_ERR_CUDA;
 
     fa::FwdParams p;
@@ -213,8 +240,8 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
     p.fault_skip_v = g_fault_mode == 1 ? 1 : 0;
 
     int grid = st->num_sms;
-    if (!cu_seqlens) {
-        const int64_t items = static_cast<int64_t>(B) * H * ((N + 255) / 256);
+    if (!packed) {
+        const int64_t items = static_cast<int64_t>(B) * H * ((Nq + 255) / 256);
         if (items < grid) grid = static_cast<int>(items);
     }
     const int slot = prof_start(0, stream);

@@ -153,10 +153,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             int s, h, blk;
             for (; ok && it.next(sch, s, h, blk); ++item_it) {
                 const SeqSpan sp = sch.span(s);
+                const SeqSpan kp = sch.kspan(s);
+                const int off = kp.len - sp.len;        // key position of query row 0
                 const int r_lo = blk * C::ROWS;
                 const int r_hi = min(sp.len, r_lo + C::ROWS);
                 int jb, je;
-                key_tile_range(r_lo, r_hi, sp.len, p.g.causal, p.g.window, C::BN, jb, je);
+                key_tile_range(r_lo + off, r_hi + off, kp.len, p.g.causal, p.g.window, C::BN, jb, je);
                 if (!mbar_wait(q_empty, (item_it & 1) ^ 1, wc)) { ok = false; break; }
                 mbar_arrive_expect_tx(q_full, 2 * C::TILE_BYTES);
                 for (int t = 0; t < 2; ++t)
@@ -179,7 +181,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                             const CUtensorMap* tm = kv == 0 ? &tm_k : &tm_v;
                             for (int b = 0; b < C::NBOX; ++b)
                                 tma_load_3d(sKV + slot * C::TILE_BYTES + b * C::BOX_BYTES, tm,
-                                            slot_full + slot, b * 64, h, sp.start + j * C::BN);
+                                            slot_full + slot, b * 64, h, kp.start + j * C::BN);
                         }
                         ++cnt;
                     }
@@ -230,10 +232,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             int s, h, blk;
             for (; ok && it.next(sch, s, h, blk); ++item_it) {
                 const SeqSpan sp = sch.span(s);
+                const SeqSpan kp = sch.kspan(s);
+                const int off = kp.len - sp.len;
                 const int r_lo = blk * C::ROWS;
                 const int r_hi = min(sp.len, r_lo + C::ROWS);
                 int jb, je;
-                key_tile_range(r_lo, r_hi, sp.len, p.g.causal, p.g.window, C::BN, jb, je);
+                key_tile_range(r_lo + off, r_hi + off, kp.len, p.g.causal, p.g.window, C::BN, jb, je);
                 if (!mbar_wait(q_full, item_it & 1, wc)) { ok = false; break; }
                 // first key tile
                 uint32_t kslot = cnt % C::NSLOT;
@@ -310,11 +314,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         int s, h, blk;
         for (; ok && it.next(sch, s, h, blk); ++item_it) {
             const SeqSpan sp = sch.span(s);
+            const SeqSpan kp = sch.kspan(s);
             const int n = sp.len;
+            const int nk = kp.len;
+            const int off = nk - n;                     // key position of query row 0
             const int r_lo = blk * C::ROWS;
             const int r_hi = min(n, r_lo + C::ROWS);
             int jb, je;
-            key_tile_range(r_lo, r_hi, n, p.g.causal, p.g.window, C::BN, jb, je);
+            key_tile_range(r_lo + off, r_hi + off, nk, p.g.causal, p.g.window, C::BN, jb, je);
             const int r0 = r_lo + t * C::BM;            // first row of this tile
             const int i = r0 + row_in_tile;             // this thread's row
             float m_ref = -INFINITY;
@@ -333,11 +340,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     for (int e = 0; e < C::BN; ++e) sv[e] = __uint_as_float(r[e]);
                 }
                 const int k0 = j * C::BN;
-                const bool masked = tile_needs_mask(r0, C::BM, k0, C::BN, n, p.g.causal, p.g.window);
+                const bool masked = tile_needs_mask_pos(r0 + off, min(r0 + C::BM, n) + off, k0, C::BN,
+                                                        nk, p.g.causal, p.g.window);
                 if (masked) {
 #pragma unroll
                     for (int c = 0; c < C::BN; ++c)
-                        if (!key_allowed(i, k0 + c, n, p.g.causal, p.g.window)) sv[c] = -INFINITY;
+                        if (!key_allowed(i + off, k0 + c, nk, p.g.causal, p.g.window)) sv[c] = -INFINITY;
                 }
                 // row maximum as a tree (the max is exact in any order), so the
                 // 127 compares are not one dependent chain

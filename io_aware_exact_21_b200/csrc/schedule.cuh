@@ -19,11 +19,17 @@ constexpr int kMaxVarlenSeqs = 2048;   // sequences a packed batch may hold
 struct Geometry {
     int B;                  // sequences
     int H;                  // heads
-    int N;                  // fixed length; 0 for packed batches
-    int T;                  // token rows of the [T, H, d] buffers
+    int N;                  // fixed length of the query sequences; 0 for packed batches
+    int T;                  // token rows of the query buffers [T, H, d]
     const int* cu_seqlens;  // device, B + 1 entries, or nullptr
     int causal;
     int window;             // <= 0: none
+    // Key/value sequences (equal to the query ones for self-attention).  The
+    // queries of a sequence are the last ones of its key sequence, so query
+    // row i sits at key position i + (nk - nq).
+    int Nk;                 // fixed key length
+    int Tk;                 // token rows of the key/value buffers
+    const int* cu_seqlens_k;
 };
 
 struct SeqSpan {
@@ -36,30 +42,39 @@ __device__ __forceinline__ bool key_allowed(int i, int j, int n, int causal, int
     return j < n && (!causal || j <= i) && (window <= 0 || j > i - window);
 }
 
-// Key-tile range [jb, je) that query rows [r_lo, r_hi) of a sequence of
-// length n need, for key tiles of BN keys; tiles outside it are fully masked
-// and never loaded.
-__device__ __forceinline__ void key_tile_range(int r_lo, int r_hi, int n, int causal, int window,
+// Key-tile range [jb, je) that queries at key positions [p_lo, p_hi) need in
+// a key sequence of length nk, for key tiles of BN keys; tiles outside it are
+// fully masked and never loaded.  An empty range becomes one (fully masked)
+// tile, so every block runs the same protocol and its queries without any
+// allowed key come out as O = 0, LSE = -inf.
+__device__ __forceinline__ void key_tile_range(int p_lo, int p_hi, int nk, int causal, int window,
                                                int BN, int& jb, int& je) {
     int k_lo = 0;
-    if (window > 0) k_lo = max(0, r_lo - window + 1);
-    int k_hi = causal ? min(n, r_hi) : n;
+    if (window > 0) k_lo = max(0, p_lo - window + 1);
+    int k_hi = causal ? min(nk, p_hi) : nk;
     jb = k_lo / BN;
     je = (k_hi + BN - 1) / BN;
-    if (je < jb) je = jb;
+    if (je <= jb) je = jb + 1;
 }
 
-// True when some pair of (rows [r0, r0+BM) inside the sequence, keys
-// [k0, k0+BN)) is masked out, so the tile needs the element-wise mask.  Rows
-// past the sequence end are not considered: their results are never stored,
-// and ignoring them makes the decision depend only on the mask's meaning (a
-// window of n or more keys classifies every tile exactly like plain causal).
+// True when some pair of (queries at key positions [p0, p_end), keys
+// [k0, k0+BN)) is masked out, so the tile needs the element-wise mask.
+// p_end excludes rows past the query sequence end: their results are never
+// stored, and ignoring them makes the decision depend only on the mask's
+// meaning (a window of n or more keys classifies every tile like causal).
+__device__ __forceinline__ bool tile_needs_mask_pos(int p0, int p_end, int k0, int BN, int nk,
+                                                    int causal, int window) {
+    if (k0 + BN > nk) return true;
+    if (p0 < 0) return true;
+    if (causal && k0 + BN - 1 > p0) return true;
+    if (window > 0 && k0 <= p_end - 1 - window) return true;
+    return false;
+}
+
+// Self-attention form: rows [r0, r0+BM) of a sequence of n tokens.
 __device__ __forceinline__ bool tile_needs_mask(int r0, int BM, int k0, int BN, int n, int causal,
                                                 int window) {
-    if (k0 + BN > n) return true;
-    if (causal && k0 + BN - 1 > r0) return true;
-    if (window > 0 && k0 <= min(r0 + BM, n) - 1 - window) return true;
-    return false;
+    return tile_needs_mask_pos(r0, min(r0 + BM, n), k0, BN, n, causal, window);
 }
 
 // Static persistent schedule.  The rows of a (sequence, head) are cut into
@@ -86,6 +101,15 @@ struct Schedule {
             return SeqSpan{a, g.cu_seqlens[s + 1] - a};
         }
         return SeqSpan{s * g.N, g.N};
+    }
+
+    // Key/value span of sequence s.
+    __device__ __forceinline__ SeqSpan kspan(int s) const {
+        if (g.cu_seqlens_k) {
+            int a = g.cu_seqlens_k[s];
+            return SeqSpan{a, g.cu_seqlens_k[s + 1] - a};
+        }
+        return SeqSpan{s * g.Nk, g.Nk};
     }
 
     // Blocks of the sequences before s (packed batches; 0 for fixed length).

@@ -12,7 +12,11 @@ Recipe (the pages fix only "i.i.d. N(0,1) bf16, seed s"):
     ``torch.randint(lo, hi + 1, (nseq,), generator=g)`` from the same seeded
     generator, then Q, K, V (and dO) with shape ``[T, H, d]``,
     ``T = sum(lengths)``; ``cu_seqlens`` is the int32 prefix sum with a
-    leading 0.
+    leading 0;
+  * queries against longer cached keys/values: as above, with Q drawn over
+    the query rows and K, V over the key rows (fixed ``[B, Nq, H, d]`` and
+    ``[B, Nk, H, d]``; packed ``[Tq, H, d]`` and ``[Tk, H, d]`` with
+    ``cu_seqlens_q`` / ``cu_seqlens_k`` from explicit per-sequence lengths).
 """
 from __future__ import annotations
 
@@ -53,6 +57,27 @@ def varlen_inputs(nseq: int, lo: int, hi: int, H: int, d: int, seed: int,
     return out
 
 
+def kv_inputs(B: int, Nq: int, Nk: int, H: int, d: int, seed: int):
+    g = torch.Generator("cpu").manual_seed(seed)
+    shapes = {"q": [B, Nq, H, d], "k": [B, Nk, H, d], "v": [B, Nk, H, d]}
+    return {n: torch.randn(shp, dtype=torch.float32, generator=g).to(torch.bfloat16)
+            for n, shp in shapes.items()}
+
+
+def varlen_kv_inputs(lens_q, lens_k, H: int, d: int, seed: int):
+    """Packed queries and keys/values with the given per-sequence lengths."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    out = {}
+    for name, lens in (("q", lens_q), ("k", lens_k)):
+        cu = torch.zeros(len(lens) + 1, dtype=torch.int32)
+        cu[1:] = torch.cumsum(torch.as_tensor(lens, dtype=torch.int64), 0).to(torch.int32)
+        out["cu_seqlens_" + name] = cu
+    Tq, Tk = int(out["cu_seqlens_q"][-1]), int(out["cu_seqlens_k"][-1])
+    for name, T in (("q", Tq), ("k", Tk), ("v", Tk)):
+        out[name] = torch.randn([T, H, d], dtype=torch.float32, generator=g).to(torch.bfloat16)
+    return out
+
+
 @dataclass(frozen=True)
 class Workload:
     """One named workload: shapes, seed and mask of a parity or bench case."""
@@ -66,12 +91,15 @@ class Workload:
     window: int = 0
     varlen: tuple = field(default=None)   # (nseq, lo, hi) for packed inputs
     backward: bool = False
+    Nk: int = 0                           # > 0: keys/values per sequence (cached-KV prefill)
 
     @property
     def scale(self) -> float:
         return 1.0 / math.sqrt(self.d)
 
     def make(self):
+        if self.Nk > 0:
+            return kv_inputs(self.B, self.N, self.Nk, self.H, self.d, self.seed)
         if self.varlen is not None:
             nseq, lo, hi = self.varlen
             return varlen_inputs(nseq, lo, hi, self.H, self.d, self.seed, with_dout=self.backward)
@@ -95,4 +123,7 @@ WORKLOADS = {
                               window=1024, varlen=(16, 128, 4096)),
     "bwd_causal": Workload("bwd_causal", B=2, H=16, N=4096, d=128, seed=4, causal=True,
                            backward=True),
+    # a 2048-token prompt chunk after 6144 cached tokens
+    "prefill_kv_causal": Workload("prefill_kv_causal", B=4, H=16, N=2048, d=128, seed=5,
+                                  causal=True, Nk=8192),
 }

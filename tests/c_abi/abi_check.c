@@ -22,6 +22,9 @@ int main(void) {
     CHECK(fa_fwd(p, p, p, p, f, 1, 1, 128, 128, 0.1f, 0, 7, NULL, 0), FA_ERR_BAD_MASK);
     CHECK(fa_fwd(p, p, p, p, f, 1, 1, 128, 128, -1.0f, 0, 0, NULL, 0), FA_ERR_BAD_SCALE);
     CHECK(fa_fwd(p, p, p, p, f, 0, 1, 128, 128, 0.1f, 0, 0, NULL, 0), FA_OK);
+    CHECK(fa_fwd_kv(p, p, p, p, f, 1, 1, 128, 512, 128, 0.1f, 1, 0, (const int*)p, NULL, 0),
+          FA_ERR_BAD_SHAPE);
+    CHECK(fa_fwd_kv(p, p, p, p, f, 2, 1, 0, 512, 128, 0.1f, 1, 0, NULL, NULL, 0), FA_OK);
     CHECK(fa_bwd(p, p, p, p, f, p, p, p, p, 1, 1, 128, 128, 0.1f, 0, 0, NULL, NULL, 0, 0),
           FA_ERR_WORKSPACE);
     CHECK(fa_bwd_noalloc(p, p, p, p, f, p, p, p, p, 1, 16, 65537, 128, 0.1f, 0, 0, NULL, 0),

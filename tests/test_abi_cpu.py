@@ -84,7 +84,30 @@ def test_bwd_validation(kw, code):
     assert bwd(**kw) == code
 
 
+def fwd_kv(**kw):
+    args = dict(q=P, k=P, v=P, o=P, lse=P, B=1, H=1, Nq=128, Nk=512, d=128, scale=0.1,
+                causal=1, window=0, cu_seqlens_q=None, cu_seqlens_k=None, stream=0)
+    args.update(kw)
+    return fa.fa_fwd_kv(**args)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(k=None), -1), (dict(lse=None), -1),
+    (dict(d=80), -2),
+    (dict(Nk=-1), -3), (dict(Nq=-1), -3),
+    (dict(cu_seqlens_q=P), -3), (dict(cu_seqlens_k=P), -3),
+    (dict(cu_seqlens_q=P, cu_seqlens_k=P + 2), -4),
+    (dict(v=P + 4), -4),
+    (dict(causal=0, window=8), -5),
+    (dict(scale=float("nan")), -9),
+])
+def test_fwd_kv_validation(kw, code):
+    assert fwd_kv(**kw) == code
+
+
 def test_empty_problems_are_noops():
+    assert fwd_kv(B=0) == 0
+    assert fwd_kv(Nq=0) == 0
     assert fwd(B=0) == 0
     assert fwd(N=0) == 0
     assert bwd(B=0, workspace=None, workspace_bytes=0) == 0
@@ -103,6 +126,9 @@ def test_workspace_size():
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
 def test_valid_call_without_gpu_reports_cuda_error():
     assert fwd() == -7
+    assert fwd_kv() == -7
+    assert fwd_kv(Nk=0) == -7
+    assert fwd_kv(Nk=0, k=None, v=None) == -7      # no key rows: k, v may be NULL
 
 
 def test_noalloc_validation_on_host():
