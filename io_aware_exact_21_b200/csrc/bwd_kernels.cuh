@@ -329,10 +329,12 @@ __device__ __forceinline__ uint32_t bwd_prologue(uint8_t* smem, const BwdBarrier
     }
     sch.g = p.g;
     sch.rows_per_item = C::BM;
+    sch.order = schedule_order(p.g, 0);     // key blocks: fewer queries see later keys
     sch.bprefix = prefix;
     sch.uprefix = prefix + kMaxVarlenSeqs + 1;
     sch.total_units = build_schedule_prefix(p.g, C::BM, prefix, prefix + kMaxVarlenSeqs + 1,
                                             scratch);   // __syncthreads inside
+    schedule_split_tail(sch);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -375,7 +377,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             // ---------------------------------- producer (whole warp) --
             uint32_t cnt = 0, item_it = 0, fix_issued = 0;
             bool ok = true;
-            ItemIter it;
+            ItemIter<true> it;
             int s, h, blk;
             for (; ok && it.next(sch, s, h, blk); ++item_it) {
                 const SeqSpan sp = sch.span(s);
@@ -436,7 +438,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             const uint32_t st_addr = smem_u32(smem + C::OFF_ST);
             uint32_t cnt = 0, item_it = 0;
             bool ok = true;
-            ItemIter it;
+            ItemIter<true> it;
             int s, h, blk;
             for (; ok && it.next(sch, s, h, blk); ++item_it) {
                 const SeqSpan sp = sch.span(s);
@@ -515,7 +517,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
         const uint32_t tP = tmem + lane_base + C::COL_DP + 64 * g;
         uint32_t cnt = 0, item_it = 0;
         bool ok = true;
-        ItemIter it;
+        ItemIter<true> it;
         int s, h, blk;
         for (; ok && it.next(sch, s, h, blk); ++item_it) {
             const SeqSpan sp = sch.span(s);
@@ -712,10 +714,12 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
     Schedule sch;
     sch.g = p.g;
     sch.rows_per_item = C::BM;
+    sch.order = schedule_order(p.g, 1);     // query blocks: later queries see more keys
     sch.bprefix = prefix;
     sch.uprefix = prefix + kMaxVarlenSeqs + 1;
     sch.total_units = build_schedule_prefix(p.g, C::BM, prefix, prefix + kMaxVarlenSeqs + 1,
                                             scratch);   // __syncthreads inside
+    schedule_split_tail(sch);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -729,7 +733,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
             // -------------------------------------------------- producer --
             uint32_t cnt = 0;
             bool ok = true;
-            ItemIter it;
+            ItemIter<true> it;
             int s, h, blk;
             while (ok && it.next(sch, s, h, blk)) {
                 const SeqSpan sp = sch.span(s);
@@ -764,7 +768,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
             const uint32_t st_addr = smem_u32(smem + C::OFF_ST);
             uint32_t cnt = 0, item_it = 0;
             bool ok = true;
-            ItemIter it;
+            ItemIter<true> it;
             int s, h, blk;
             for (; ok && it.next(sch, s, h, blk); ++item_it) {
                 const SeqSpan sp = sch.span(s);
@@ -836,7 +840,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
         const uint32_t tP = tmem + lane_base + C::COL_DP + 64 * g;
         uint32_t cnt = 0, item_it = 0;
         bool ok = true;
-        ItemIter it;
+        ItemIter<true> it;
         int s, h, blk;
         for (; ok && it.next(sch, s, h, blk); ++item_it) {
             const SeqSpan sp = sch.span(s);

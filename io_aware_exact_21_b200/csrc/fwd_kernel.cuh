@@ -129,6 +129,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     Schedule sch;
     sch.g = p.g;
     sch.rows_per_item = C::ROWS;
+    sch.order = 0;                              // pairs only (ItemIter<false>)
     sch.bprefix = prefix;
     sch.uprefix = prefix + kMaxVarlenSeqs + 1;
     sch.total_units = build_schedule_prefix(p.g, C::ROWS, prefix, prefix + kMaxVarlenSeqs + 1,
@@ -149,7 +150,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             bool ok = true;
             bool skipped = false;
             uint32_t skipped_at = 0xffffffffu;
-            ItemIter it;
+            ItemIter<false> it;
             int s, h, blk;
             for (; ok && it.next(sch, s, h, blk); ++item_it) {
                 const SeqSpan sp = sch.span(s);
@@ -228,7 +229,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                             IDESC_O, (accumulate | kk) != 0);
                 }
             };
-            ItemIter it;
+            ItemIter<false> it;
             int s, h, blk;
             for (; ok && it.next(sch, s, h, blk); ++item_it) {
                 const SeqSpan sp = sch.span(s);
@@ -310,7 +311,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         const float sl2 = p.scale_log2;
         uint32_t step = 0, item_it = 0;
         bool ok = true;
-        ItemIter it;
+        ItemIter<false> it;
         int s, h, blk;
         for (; ok && it.next(sch, s, h, blk); ++item_it) {
             const SeqSpan sp = sch.span(s);

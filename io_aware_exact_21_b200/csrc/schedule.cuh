@@ -78,15 +78,35 @@ __device__ __forceinline__ bool tile_needs_mask(int r0, int BM, int k0, int BN, 
 }
 
 // Static persistent schedule.  The rows of a (sequence, head) are cut into
-// blocks of `rows_per_item` rows; a work unit is the pair of blocks p and
-// nb-1-p of one (sequence, head) (the middle block alone when nb is odd), so
-// that under a causal mask -- where a block's cost grows or shrinks linearly
-// with its index -- every unit costs the same.  Units are ordered sequence-
-// major, then head, then p, so the CTAs running at the same time share K/V of
-// few heads in L2; unit w goes to CTA w % gridDim.x.
+// blocks of `rows_per_item` rows, and each CTA walks its own list of blocks;
+// every role of a CTA walks the same list independently.
+//
+// Pairs: a work unit is the pair of blocks p and nb-1-p of one (sequence,
+// head) (the middle block alone when nb is odd), so that under a causal mask
+// -- where a block's cost grows or shrinks linearly with its index -- every
+// unit costs the same.  Units are ordered sequence-major, then head, then p,
+// so the CTAs running at the same time share K/V of few heads in L2; unit w
+// goes to CTA w % gridDim.x.  This is the whole schedule for packed batches
+// and for fixed length without a causal or window mask.
+//
+// Pairs + snake tail (the backward kernels, for fixed length with a causal or
+// window mask, where a block's cost is monotone in its index; the forward
+// kernel keeps pairs alone): when the units per CTA are few, the
+// last round of units leaves up to a unit's worth of imbalance.  So only the
+// whole heads that fit in all rounds but the last go out as units; the blocks
+// of the remaining heads are sorted heaviest first (block index major, then
+// head) and dealt one by one in rounds of gridDim.x CTAs, forwards in even
+// rounds and backwards in odd ones, starting at the CTA after the last unit.
+// `order` is +1 when cost grows with the block index (query blocks), -1 when
+// it shrinks (key blocks), 0 for pairs alone.
 struct Schedule {
     Geometry g;
     int rows_per_item;
+    int order;              // 0: pairs; +1 / -1: snake tail, heaviest block last / first
+    int bulk_units;         // snake tail: units dealt as pairs
+    int tail_sh0;           // snake tail: first (sequence, head) of the tail
+    int tail_heads;         //   (sequence, head)s in the tail
+    int tail_c0;            //   CTA that takes the tail's first block
     const int* bprefix;     // shared memory: blocks of the sequences before s (packed only)
     const int* uprefix;     // shared memory: units of the sequences before s (packed only)
     int total_units;
@@ -142,13 +162,19 @@ struct Schedule {
     }
 };
 
-// Walks the blocks one CTA processes: its units in order, both blocks of each.
+// Walks the blocks one CTA processes: its units in order, both blocks of each
+// (pairs), then, with kTail and a non-zero order, its blocks of the snake
+// tail round by round.  Without kTail the walk is pairs alone (no tail state
+// is kept: the forward kernel's roles have no registers to spare).
+template <bool kTail>
 struct ItemIter {
-    int w;
+    int w;        // pairs: next unit
     int half;
-    __device__ __forceinline__ ItemIter() : w(blockIdx.x), half(0) {}
+    int round;    // snake: next round
+    __device__ __forceinline__ ItemIter() : w(blockIdx.x), half(0), round(0) {}
     __device__ __forceinline__ bool next(const Schedule& sch, int& s, int& h, int& blk) {
-        while (w < sch.total_units) {
+        const int limit = (kTail && sch.order != 0) ? sch.bulk_units : sch.total_units;
+        while (w < limit) {
             int p, nb;
             sch.unit(w, s, h, p, nb);
             if (half == 0) {
@@ -163,9 +189,45 @@ struct ItemIter {
                 return true;
             }
         }
-        return false;
+        if (!kTail || sch.order == 0) return false;
+        const int G = gridDim.x;
+        const int x0 = (static_cast<int>(blockIdx.x) - sch.tail_c0 + G) % G;
+        const int r = round * G + ((round & 1) ? G - 1 - x0 : x0);
+        const int nb = sch.blocks_of(sch.g.N);
+        if (r >= sch.tail_heads * nb) return false;
+        ++round;
+        const int q = r / sch.tail_heads;              // rank of the block index, heaviest first
+        const int sh = sch.tail_sh0 + (r - q * sch.tail_heads);
+        blk = sch.order > 0 ? nb - 1 - q : q;
+        s = sh / sch.g.H;
+        h = sh - s * sch.g.H;
+        return true;
     }
 };
+
+// Fill in the snake-tail split (see Schedule) once total_units is known.
+__device__ __forceinline__ void schedule_split_tail(Schedule& sch) {
+    sch.bulk_units = sch.total_units;
+    sch.tail_sh0 = 0;
+    sch.tail_heads = 0;
+    sch.tail_c0 = 0;
+    if (sch.order == 0) return;
+    const int G = gridDim.x;
+    const int nu = (sch.blocks_of(sch.g.N) + 1) >> 1;
+    if (nu == 0) return;
+    const int rounds = max(0, sch.total_units / G - 1);
+    sch.bulk_units = (rounds * G / nu) * nu;
+    sch.tail_sh0 = sch.bulk_units / nu;
+    sch.tail_heads = sch.g.B * sch.g.H - sch.tail_sh0;
+    sch.tail_c0 = sch.bulk_units % G;
+}
+
+// The order a kernel uses: snake for fixed length under a causal or window
+// mask, with the direction in which its blocks' cost grows; pairs otherwise.
+__device__ __forceinline__ int schedule_order(const Geometry& g, int cost_grows_with_index) {
+    if (g.cu_seqlens || (!g.causal && g.window <= 0)) return 0;
+    return cost_grows_with_index ? 1 : -1;
+}
 
 // Build the per-sequence block and unit prefixes in shared memory (packed
 // batches only) and return the number of work units.  All threads of the CTA
