@@ -14,6 +14,11 @@ replicas (no collective: the (sequence, head) units share nothing).
 no runnable reference implementation) on a bounded sample of the same
 workload on the host cores.
 
+--workload decode measures decode against a padded K/V cache
+(fa_fwd_kvcache: B=16, H=16, one query per sequence, caches of 4096..8192
+tokens in an 8192-row buffer, d=128) in GB/s of cache read against the HBM
+roofline.
+
 --workload prefill_kv measures the cached-KV prefill forward instead
 (fa_fwd_kv: B=4, H=16, 2048 new query tokens after 6144 cached ones, so
 Nk=8192, d=128, causal aligned bottom-right), with its own oracle sample.
@@ -490,6 +495,167 @@ def run_prefill_kv(args, rank, world, device):
     }
 
 
+# ------------------------------------------------------------ decode arm ---
+
+DECODE_UNIT = "GB/s"
+DECODE_METRIC = "attention decode: K/V-cache bytes read per second (BF16, d=128), % of measured HBM bandwidth"
+
+
+def decode_workload():
+    from io_aware_exact_21_b200.inputs import WORKLOADS
+    return WORKLOADS["decode"]
+
+
+def decode_bytes(wl, lens):
+    """Algorithmic HBM bytes of one decode call: the used K and V rows of every
+    (sequence, head), plus Q read and O, LSE written."""
+    kv = 2 * int(sum(int(n) for n in lens)) * wl.H * wl.d * 2
+    qo = 2 * wl.B * wl.N * wl.H * wl.d * 2 + wl.B * wl.H * wl.N * 4
+    return kv + qo
+
+
+def decode_config(wl, extra=None):
+    cfg = {"workload": "decode B%d H%d Nq%d cache %d..%d of %d rows d%d, bottom-right causal" % (
+        wl.B, wl.H, wl.N, wl.cache_lens[0], wl.cache_lens[1], wl.Nk, wl.d),
+        "B": wl.B, "H": wl.H, "Nq": wl.N, "Nk": wl.Nk, "cache_lens": list(wl.cache_lens),
+        "d": wl.d, "causal": wl.causal, "seed": wl.seed,
+        "l2": "cache larger than L2 (K, V about 400 MB each); L2 not flushed"}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+def run_decode(args, rank, world, device):
+    import io_aware_exact_21_b200 as fa
+    wl = decode_workload()
+    host = wl.make()
+    q, k, v = (host[n].to(device) for n in ("q", "k", "v"))
+    lens = host["seqlens_k"].to(device)
+    B, H, Nq, Nk, d = wl.B, wl.H, wl.N, wl.Nk, wl.d
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=device)
+    ns = fa.fa_fwd_kvcache_num_splits(B, H, Nq, Nk, d)
+    ws = torch.empty(max(16, fa.fa_fwd_kvcache_workspace_size(B, H, Nq, d, ns)), dtype=torch.uint8,
+                     device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(qq, ll, oo, ls):
+        fa.forward_kvcache(qq, k, v, seqlens_k=ll, causal=wl.causal, window=wl.window,
+                           num_splits=ns, out=oo, lse=ls, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step(q, lens, o, lse)
+    torch.cuda.synchronize(device)
+    assert fa.fa_get_device_error() == 0
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    clocks = ClockSampler(device)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize(device)
+    fa.fa_profile_begin()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step(q, lens, o, lse)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    elapsed = e0.elapsed_time(e1)
+    prof = fa.fa_profile_end()
+    clk = clocks.stop()
+    assert fa.fa_get_device_error() == 0
+
+    # end to end: per step the new query and the cache lengths come from pinned
+    # host memory and O, LSE go back (the cache stays resident, as in decoding)
+    pin_q = host["q"].pin_memory()
+    pin_l = host["seqlens_k"].pin_memory()
+    dq_in = torch.empty_like(q)
+    dl_in = torch.empty_like(lens)
+    host_o = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    host_l = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    h2d = pin_q.numel() * pin_q.element_size() + pin_l.numel() * pin_l.element_size()
+    d2h = host_o.numel() * host_o.element_size() + host_l.numel() * host_l.element_size()
+
+    def e2e_step():
+        dq_in.copy_(pin_q, non_blocking=True)
+        dl_in.copy_(pin_l, non_blocking=True)
+        step(dq_in, dl_in, o, lse)
+        host_o.copy_(o, non_blocking=True)
+        host_l.copy_(lse, non_blocking=True)
+
+    e2e_steps = max(2, args.steps)
+    e2e_step()
+    torch.cuda.synchronize(device)
+    barrier()
+    e2 = torch.cuda.Event(enable_timing=True)
+    e3 = torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e3.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    e2e_elapsed = e2.elapsed_time(e3)
+    assert fa.fa_get_device_error() == 0
+
+    elapsed, e2e_elapsed = max_over_ranks([elapsed, e2e_elapsed], world, device)
+    if rank != 0:
+        return None
+    nbytes = decode_bytes(wl, host["seqlens_k"].tolist())
+    value = nbytes * world * args.steps / (elapsed * 1e-3) / 1e9
+    e2e_value = nbytes * world * e2e_steps / (e2e_elapsed * 1e-3) / 1e9
+    dec_ms, dec_n = prof["decode"]
+    cmb_ms, cmb_n = prof["combine"]
+    kernel_ms = dec_ms / dec_n
+    peaks, peak_src = load_peaks()
+    peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    # the decode kernel reads the K/V rows and Q; the merge kernel the partials
+    dec_bytes = nbytes - B * H * Nq * (d * 2 + 4)
+    achieved = dec_bytes / (kernel_ms * 1e-3) / 1e9
+    return {
+        "metric": DECODE_METRIC, "value": round(value, 1), "unit": DECODE_UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(elapsed / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: i.i.d. N(0,1) bf16 Q, K/V cache (seeded), cache lengths seeded uniform",
+        "config": decode_config(wl, {"parallelism": "replicas" if world > 1 else "single GPU",
+                                     "num_splits": ns}),
+        "kernels_ms": {"decode": round(kernel_ms, 5),
+                       "merge": round(cmb_ms / cmb_n, 5) if cmb_n else None},
+        "roofline": {"kernel": "decode", "bound": "hbm", "achieved": round(achieved, 1),
+                     "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "peak_source": "%s hbm_gbs (copy bandwidth)" % peak_src,
+                     "traffic": None,
+                     "traffic_unit": "bytes per launch (ncu dram read + write)"},
+        "e2e": {"value": round(e2e_value, 1), "unit": DECODE_UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "how": "pinned host -> device copy of the new queries and cache lengths, device -> "
+                       "host copy of O and LSE every step, in order on the compute stream; the "
+                       "cache stays resident"},
+        "gpu_launches": sum(c for (_, c) in prof.values()),
+        "clocks": clk,
+    }
+
+
+def oracle_sample_decode():
+    """The float64 oracle's decode on the whole decode workload."""
+    from oracle import oracle as orc
+    wl = decode_workload()
+    x = wl.make()
+    t0 = time.perf_counter()
+    orc.fwd_kvcache(x["q"], x["k"], x["v"], wl.scale, seqlens_k=x["seqlens_k"],
+                    causal=wl.causal, window=wl.window)
+    secs = time.perf_counter() - t0
+    nbytes = decode_bytes(wl, x["seqlens_k"].tolist())
+    desc = ("decode of the whole workload (B%d H%d, caches %d..%d): %.2f s on %d threads"
+            % (wl.B, wl.H, wl.cache_lens[0], wl.cache_lens[1], secs, orc.num_threads()))
+    return nbytes / secs / 1e9, desc, orc.num_threads(), secs
+
+
 def oracle_sample_kv(n_q=None, seed=5):
     """Time the float64 oracle's cached-KV forward on one (sequence, head) of
     the prefill workload, optionally with fewer queries (the key length and
@@ -540,6 +706,26 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return None
+    if args.workload == "decode":
+        for _ in range(args.warmup):
+            oracle_sample_decode()
+        vals = []
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            val, desc, threads, _ = oracle_sample_decode()
+            vals.append(val)
+        elapsed = time.perf_counter() - t0
+        value = statistics.mean(vals)
+        return {"impl": "reference", "metric": DECODE_METRIC, "value": value, "unit": DECODE_UNIT,
+                "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": elapsed * 1e3 / max(1, args.steps),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic: i.i.d. N(0,1) bf16 inputs upcast to float64",
+                "config": decode_config(decode_workload(), {"parallelism": "host cores"}),
+                "cpu_baseline": {"value": value, "unit": DECODE_UNIT, "cores": threads,
+                                 "kind": "oracle", "sample": desc},
+                "e2e": {"value": value, "unit": DECODE_UNIT, "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
     kv = args.workload == "prefill_kv"
     for _ in range(args.warmup):
         if kv:
@@ -576,9 +762,9 @@ def main():
     ap.add_argument("--shape", default=None,
                     help="B,H,N,d override of the workload (profiling of smaller cases)")
     ap.add_argument("--causal", action="store_true", help="causal mask (profiling)")
-    ap.add_argument("--workload", choices=["train", "prefill_kv"], default="train",
+    ap.add_argument("--workload", choices=["train", "prefill_kv", "decode"], default="train",
                     help="train: forward+backward step (default); prefill_kv: cached-KV "
-                         "prefill forward")
+                         "prefill forward; decode: decode against a K/V cache")
     args = ap.parse_args()
     if args.shape:
         B, H, N, d = (int(x) for x in args.shape.split(","))
@@ -605,13 +791,15 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                              device_id=device)
-    kv = args.workload == "prefill_kv"
+    runner = {"train": run_ours, "prefill_kv": run_prefill_kv, "decode": run_decode}[args.workload]
+    sampler = {"train": oracle_sample, "prefill_kv": oracle_sample_kv,
+               "decode": oracle_sample_decode}[args.workload]
     try:
-        out = (run_prefill_kv if kv else run_ours)(args, rank, world, device)
+        out = runner(args, rank, world, device)
         if out is not None:
             if not args.no_cpu_baseline and world == 1:
-                val, desc, threads, secs = oracle_sample_kv() if kv else oracle_sample()
-                out["cpu_baseline"] = {"value": val, "unit": UNIT, "cores": threads,
+                val, desc, threads, secs = sampler()
+                out["cpu_baseline"] = {"value": val, "unit": out["unit"], "cores": threads,
                                        "kind": "oracle", "sample": desc}
             else:
                 out["cpu_baseline"] = None

@@ -121,6 +121,52 @@ int fa_fwd_kv(const void* q, const void* k, const void* v, void* o, float* lse,
               const int* cu_seqlens_q, const int* cu_seqlens_k, cudaStream_t stream);
 
 /*
+ * Decode against a key/value cache, split along the keys.  A few new queries
+ * per sequence (one per generated token; several for speculative decoding or
+ * a short chunk) attend to the sequence's cached keys and values.  The pages
+ * single out this shape: each step reads the whole accumulated K/V cache, so
+ * it is bound by the cache's bandwidth rather than by matrix throughput
+ * (IO-aware essay, section on training, prefill and per-token decode, and its
+ * scenario table), and they list inference with cached keys and values among
+ * the interfaces (FlashAttention encyclopedia page, "software integration").
+ *
+ * q, o    : [B, Nq, H, d] bf16 (1 <= Nq <= 16; Nq = 0 is a no-op).
+ * k_cache, v_cache : [B, Nk, H, d] bf16; sequence b uses rows 0 .. nk_b - 1
+ *           of its slice, nk_b = seqlens_k[b] (device int32 [B], clamped to
+ *           [0, Nk]) or Nk when seqlens_k is NULL.  Rows past nk_b are never
+ *           used (they may hold anything).  k_cache and v_cache may be NULL
+ *           when B * Nk = 0.
+ * lse     : [B, H, Nq] fp32, natural log.
+ * Masks   : as fa_fwd_kv with the queries at the last Nq positions of the
+ *           nk_b keys: query i is at position nk_b - Nq + i.
+ * Splits  : the keys of each (sequence, head) are cut into num_splits
+ *           contiguous ranges that run as separate CTAs (so that few
+ *           sequences still fill the GPU); each writes a partial output and
+ *           log-sum-exp to `workspace`, and a second kernel merges them.
+ *           num_splits = 0 lets the library choose
+ *           (fa_fwd_kvcache_num_splits returns that choice); 1 writes o and
+ *           lse directly and needs no workspace; at most 32.
+ * workspace : device memory of at least fa_fwd_kvcache_workspace_size(B, H,
+ *           Nq, d, splits) bytes, 16-byte aligned, for splits > 1 (NULL
+ *           otherwise); contents on entry do not matter.
+ * Errors as fa_fwd; Nq > 16 or num_splits outside [0, 32] is
+ * FA_ERR_BAD_SHAPE, a missing or short workspace FA_ERR_WORKSPACE.
+ */
+int fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, void* o,
+                   float* lse, int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                   int window, const int* seqlens_k, int num_splits, void* workspace,
+                   size_t workspace_bytes, cudaStream_t stream);
+
+/* The split count fa_fwd_kvcache uses for num_splits = 0 on the current
+ * device (1 for empty problems). */
+int fa_fwd_kvcache_num_splits(int B, int H, int Nq, int Nk, int d);
+
+/* Workspace bytes fa_fwd_kvcache needs for `num_splits` splits:
+ * num_splits * B * Nq * H * (d + 1) * 4 rounded up to 256, or 0 when
+ * num_splits <= 1 or the problem is empty. */
+size_t fa_fwd_kvcache_workspace_size(int B, int H, int Nq, int d, int num_splits);
+
+/*
  * Bytes of device workspace fa_bwd needs: 8 bytes per (head, row) for the
  * per-row statistics {-LSE_i * log2(e), D_i = rowsum(dO_i * O_i)}, stored with
  * every sequence padded to a multiple of 128 rows.  Fixed length:
@@ -189,15 +235,17 @@ int fa_get_device_error(cudaStream_t stream);
 
 /*
  * Per-kernel device timing.  fa_profile_begin() resets the counters and makes
- * the following fa_fwd / fa_bwd calls on the calling thread's current device
+ * the following calls of the entry points above on the calling thread's current device
  * record a CUDA event pair on the launch stream around each kernel they launch
  * (up to 1024 launches per kernel kind; later ones are not recorded).
  * fa_profile_end() waits for the recorded events, stops recording, and writes
- * for each kind k (0 forward, 1 D pre-pass, 2 dK/dV, 3 dQ) the summed device
- * milliseconds ms[k] and the number of recorded launches counts[k].
+ * for each kind k (0 forward, 1 D pre-pass, 2 dK/dV, 3 dQ, 4 decode, 5 decode
+ * split merge) the summed device milliseconds ms[k] and the number of
+ * recorded launches counts[k] (arrays of FA_PROFILE_KINDS entries).
  * Either output pointer may be NULL.  The events are created once per device
  * on the first fa_profile_begin() call.
  */
+#define FA_PROFILE_KINDS 6
 int fa_profile_begin(void);
 int fa_profile_end(double* ms, int* counts);
 

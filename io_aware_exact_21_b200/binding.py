@@ -26,6 +26,10 @@ _VP, _I, _F, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_
 SIGNATURES = {
     "fa_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _I, _VP, _VP]),
     "fa_fwd_kv": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _I, _VP, _VP, _VP]),
+    "fa_fwd_kvcache": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _I, _VP, _I,
+                            _VP, _SZ, _VP]),
+    "fa_fwd_kvcache_num_splits": (_I, [_I, _I, _I, _I, _I]),
+    "fa_fwd_kvcache_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "fa_bwd_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "fa_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _I,
                     _VP, _VP, _SZ, _VP]),
@@ -38,7 +42,7 @@ SIGNATURES = {
     "fa_profile_end": (_I, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]),
 }
 
-PROFILE_KINDS = ("fwd", "dot", "dkdv", "dq")
+PROFILE_KINDS = ("fwd", "dot", "dkdv", "dq", "decode", "combine")   # FA_PROFILE_KINDS order
 
 
 class FaError(RuntimeError):
@@ -114,6 +118,24 @@ def fa_fwd_kv(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, window, cu_seqlen
                                     _stream(stream))
 
 
+def fa_fwd_kvcache(q, k_cache, v_cache, o, lse, B, H, Nq, Nk, d, scale, causal, window,
+                   seqlens_k, num_splits, workspace, workspace_bytes, stream=None) -> int:
+    return load_library().fa_fwd_kvcache(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o),
+                                         _ptr(lse), int(B), int(H), int(Nq), int(Nk), int(d),
+                                         float(scale), int(causal), int(window), _ptr(seqlens_k),
+                                         int(num_splits), _ptr(workspace), int(workspace_bytes),
+                                         _stream(stream))
+
+
+def fa_fwd_kvcache_num_splits(B, H, Nq, Nk, d) -> int:
+    return int(load_library().fa_fwd_kvcache_num_splits(int(B), int(H), int(Nq), int(Nk), int(d)))
+
+
+def fa_fwd_kvcache_workspace_size(B, H, Nq, d, num_splits) -> int:
+    return int(load_library().fa_fwd_kvcache_workspace_size(int(B), int(H), int(Nq), int(d),
+                                                            int(num_splits)))
+
+
 def fa_bwd_workspace_size(B, H, N, d, varlen_total=0) -> int:
     return int(load_library().fa_bwd_workspace_size(int(B), int(H), int(N), int(d),
                                                     int(varlen_total)))
@@ -156,8 +178,8 @@ def fa_profile_begin() -> int:
 def fa_profile_end():
     """Returns {kind: (total_ms, launches)} for the launches recorded since
     fa_profile_begin()."""
-    ms = (ctypes.c_double * 4)()
-    cnt = (ctypes.c_int * 4)()
+    ms = (ctypes.c_double * len(PROFILE_KINDS))()
+    cnt = (ctypes.c_int * len(PROFILE_KINDS))()
     _check(load_library().fa_profile_end(ms, cnt), "fa_profile_end")
     return {k: (ms[i], cnt[i]) for i, k in enumerate(PROFILE_KINDS)}
 
@@ -210,6 +232,32 @@ def forward_kv(q, k, v, causal=False, window=0, cu_seqlens_q=None, cu_seqlens_k=
                           device=q.device)
     _check(fa_fwd_kv(q, k, v, out, lse, B, H, Nq, Nk, d, scale, causal, window, cu_seqlens_q,
                      cu_seqlens_k, stream), "fa_fwd_kv")
+    return out, lse
+
+
+def forward_kvcache(q, k_cache, v_cache, seqlens_k=None, causal=False, window=0, scale=None,
+                    num_splits=0, out=None, lse=None, workspace=None, stream=None):
+    """Decode: q [B, Nq, H, d] (Nq <= 16) against k_cache, v_cache [B, Nk, H, d],
+    of which sequence b uses its first seqlens_k[b] rows (int32 CUDA tensor, or
+    None for all Nk); queries are the last Nq of those positions.  Returns
+    (O, LSE)."""
+    import torch
+    B, Nq, H, d = q.shape
+    Nk = k_cache.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    ns = num_splits if num_splits > 0 else fa_fwd_kvcache_num_splits(B, H, Nq, Nk, d)
+    need = fa_fwd_kvcache_workspace_size(B, H, Nq, d, ns)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _check(fa_fwd_kvcache(q, k_cache, v_cache, out, lse, B, H, Nq, Nk, d, scale, causal, window,
+                          seqlens_k, ns, workspace,
+                          0 if workspace is None else workspace.numel(), stream),
+           "fa_fwd_kvcache")
     return out, lse
 
 

@@ -3,12 +3,14 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
 
 #include "../../include/fa.h"
 #include "bwd_kernels.cuh"
+#include "decode_kernel.cuh"
 #include "fwd_kernel.cuh"
 
 namespace {
@@ -20,14 +22,14 @@ constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;
 
 // ----------------------------------------------------------- profiling --
 // Event pairs recorded around each launch while profiling is on.
-constexpr int kProfKinds = 4;          // forward, D pre-pass, dK/dV, dQ
+constexpr int kProfKinds = 6;          // forward, D pre-pass, dK/dV, dQ, decode, combine
 constexpr int kProfCap = 1024;
 struct Profiler {
     bool created = false;
     bool on = false;
     int device = -1;
     cudaEvent_t ev[kProfKinds][kProfCap][2];
-    int n[kProfKinds] = {0, 0, 0, 0};
+    int n[kProfKinds] = {};
 };
 thread_local Profiler g_prof;
 
@@ -65,6 +67,22 @@ cudaError_t allow_smem(K kernel, int bytes) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
+template <int D>
+cudaError_t decode_set_smem_limits_d() {
+    const int b = fa::DecCfg<D>::SMEM_BYTES;
+    cudaError_t e = allow_smem(fa::decode_kernel<D, 1>, b);
+    if (e == cudaSuccess) e = allow_smem(fa::decode_kernel<D, 2>, b);
+    if (e == cudaSuccess) e = allow_smem(fa::decode_kernel<D, 4>, b);
+    if (e == cudaSuccess) e = allow_smem(fa::decode_kernel<D, 8>, b);
+    if (e == cudaSuccess) e = allow_smem(fa::decode_kernel<D, 16>, b);
+    return e;
+}
+
+cudaError_t decode_set_smem_limits() {
+    cudaError_t e = decode_set_smem_limits_d<64>();
+    return e == cudaSuccess ? decode_set_smem_limits_d<128>() : e;
+}
+
 // Per-device one-time set-up: SM count, the device address of the error word,
 // the driver's tensor-map encoder and the kernels' shared-memory limits.
 int device_setup(DeviceState** out) {
@@ -90,6 +108,7 @@ int device_setup(DeviceState** out) {
         }
         if (allow_smem(fa::fwd_kernel<64>, fa::FwdCfg<64>::SMEM_BYTES) != cudaSuccess ||
             allow_smem(fa::fwd_kernel<128>, fa::FwdCfg<128>::SMEM_BYTES) != cudaSuccess ||
+            decode_set_smem_limits() != cudaSuccess ||
             fa::bwd_set_smem_limits() != cudaSuccess)
             return FA_ERR_CUDA;
         st.ready = true;
@@ -153,6 +172,68 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
     fa::fwd_kernel<D><<<grid, fa::FwdCfg<D>::THREADS, fa::FwdCfg<D>::SMEM_BYTES, stream>>>(
         mq, mk, mv, p);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// ------------------------------------------------------ decode / split-KV --
+// Split count for a decode call: each split gets at least 4 key tiles (256
+// keys); among the counts up to that limit, the smallest whose CTAs fill the
+// GPU's slots (two CTAs per SM) to at least 90 % of whole waves, else the
+// best-filling one.
+int decode_splits(int B, int H, int Nk, int num_sms) {
+    const int64_t items = static_cast<int64_t>(B) * H;
+    const int tiles = (Nk + 63) / 64;
+    const int max_ns = std::max(1, std::min(fa::kDecMaxSplits, tiles / 4));
+    const int64_t slots = 2 * static_cast<int64_t>(num_sms);
+    int best = 1;
+    double best_fill = -1.0;
+    for (int ns = 1; ns <= max_ns; ++ns) {
+        const int64_t ctas = items * ns;
+        const int64_t waves = (ctas + slots - 1) / slots;
+        const double fill = static_cast<double>(ctas) / static_cast<double>(waves * slots);
+        if (fill >= 0.9) return ns;
+        if (fill > best_fill + 1e-9) {
+            best_fill = fill;
+            best = ns;
+        }
+    }
+    return best;
+}
+
+size_t decode_workspace_bytes(int B, int H, int Nq, int d, int ns) {
+    if (ns <= 1) return 0;
+    const size_t rows = static_cast<size_t>(B) * Nq;
+    const size_t bytes = static_cast<size_t>(ns) * rows * H * (static_cast<size_t>(d) + 1) * 4;
+    return (bytes + 255) & ~static_cast<size_t>(255);
+}
+
+template <int D>
+int launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const fa::DecodeParams& p,
+                  cudaStream_t stream) {
+    const int grid = p.B * p.H * p.nsplit;
+    constexpr int T = fa::DecCfg<D>::THREADS, S = fa::DecCfg<D>::SMEM_BYTES;
+    const int slot = prof_start(4, stream);
+    if (p.Nq <= 1)
+        fa::decode_kernel<D, 1><<<grid, T, S, stream>>>(mk, mv, p);
+    else if (p.Nq <= 2)
+        fa::decode_kernel<D, 2><<<grid, T, S, stream>>>(mk, mv, p);
+    else if (p.Nq <= 4)
+        fa::decode_kernel<D, 4><<<grid, T, S, stream>>>(mk, mv, p);
+    else if (p.Nq <= 8)
+        fa::decode_kernel<D, 8><<<grid, T, S, stream>>>(mk, mv, p);
+    else
+        fa::decode_kernel<D, 16><<<grid, T, S, stream>>>(mk, mv, p);
+    prof_stop(4, slot, stream);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    if (p.nsplit > 1) {
+        const int64_t warps = static_cast<int64_t>(p.B) * p.Nq * p.H;
+        const int blocks = static_cast<int>((warps + 7) / 8);
+        const int slot2 = prof_start(5, stream);
+        fa::combine_kernel<D><<<blocks, 256, 0, stream>>>(p.o_part, p.lse_part, p.o, p.lse,
+                                                           p.B * p.Nq, p.H, p.Nq, p.nsplit);
+        prof_stop(5, slot2, stream);
+        if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    }
+    return FA_OK;
 }
 
 // ------------------------------------------------ allocation-free backward --
@@ -249,6 +330,84 @@ int fa_fwd_kv(const void* q, const void* k, const void* v, void* o, float* lse, 
                  : launch_fwd<128>(mq, mk, mv, p, grid, stream);
     prof_stop(0, slot, stream);
     return rc;
+}
+
+int fa_fwd_kvcache_num_splits(int B, int H, int Nq, int Nk, int d) {
+    (void)Nq;
+    (void)d;
+    if (B <= 0 || H <= 0 || Nk <= 0) return 1;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+    return decode_splits(B, H, Nk, sms);
+}
+
+size_t fa_fwd_kvcache_workspace_size(int B, int H, int Nq, int d, int num_splits) {
+    if (B <= 0 || H <= 0 || Nq <= 0 || d <= 0) return 0;
+    return decode_workspace_bytes(B, H, Nq, d, num_splits);
+}
+
+int fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                   int B, int H, int Nq, int Nk, int d, float scale, int causal, int window,
+                   const int* seqlens_k, int num_splits, void* workspace, size_t workspace_bytes,
+                   cudaStream_t stream) {
+    if (!q || !o || !lse) return FA_ERR_NULLPTR;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED_D;
+    if (B < 0 || H <= 0 || Nq < 0 || Nk < 0 || Nq > fa::kDecMaxQ) return FA_ERR_BAD_SHAPE;
+    if (num_splits < 0 || num_splits > fa::kDecMaxSplits) return FA_ERR_BAD_SHAPE;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_BAD_SCALE;
+    if (window > 0 && !causal) return FA_ERR_BAD_MASK;
+    const int64_t rows_q = static_cast<int64_t>(B) * Nq;
+    const int64_t rows_k = static_cast<int64_t>(B) * Nk;
+    if (rows_k > (int64_t{1} << 31) - 1 || rows_k * H * d > (int64_t{1} << 40) ||
+        rows_q * H * d > (int64_t{1} << 40) || static_cast<int64_t>(B) * H * fa::kDecMaxSplits > (int64_t{1} << 31) - 1)
+        return FA_ERR_BAD_SHAPE;
+    if (rows_k > 0 && (!k_cache || !v_cache)) return FA_ERR_NULLPTR;
+    if (misaligned(q) || misaligned(k_cache) || misaligned(v_cache) || misaligned(o) ||
+        misaligned(lse) || (reinterpret_cast<uintptr_t>(seqlens_k) & 3u))
+        return FA_ERR_MISALIGNED;
+    if (rows_q == 0) return FA_OK;
+    auto check_ws = [&](int ns) {
+        const size_t need = decode_workspace_bytes(B, H, Nq, d, ns);
+        if (need == 0) return FA_OK;
+        if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
+        return misaligned(workspace) ? FA_ERR_MISALIGNED : FA_OK;
+    };
+    int rc = num_splits > 0 ? check_ws(num_splits) : FA_OK;
+    if (rc != FA_OK) return rc;
+    DeviceState* st = nullptr;
+    if ((rc = device_setup(&st)) != FA_OK) return rc;
+    const int ns = num_splits > 0 ? num_splits : decode_splits(B, H, Nk, st->num_sms);
+    if ((rc = check_ws(ns)) != FA_OK) return rc;
+    // With no cache rows every split is empty and no tile is loaded; the maps
+    // still need a valid base, so they are pointed at q.
+    const void* kk = rows_k > 0 ? k_cache : q;
+    const void* vv = rows_k > 0 ? v_cache : q;
+    const int64_t map_rows = rows_k > 0 ? rows_k : rows_q;
+    CUtensorMap mk, mv;
+    if (make_map(&mk, kk, map_rows, H, d, 64) || make_map(&mv, vv, map_rows, H, d, 64))
+        return FA_ERR_CUDA;
+
+    fa::DecodeParams p;
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.o_part = ns > 1 ? static_cast<float*>(workspace) : nullptr;
+    p.lse_part = ns > 1 ? static_cast<float*>(workspace) + static_cast<size_t>(ns) * rows_q * H * d
+                        : nullptr;
+    p.seqlens_k = seqlens_k;
+    p.B = B;
+    p.H = H;
+    p.Nq = Nq;
+    p.Nk = Nk;
+    p.causal = causal ? 1 : 0;
+    p.window = window > 0 ? window : 0;
+    p.nsplit = ns;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.error_word = st->error_word;
+    p.timeout_ns = g_fault_timeout_ns ? g_fault_timeout_ns : kDefaultTimeoutNs;
+    return d == 64 ? launch_decode<64>(mk, mv, p, stream) : launch_decode<128>(mk, mv, p, stream);
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d, int varlen_total) {

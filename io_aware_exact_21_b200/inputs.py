@@ -16,7 +16,9 @@ Recipe (the pages fix only "i.i.d. N(0,1) bf16, seed s"):
   * queries against longer cached keys/values: as above, with Q drawn over
     the query rows and K, V over the key rows (fixed ``[B, Nq, H, d]`` and
     ``[B, Nk, H, d]``; packed ``[Tq, H, d]`` and ``[Tk, H, d]`` with
-    ``cu_seqlens_q`` / ``cu_seqlens_k`` from explicit per-sequence lengths).
+    ``cu_seqlens_q`` / ``cu_seqlens_k`` from explicit per-sequence lengths);
+  * decode: Q ``[B, Nq, H, d]``, a padded cache K, V ``[B, Nk, H, d]``, then
+    the used cache rows per sequence from ``torch.randint`` (``kvcache_inputs``).
 """
 from __future__ import annotations
 
@@ -78,6 +80,25 @@ def varlen_kv_inputs(lens_q, lens_k, H: int, d: int, seed: int):
     return out
 
 
+def kvcache_inputs(B: int, Nq: int, Nk: int, H: int, d: int, seed: int, lens=None):
+    """Decode inputs: q [B, Nq, H, d], a padded cache k, v [B, Nk, H, d] and
+    the used cache rows per sequence (``lens`` = (lo, hi) draws them with
+    ``torch.randint(lo, hi + 1, (B,))`` after the tensors; a list fixes them;
+    None leaves all Nk rows in use and ``seqlens_k`` None)."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    shapes = {"q": [B, Nq, H, d], "k": [B, Nk, H, d], "v": [B, Nk, H, d]}
+    out = {n: torch.randn(shp, dtype=torch.float32, generator=g).to(torch.bfloat16)
+           for n, shp in shapes.items()}
+    if lens is None:
+        out["seqlens_k"] = None
+    elif isinstance(lens, tuple):
+        out["seqlens_k"] = torch.randint(lens[0], lens[1] + 1, (B,), generator=g,
+                                         dtype=torch.int64).to(torch.int32)
+    else:
+        out["seqlens_k"] = torch.as_tensor(lens, dtype=torch.int32)
+    return out
+
+
 @dataclass(frozen=True)
 class Workload:
     """One named workload: shapes, seed and mask of a parity or bench case."""
@@ -92,12 +113,16 @@ class Workload:
     varlen: tuple = field(default=None)   # (nseq, lo, hi) for packed inputs
     backward: bool = False
     Nk: int = 0                           # > 0: keys/values per sequence (cached-KV prefill)
+    cache_lens: tuple = None              # (lo, hi): decode against a padded cache of Nk rows
 
     @property
     def scale(self) -> float:
         return 1.0 / math.sqrt(self.d)
 
     def make(self):
+        if self.cache_lens is not None:
+            return kvcache_inputs(self.B, self.N, self.Nk, self.H, self.d, self.seed,
+                                  lens=self.cache_lens)
         if self.Nk > 0:
             return kv_inputs(self.B, self.N, self.Nk, self.H, self.d, self.seed)
         if self.varlen is not None:
@@ -123,6 +148,10 @@ WORKLOADS = {
                               window=1024, varlen=(16, 128, 4096)),
     "bwd_causal": Workload("bwd_causal", B=2, H=16, N=4096, d=128, seed=4, causal=True,
                            backward=True),
+    # one new token per sequence against caches of 4096..8192 tokens
+    # (N is the query count, Nk the cache capacity)
+    "decode": Workload("decode", B=16, H=16, N=1, d=128, seed=6, causal=True, Nk=8192,
+                       cache_lens=(4096, 8192)),
     # a 2048-token prompt chunk after 6144 cached tokens
     "prefill_kv_causal": Workload("prefill_kv_causal", B=4, H=16, N=2048, d=128, seed=5,
                                   causal=True, Nk=8192),

@@ -229,3 +229,27 @@ def fwd_kv(q, k, v, scale, causal=False, window=0, cu_seqlens_q=None, cu_seqlens
     if cu_seqlens_q is None:
         return O.reshape(B, Nq, H, d), L.reshape(H, B, Nq).transpose(1, 0, 2).copy()
     return O, L
+
+
+def fwd_kvcache(q, k_cache, v_cache, scale, seqlens_k=None, causal=False, window=0):
+    """Decode against a padded key/value cache: q [B, Nq, H, d], k_cache and
+    v_cache [B, Nk, H, d] of which sequence b uses its first seqlens_k[b] rows
+    (all Nk when None); the queries are the last Nq of those positions.
+    Returns O [B, Nq, H, d], LSE [B, H, Nq]."""
+    B, Nq, H, d = q.shape
+    Nk = k_cache.shape[1]
+    Q, K, V = (_f64(x).reshape(-1, H, d) for x in (q, k_cache, v_cache))
+    if seqlens_k is None:
+        kl = np.full(B, Nk, dtype=np.int32)
+    else:
+        sk = seqlens_k.cpu() if hasattr(seqlens_k, "cpu") else seqlens_k
+        kl = np.ascontiguousarray(np.clip(np.asarray(sk, dtype=np.int64), 0, Nk), dtype=np.int32)
+    qs = np.ascontiguousarray(np.arange(B, dtype=np.int32) * Nq)
+    ks = np.ascontiguousarray(np.arange(B, dtype=np.int32) * Nk)
+    ql = np.full(B, Nq, dtype=np.int32)
+    O = np.zeros_like(Q)
+    L = np.zeros((H, B * Nq), dtype=np.float64)
+    _check(_load().oracle_fwd_kv(_dp(Q), _dp(K), _dp(V), B * Nq, B * Nk, H, d, B, _ip(qs),
+                                 _ip(ql), _ip(ks), _ip(kl), float(scale), int(bool(causal)),
+                                 int(window), _dp(O), _dp(L)))
+    return O.reshape(B, Nq, H, d), L.reshape(H, B, Nq).transpose(1, 0, 2).copy()

@@ -105,7 +105,44 @@ def test_fwd_kv_validation(kw, code):
     assert fwd_kv(**kw) == code
 
 
+def kvcache(**kw):
+    args = dict(q=P, k_cache=P, v_cache=P, o=P, lse=P, B=2, H=2, Nq=1, Nk=512, d=128, scale=0.1,
+                causal=1, window=0, seqlens_k=None, num_splits=1, workspace=None,
+                workspace_bytes=0, stream=0)
+    args.update(kw)
+    return fa.fa_fwd_kvcache(**args)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), -1), (dict(v_cache=None), -1),
+    (dict(d=96), -2),
+    (dict(Nq=17), -3), (dict(Nk=-1), -3), (dict(num_splits=33), -3), (dict(num_splits=-1), -3),
+    (dict(seqlens_k=P + 2), -4), (dict(o=P + 8), -4),
+    (dict(causal=0, window=4), -5),
+    (dict(scale=0.0), -9),
+    (dict(num_splits=4), -6), (dict(num_splits=4, workspace=P, workspace_bytes=64), -6),
+    (dict(num_splits=4, workspace=P + 4, workspace_bytes=1 << 20), -4),
+])
+def test_kvcache_validation(kw, code):
+    assert kvcache(**kw) == code
+
+
+def test_kvcache_workspace_size_and_splits():
+    # num_splits * B * Nq * H * (d + 1) * 4, rounded to 256; none for one split
+    assert fa.fa_fwd_kvcache_workspace_size(2, 2, 1, 128, 4) == 8448      # 8256 rounded up
+    assert fa.fa_fwd_kvcache_workspace_size(16, 16, 1, 128, 8) == 8 * 16 * 16 * 129 * 4
+    assert fa.fa_fwd_kvcache_workspace_size(2, 2, 1, 128, 1) == 0
+    assert fa.fa_fwd_kvcache_workspace_size(0, 2, 1, 128, 4) == 0
+    assert fa.fa_fwd_kvcache_num_splits(0, 1, 1, 128, 128) == 1
+    ns = fa.fa_fwd_kvcache_num_splits(16, 16, 1, 8192, 128)
+    assert 1 <= ns <= 32
+    # at least 4 key tiles of 64 per split
+    assert fa.fa_fwd_kvcache_num_splits(1, 1, 1, 300, 128) == 1
+
+
 def test_empty_problems_are_noops():
+    assert kvcache(Nq=0) == 0
+    assert kvcache(B=0) == 0
     assert fwd_kv(B=0) == 0
     assert fwd_kv(Nq=0) == 0
     assert fwd(B=0) == 0

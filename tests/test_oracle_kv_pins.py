@@ -100,3 +100,49 @@ def test_packed_equals_separate_and_empty_rows():
     # query 0 of the last sequence sits at position -1: no key, O = 0, LSE = -inf
     assert (O[cq[3]] == 0).all() and np.isneginf(L[:, cq[3]]).all()
     np.testing.assert_allclose(O[cq[3] + 1], v[ck[3]], atol=1e-14)
+
+
+# ------------------------------------------------ padded cache (decode) ---
+
+@pytest.mark.parametrize("causal,window", [(False, 0), (True, 0), (True, 2)])
+def test_kvcache_uses_only_the_first_seqlens_rows(causal, window):
+    # Each sequence's result equals the fixed-length cached-KV forward of the
+    # rows it uses; the unused rows (filled with NaN here) are never read.
+    B, Nq, Nk, H, d = 3, 2, 9, 2, 4
+    q = _rand((B, Nq, H, d), 11)
+    k = _rand((B, Nk, H, d), 12)
+    v = _rand((B, Nk, H, d), 13)
+    lens = np.array([9, 4, 1], dtype=np.int32)
+    for b in range(B):
+        k[b, lens[b]:] = np.nan
+        v[b, lens[b]:] = np.nan
+    O, L = orc.fwd_kvcache(q, k, v, 0.5, seqlens_k=lens, causal=causal, window=window)
+    for b in range(B):
+        n = lens[b]
+        Ob, Lb = _brute_kv(q[b:b + 1], k[b:b + 1, :n], v[b:b + 1, :n], 0.5, causal, window)
+        np.testing.assert_allclose(O[b:b + 1], Ob, rtol=0, atol=1e-12)
+        np.testing.assert_array_equal(np.isneginf(L[b:b + 1]), np.isneginf(Lb))
+        fin = ~np.isneginf(Lb)
+        np.testing.assert_allclose(L[b:b + 1][fin], Lb[fin], rtol=0, atol=1e-12)
+
+
+def test_kvcache_without_seqlens_is_fwd_kv():
+    q = _rand((2, 3, 2, 8), 21)
+    k = _rand((2, 40, 2, 8), 22)
+    v = _rand((2, 40, 2, 8), 23)
+    O1, L1 = orc.fwd_kvcache(q, k, v, 0.3, causal=True)
+    O2, L2 = orc.fwd_kv(q, k, v, 0.3, causal=True)
+    assert np.array_equal(O1, O2) and np.array_equal(L1, L2)
+
+
+def test_kvcache_empty_cache_rows():
+    # nk = 0: no key at all; nk < Nq under causal: the first queries see none
+    q = _rand((2, 3, 1, 4), 31)
+    k = _rand((2, 5, 1, 4), 32)
+    v = _rand((2, 5, 1, 4), 33)
+    O, L = orc.fwd_kvcache(q, k, v, 1.0, seqlens_k=np.array([0, 2], np.int32), causal=True)
+    assert np.all(O[0] == 0) and np.all(np.isneginf(L[0]))
+    # sequence 1: positions -1, 0, 1 -> query 0 sees nothing, query 1 sees key 0
+    assert np.all(O[1, 0] == 0) and np.isneginf(L[1, 0, 0])
+    np.testing.assert_allclose(O[1, 1, 0], v[1, 0, 0], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(L[1, 0, 1], 1.0 * q[1, 1, 0] @ k[1, 0, 0], rtol=0, atol=1e-14)
