@@ -47,26 +47,29 @@ WORKLOAD = dict(B=4, H=16, N=8192, d=128, causal=False, window=0, seed=2)
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
-# one ncu capture of the B=2 H=16 N=8192 d=128 non-causal case, scaled by 2 to
-# the B=4 workload (each kernel's traffic grows with the number of heads it
-# processes).  Valid only for the kernel sources it was taken on: the entry
-# carries a hash of them and is reported as null once they change.
-# Summaries and commands: profiles/*_kernel_B2H16N8192d128.md.
+# ncu captures.  Training step: the B=2 H=16 N=8192 d=128 non-causal case,
+# scaled by 2 to the B=4 workload (each kernel's traffic grows with the number
+# of heads it processes).  Decode: the decode workload itself.  Valid only for
+# the kernel sources a capture was taken on: each entry carries a hash of them
+# and is reported as null once they change.  Summaries and commands:
+# profiles/*_kernel_*.md.
 TRAFFIC = {
-    "fwd": {"bytes_per_launch": 2 * (207.27e6 + 50.36e6), "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh"),
-            "sha": "f46501df6dc6d3e3"},
-    "dkdv": {"bytes_per_launch": 2 * (273.03e6 + 107.20e6),
-             "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "5fe302c77f19a617"},
-    "dq": {"bytes_per_launch": 2 * (271.28e6 + 52.17e6),
-           "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "5fe302c77f19a617"},
+    "fwd": {"bytes_per_launch": 2 * (203.64e6 + 49.21e6), "workload": "train",
+            "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh"), "sha": "b41eb356c35423da"},
+    "dkdv": {"bytes_per_launch": 2 * (272.13e6 + 106.88e6), "workload": "train",
+             "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "81faa9db662491cc"},
+    "dq": {"bytes_per_launch": 2 * (271.25e6 + 53.68e6), "workload": "train",
+           "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "81faa9db662491cc"},
+    "decode": {"bytes_per_launch": 792.91e6 + 4.74e6, "workload": "decode",
+               "sources": ("decode_kernel.cuh", "sm100.cuh"), "sha": "beaec1c610a97f43"},
 }
 
 
-def traffic_for(kernel):
+def traffic_for(kernel, workload="train"):
     """ncu traffic per launch if the kernel's sources still match the capture."""
     import hashlib
     t = TRAFFIC.get(kernel)
-    if not t:
+    if not t or t["workload"] != workload:
         return None
     h = hashlib.sha256()
     try:
@@ -77,9 +80,10 @@ def traffic_for(kernel):
         return None
     if h.hexdigest()[:16] != t["sha"]:
         return None
-    w = WORKLOAD
-    if (w["B"], w["H"], w["N"], w["d"], w["causal"]) != (4, 16, 8192, 128, False):
-        return None
+    if workload == "train":
+        w = WORKLOAD
+        if (w["B"], w["H"], w["N"], w["d"], w["causal"]) != (4, 16, 8192, 128, False):
+            return None
     return t["bytes_per_launch"]
 
 
@@ -629,7 +633,7 @@ def run_decode(args, rank, world, device):
         "roofline": {"kernel": "decode", "bound": "hbm", "achieved": round(achieved, 1),
                      "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "peak_source": "%s hbm_gbs (copy bandwidth)" % peak_src,
-                     "traffic": None,
+                     "traffic": traffic_for("decode", "decode"),
                      "traffic_unit": "bytes per launch (ncu dram read + write)"},
         "e2e": {"value": round(e2e_value, 1), "unit": DECODE_UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
