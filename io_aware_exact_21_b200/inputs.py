@@ -80,6 +80,13 @@ def varlen_kv_inputs(lens_q, lens_k, H: int, d: int, seed: int):
     return out
 
 
+def fp8_signs(seed: int, d: int = 128):
+    """The random sign vector of the FP8 path's rotation: d entries of +-1
+    from ``torch.randint(0, 2, (d,))`` of a generator seeded with ``seed``."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    return (torch.randint(0, 2, (d,), generator=g) * 2 - 1).to(torch.float32)
+
+
 def kvcache_inputs(B: int, Nq: int, Nk: int, H: int, d: int, seed: int, lens=None):
     """Decode inputs: q [B, Nq, H, d], a padded cache k, v [B, Nk, H, d] and
     the used cache rows per sequence (``lens`` = (lo, hi) draws them with

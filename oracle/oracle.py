@@ -28,6 +28,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "attn_oracle.c")
+_SRC_FP8 = os.path.join(_HERE, "fp8_oracle.c")
 _LIB_DIR = os.path.join(_HERE, "_build")
 _LIB = os.path.join(_LIB_DIR, "libattn_oracle.so")
 
@@ -35,12 +36,15 @@ _lib = None
 
 
 def build(force: bool = False) -> str:
-    """Compile ``attn_oracle.c`` into ``oracle/_build/libattn_oracle.so``."""
+    """Compile ``attn_oracle.c`` and ``fp8_oracle.c`` into
+    ``oracle/_build/libattn_oracle.so``.  ``-ffp-contract=off``: the float32
+    steps of the FP8 quantiser must stay single IEEE operations."""
     os.makedirs(_LIB_DIR, exist_ok=True)
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+    newest = max(os.path.getmtime(_SRC), os.path.getmtime(_SRC_FP8))
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < newest:
         tmp = _LIB + ".tmp%d" % os.getpid()
         subprocess.check_call(["gcc", "-O3", "-fopenmp", "-fPIC", "-shared", "-std=c11",
-                               "-o", tmp, _SRC, "-lm"])
+                               "-ffp-contract=off", "-o", tmp, _SRC, _SRC_FP8, "-lm"])
         os.replace(tmp, _LIB)
     return _LIB
 
@@ -66,6 +70,18 @@ def _load():
         for f in (lib.oracle_fwd, lib.oracle_fwd_rows, lib.oracle_fwd_online, lib.oracle_bwd):
             f.restype = ctypes.c_int
         lib.oracle_num_threads.restype = ctypes.c_int
+        fp = ctypes.POINTER(ctypes.c_float)
+        lib.oracle_e4m3_round.argtypes = [ctypes.c_float]
+        lib.oracle_e4m3_round.restype = ctypes.c_float
+        lib.oracle_rotate_rows.argtypes = [fp, ctypes.c_int, ctypes.c_int, fp]
+        lib.oracle_rotate_rows.restype = ctypes.c_int
+        lib.oracle_quantize_fp8.argtypes = [fp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_int, fp, fp, fp]
+        lib.oracle_quantize_fp8.restype = ctypes.c_int
+        lib.oracle_fwd_fp8.argtypes = [fp, fp, fp, fp, fp, fp, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int,
+                                       ctypes.c_int, ctypes.c_int, dp, dp]
+        lib.oracle_fwd_fp8.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -253,3 +269,59 @@ def fwd_kvcache(q, k_cache, v_cache, scale, seqlens_k=None, causal=False, window
                                  _ip(ql), _ip(ks), _ip(kl), float(scale), int(bool(causal)),
                                  int(window), _dp(O), _dp(L)))
     return O.reshape(B, Nq, H, d), L.reshape(H, B, Nq).transpose(1, 0, 2).copy()
+
+
+# ------------------------------------------------------------ FP8 path ---
+# Block-quantised e4m3 forward (see the header of fp8_oracle.c for the steps).
+
+def _f32(x) -> np.ndarray:
+    if hasattr(x, "detach"):
+        x = x.detach().float().cpu().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+
+
+def _fp(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_float))
+
+
+def e4m3_round(x) -> np.ndarray:
+    """Element-wise nearest e4m3 value (ties to even, saturating at 448)."""
+    f = _load().oracle_e4m3_round
+    a = _f32(x)
+    return np.vectorize(lambda v: f(float(v)), otypes=[np.float32])(a) if a.size else a
+
+
+def rotate_rows(x, signs) -> np.ndarray:
+    """Random-sign Walsh-Hadamard rotation of the last axis (d = 128), float32."""
+    a = _f32(x).copy()
+    sg = _f32(signs)
+    rows = a.size // a.shape[-1] if a.size else 0
+    _check(_load().oracle_rotate_rows(_fp(a), rows, a.shape[-1], _fp(sg)))
+    return a
+
+
+def quantize_fp8(x, signs=None):
+    """x [B, N, H, 128] -> (codes [B, N, H, 128] float32 e4m3 values,
+    scales [B, H, ceil(N / 128)] float32); rotated first when signs is given."""
+    a = _f32(x)
+    B, N, H, d = a.shape
+    nb = (N + 127) // 128
+    codes = np.zeros_like(a)
+    scales = np.zeros((B, H, nb), dtype=np.float32)
+    sg = None if signs is None else _f32(signs)
+    _check(_load().oracle_quantize_fp8(_fp(a), B, N, H, d, None if sg is None else _fp(sg),
+                                       _fp(codes), _fp(scales)))
+    return codes, scales
+
+
+def fwd_fp8(qc, kc, vc, sq, sk, sv, scale, causal=False, window=0, quantize_p=True):
+    """FP8 forward from codes and block scales (fixed length [B, N, H, d]).
+    Returns O [B, N, H, d] and LSE [B, H, N] in float64."""
+    q, k, v = _f32(qc), _f32(kc), _f32(vc)
+    B, N, H, d = q.shape
+    o = np.zeros(q.shape, dtype=np.float64)
+    lse = np.zeros((B, H, N), dtype=np.float64)
+    _check(_load().oracle_fwd_fp8(_fp(q), _fp(k), _fp(v), _fp(_f32(sq)), _fp(_f32(sk)),
+                                  _fp(_f32(sv)), B, N, H, d, float(scale), int(bool(causal)),
+                                  int(window), int(bool(quantize_p)), _dp(o), _dp(lse)))
+    return o, lse
