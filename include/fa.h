@@ -167,6 +167,37 @@ int fa_fwd_kvcache_num_splits(int B, int H, int Nq, int Nk, int d);
 size_t fa_fwd_kvcache_workspace_size(int B, int H, int Nq, int d, int num_splits);
 
 /*
+ * FP8 forward (block-quantised e4m3; NOT exact attention -- a separate,
+ * lower-precision path).  The FlashAttention encyclopedia page (FlashAttention-3
+ * paragraph) names an FP8 path with block quantisation and a processing step
+ * that reduces quantisation error, to be kept apart from exact dense attention;
+ * it prints no formulas, and this library reads it as follows (d = 128 and
+ * fixed-length sequences only):
+ *
+ * fa_quantize_fp8: x bf16 [B, N, H, 128] -> e4m3 codes and one float scale per
+ *   block of 128 rows of a head, scales [B, H, ceil(N/128)]: s = amax / 448
+ *   (1 for an all-zero block), code = e4m3(x / s), round to nearest even,
+ *   saturating.  signs (128 floats of +-1, or NULL) selects the
+ *   error-reducing rotation of each row before quantising: multiply by the
+ *   signs, then the orthonormal Walsh-Hadamard transform (q.k is unchanged;
+ *   use the same signs for Q and K).  transpose = 0 writes codes as
+ *   [B, N, H, 128] (use for Q and K); transpose = 1 writes [B, H, 128, Np],
+ *   Np = N rounded up to 16, zeros past N (use for V; signs must be NULL,
+ *   else FA_ERR_BAD_SHAPE).  fa_fp8_vt_bytes gives that buffer's size.
+ * fa_fwd_fp8: O (bf16 [B, N, H, 128]) and LSE ([B, H, N]) from the codes and
+ *   scales: scores use the block scales of Q and K, P is rounded to e4m3
+ *   (after folding in the V block scale relative to the head's largest) for
+ *   the PV GEMM, the row sums use the unrounded P.  Masks as fa_fwd.
+ * Errors as fa_fwd; d != 128 is FA_ERR_UNSUPPORTED_D.
+ */
+size_t fa_fp8_vt_bytes(int B, int H, int N, int d);
+int fa_quantize_fp8(const void* x, void* out, float* scales, int B, int N, int H, int d,
+                    int transpose, const float* signs, cudaStream_t stream);
+int fa_fwd_fp8(const void* q8, const void* k8, const void* vt8, const float* sq,
+               const float* sk, const float* sv, void* o, float* lse, int B, int H, int N,
+               int d, float scale, int causal, int window, cudaStream_t stream);
+
+/*
  * Bytes of device workspace fa_bwd needs: 8 bytes per (head, row) for the
  * per-row statistics {-LSE_i * log2(e), D_i = rowsum(dO_i * O_i)}, stored with
  * every sequence padded to a multiple of 128 rows.  Fixed length:
@@ -240,12 +271,13 @@ int fa_get_device_error(cudaStream_t stream);
  * (up to 1024 launches per kernel kind; later ones are not recorded).
  * fa_profile_end() waits for the recorded events, stops recording, and writes
  * for each kind k (0 forward, 1 D pre-pass, 2 dK/dV, 3 dQ, 4 decode, 5 decode
- * split merge) the summed device milliseconds ms[k] and the number of
- * recorded launches counts[k] (arrays of FA_PROFILE_KINDS entries).
+ * split merge, 6 FP8 quantisation, 7 FP8 forward) the summed device
+ * milliseconds ms[k] and the number of recorded launches counts[k] (arrays of
+ * FA_PROFILE_KINDS entries).
  * Either output pointer may be NULL.  The events are created once per device
  * on the first fa_profile_begin() call.
  */
-#define FA_PROFILE_KINDS 6
+#define FA_PROFILE_KINDS 8
 int fa_profile_begin(void);
 int fa_profile_end(double* ms, int* counts);
 

@@ -30,6 +30,9 @@ SIGNATURES = {
                             _VP, _SZ, _VP]),
     "fa_fwd_kvcache_num_splits": (_I, [_I, _I, _I, _I, _I]),
     "fa_fwd_kvcache_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "fa_fp8_vt_bytes": (_SZ, [_I, _I, _I, _I]),
+    "fa_quantize_fp8": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP, _VP]),
+    "fa_fwd_fp8": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _I, _VP]),
     "fa_bwd_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "fa_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _I,
                     _VP, _VP, _SZ, _VP]),
@@ -42,7 +45,8 @@ SIGNATURES = {
     "fa_profile_end": (_I, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]),
 }
 
-PROFILE_KINDS = ("fwd", "dot", "dkdv", "dq", "decode", "combine")   # FA_PROFILE_KINDS order
+PROFILE_KINDS = ("fwd", "dot", "dkdv", "dq", "decode", "combine", "quant_fp8",
+                 "fwd_fp8")   # FA_PROFILE_KINDS order
 
 
 class FaError(RuntimeError):
@@ -134,6 +138,24 @@ def fa_fwd_kvcache_num_splits(B, H, Nq, Nk, d) -> int:
 def fa_fwd_kvcache_workspace_size(B, H, Nq, d, num_splits) -> int:
     return int(load_library().fa_fwd_kvcache_workspace_size(int(B), int(H), int(Nq), int(d),
                                                             int(num_splits)))
+
+
+def fa_fp8_vt_bytes(B, H, N, d) -> int:
+    return int(load_library().fa_fp8_vt_bytes(int(B), int(H), int(N), int(d)))
+
+
+def fa_quantize_fp8(x, out, scales, B, N, H, d, transpose, signs, stream=None) -> int:
+    return load_library().fa_quantize_fp8(_ptr(x), _ptr(out), _ptr(scales), int(B), int(N),
+                                          int(H), int(d), int(transpose), _ptr(signs),
+                                          _stream(stream))
+
+
+def fa_fwd_fp8(q8, k8, vt8, sq, sk, sv, o, lse, B, H, N, d, scale, causal, window,
+               stream=None) -> int:
+    return load_library().fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(vt8), _ptr(sq), _ptr(sk),
+                                     _ptr(sv), _ptr(o), _ptr(lse), int(B), int(H), int(N),
+                                     int(d), float(scale), int(causal), int(window),
+                                     _stream(stream))
 
 
 def fa_bwd_workspace_size(B, H, N, d, varlen_total=0) -> int:
@@ -258,6 +280,43 @@ def forward_kvcache(q, k_cache, v_cache, seqlens_k=None, causal=False, window=0,
                           seqlens_k, ns, workspace,
                           0 if workspace is None else workspace.numel(), stream),
            "fa_fwd_kvcache")
+    return out, lse
+
+
+def quantize_fp8(q, k, v, signs=None, stream=None):
+    """Block-quantise bf16 q, k, v [B, N, H, 128] for forward_fp8: returns a
+    dict with q8, k8 (uint8 e4m3 codes [B, N, H, 128]), vt8 (uint8 [B, H,
+    128, Np]) and their scales sq, sk, sv [B, H, ceil(N / 128)].  signs (128
+    floats of +-1 on the device) rotates Q and K first."""
+    import torch
+    B, N, H, d = q.shape
+    nb = (N + 127) // 128
+    dev = q.device
+    out = {"q8": torch.empty((B, N, H, d), dtype=torch.uint8, device=dev),
+           "k8": torch.empty((B, N, H, d), dtype=torch.uint8, device=dev),
+           "vt8": torch.empty(max(1, fa_fp8_vt_bytes(B, H, N, d)), dtype=torch.uint8, device=dev),
+           "sq": torch.empty((B, H, nb), dtype=torch.float32, device=dev),
+           "sk": torch.empty((B, H, nb), dtype=torch.float32, device=dev),
+           "sv": torch.empty((B, H, nb), dtype=torch.float32, device=dev)}
+    _check(fa_quantize_fp8(q, out["q8"], out["sq"], B, N, H, d, 0, signs, stream), "fa_quantize_fp8")
+    _check(fa_quantize_fp8(k, out["k8"], out["sk"], B, N, H, d, 0, signs, stream), "fa_quantize_fp8")
+    _check(fa_quantize_fp8(v, out["vt8"], out["sv"], B, N, H, d, 1, None, stream), "fa_quantize_fp8")
+    return out
+
+
+def forward_fp8(qz, B, N, H, d=128, causal=False, window=0, scale=None, out=None, lse=None,
+                stream=None):
+    """FP8 forward from the output of quantize_fp8.  Returns (O bf16, LSE)."""
+    import torch
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dev = qz["q8"].device
+    if out is None:
+        out = torch.empty((B, N, H, d), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    _check(fa_fwd_fp8(qz["q8"], qz["k8"], qz["vt8"], qz["sq"], qz["sk"], qz["sv"], out, lse, B, H,
+                      N, d, scale, causal, window, stream), "fa_fwd_fp8")
     return out, lse
 
 

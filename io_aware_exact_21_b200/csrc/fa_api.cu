@@ -11,6 +11,7 @@
 #include "../../include/fa.h"
 #include "bwd_kernels.cuh"
 #include "decode_kernel.cuh"
+#include "fp8_quant.cuh"
 #include "fwd_kernel.cuh"
 
 namespace {
@@ -22,7 +23,7 @@ constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;
 
 // ----------------------------------------------------------- profiling --
 // Event pairs recorded around each launch while profiling is on.
-constexpr int kProfKinds = 6;          // forward, D pre-pass, dK/dV, dQ, decode, combine
+constexpr int kProfKinds = 8;   // forward, D pre-pass, dK/dV, dQ, decode, merge, FP8 quantise, FP8 forward
 constexpr int kProfCap = 1024;
 struct Profiler {
     bool created = false;
@@ -109,6 +110,7 @@ int device_setup(DeviceState** out) {
         if (allow_smem(fa::fwd_kernel<64>, fa::FwdCfg<64>::SMEM_BYTES) != cudaSuccess ||
             allow_smem(fa::fwd_kernel<128>, fa::FwdCfg<128>::SMEM_BYTES) != cudaSuccess ||
             decode_set_smem_limits() != cudaSuccess ||
+            allow_smem(fa::fwd_kernel<128, true>, fa::FwdCfg<128, true>::SMEM_BYTES) != cudaSuccess ||
             fa::bwd_set_smem_limits() != cudaSuccess)
             return FA_ERR_CUDA;
         st.ready = true;
@@ -134,6 +136,35 @@ int make_map(CUtensorMap* map, const void* ptr, int64_t rows, int H, int d, int 
 }
 
 bool misaligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+// FP8 operands: e4m3 codes [rows, H, 128] (3-D, boxes of 128 channels x 1 head x
+// 128 rows) and transposed V codes [B*H*128, Np] (2-D, boxes of 128 keys x 128
+// channel rows); 128-byte swizzle, zero fill outside.
+int make_map_u8_3d(CUtensorMap* map, const void* ptr, int64_t rows, int H) {
+    cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(H) * 128};
+    cuuint32_t box[3] = {128, 1, 128};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+int make_map_u8_2d(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols) {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols)};
+    cuuint32_t box[2] = {128, 128};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+int64_t fp8_vt_pitch(int N) { return (static_cast<int64_t>(N) + 15) / 16 * 16; }
 
 struct Common {
     fa::Geometry g;
@@ -408,6 +439,86 @@ int fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, void
     p.error_word = st->error_word;
     p.timeout_ns = g_fault_timeout_ns ? g_fault_timeout_ns : kDefaultTimeoutNs;
     return d == 64 ? launch_decode<64>(mk, mv, p, stream) : launch_decode<128>(mk, mv, p, stream);
+}
+
+size_t fa_fp8_vt_bytes(int B, int H, int N, int d) {
+    if (B <= 0 || H <= 0 || N <= 0 || d != 128) return 0;
+    return static_cast<size_t>(B) * H * d * static_cast<size_t>(fp8_vt_pitch(N));
+}
+
+int fa_quantize_fp8(const void* x, void* out, float* scales, int B, int N, int H, int d,
+                    int transpose, const float* signs, cudaStream_t stream) {
+    if (!x || !out || !scales) return FA_ERR_NULLPTR;
+    if (d != 128) return FA_ERR_UNSUPPORTED_D;
+    if (B < 0 || N < 0 || H <= 0) return FA_ERR_BAD_SHAPE;
+    if (transpose && signs) return FA_ERR_BAD_SHAPE;     // the rotation is for Q and K only
+    const int64_t rows = static_cast<int64_t>(B) * N;
+    const int64_t nb = (static_cast<int64_t>(N) + 127) / 128;
+    if (rows * H * d > (int64_t{1} << 40) || static_cast<int64_t>(B) * H * nb > (int64_t{1} << 31) - 1)
+        return FA_ERR_BAD_SHAPE;
+    if (misaligned(x) || misaligned(out) || (reinterpret_cast<uintptr_t>(scales) & 3u) ||
+        (reinterpret_cast<uintptr_t>(signs) & 3u))
+        return FA_ERR_MISALIGNED;
+    if (rows == 0) return FA_OK;
+    DeviceState* st = nullptr;
+    int rc = device_setup(&st);
+    if (rc != FA_OK) return rc;
+    fa::QuantParams p;
+    p.x = static_cast<const __nv_bfloat16*>(x);
+    p.out = static_cast<uint8_t*>(out);
+    p.scales = scales;
+    p.signs = signs;
+    p.B = B;
+    p.N = N;
+    p.H = H;
+    p.nb = static_cast<int>(nb);
+    p.Np = static_cast<int>(fp8_vt_pitch(N));
+    p.transpose = transpose ? 1 : 0;
+    const int slot = prof_start(6, stream);
+    fa::quantize_fp8_kernel<<<static_cast<int>(static_cast<int64_t>(B) * H * nb), 128, 0, stream>>>(p);
+    prof_stop(6, slot, stream);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_fwd_fp8(const void* q8, const void* k8, const void* vt8, const float* sq, const float* sk,
+               const float* sv, void* o, float* lse, int B, int H, int N, int d, float scale,
+               int causal, int window, cudaStream_t stream) {
+    if (!q8 || !k8 || !vt8 || !sq || !sk || !sv || !o || !lse) return FA_ERR_NULLPTR;
+    if (d != 128) return FA_ERR_UNSUPPORTED_D;
+    Common c;
+    int rc = validate_common(B, H, N, d, scale, causal, window, nullptr, &c);
+    if (rc != FA_OK) return rc;
+    if (misaligned(q8) || misaligned(k8) || misaligned(vt8) || misaligned(o) || misaligned(lse) ||
+        (reinterpret_cast<uintptr_t>(sq) & 3u) || (reinterpret_cast<uintptr_t>(sk) & 3u) ||
+        (reinterpret_cast<uintptr_t>(sv) & 3u))
+        return FA_ERR_MISALIGNED;
+    if (B == 0 || c.rows == 0) return FA_OK;
+    DeviceState* st = nullptr;
+    if ((rc = device_setup(&st)) != FA_OK) return rc;
+    CUtensorMap mq, mk, mv;
+    if (make_map_u8_3d(&mq, q8, c.rows, H) || make_map_u8_3d(&mk, k8, c.rows, H) ||
+        make_map_u8_2d(&mv, vt8, static_cast<int64_t>(B) * H * d, fp8_vt_pitch(N)))
+        return FA_ERR_CUDA;
+    fa::FwdParams p;
+    p.g = c.g;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.error_word = st->error_word;
+    p.timeout_ns = g_fault_timeout_ns ? g_fault_timeout_ns : kDefaultTimeoutNs;
+    p.fault_skip_v = 0;
+    p.sq = sq;
+    p.sk = sk;
+    p.sv = sv;
+    p.nb = (N + 127) / 128;
+    int grid = st->num_sms;
+    const int64_t items = static_cast<int64_t>(B) * H * ((N + 255) / 256);
+    if (items < grid) grid = static_cast<int>(items);
+    using C8 = fa::FwdCfg<128, true>;
+    const int slot = prof_start(7, stream);
+    fa::fwd_kernel<128, true><<<grid, C8::THREADS, C8::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+    prof_stop(7, slot, stream);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d, int varlen_total) {

@@ -32,6 +32,17 @@
 // halves of 64 keys that are released to the MMA warp one at a time.
 // The MMA thread issues S_t(j+1) right after O_t += P_t(j) V_j, so while one
 // softmax warpgroup works on its tile the tensor core runs the other's GEMMs.
+//
+// kF8 = true instantiates the block-quantised FP8 variant (FlashAttention
+// encyclopedia page, FlashAttention-3 paragraph: an FP8 path with block
+// quantisation, kept apart from the exact path).  Q and K are e4m3 codes with
+// one scale per 128-row block of a head, V is e4m3 stored transposed
+// ([B, H, d, keys], so both GEMMs read K-major operands) with one scale per
+// 128-key block.  Both GEMMs are kind::f8f6f4 MMAs; the score tile is scaled
+// by scale * log2(e) * s_q * s_k in the softmax, and P is written to TMEM as
+// e4m3 after multiplying by r = s_v(block) / max s_v (so one accumulator
+// serves every V block; O is multiplied back by max s_v at the end).  The row
+// sum uses the unrounded P.  Fixed-length sequences and d = 128 only.
 #pragma once
 
 #include "schedule.cuh"
@@ -50,17 +61,24 @@ struct FwdParams {
     int* error_word;
     uint64_t timeout_ns;
     int fault_skip_v;       // test hook: producer skips the first V load
+    // FP8 variant: block scales [B, H, nb] of Q, K, V (nb = ceil(N / 128))
+    const float* sq;
+    const float* sk;
+    const float* sv;
+    int nb;
 };
 
-template <int D>
+template <int D, bool kF8 = false>
 struct FwdCfg {
     static constexpr int BM = 128;              // rows per query tile
     static constexpr int BN = 128;              // keys per key tile
     static constexpr int ROWS = 2 * BM;         // rows per CTA work item
-    static constexpr int NSLOT = 4;             // K/V ring depth
-    static constexpr int BOX_BYTES = 128 * 128; // one TMA box: 128 rows x 64 bf16
-    static constexpr int TILE_BYTES = BM * D * 2;
-    static constexpr int NBOX = D / 64;
+    static constexpr int ESIZE = kF8 ? 1 : 2;   // bytes per element
+    static constexpr int BOX_BYTES = 128 * 128; // one TMA box: 128 rows x 128 bytes
+    static constexpr int TILE_BYTES = BM * D * ESIZE;
+    static constexpr int NSLOT = kF8 ? 8 : 4;   // K/V ring depth (128 KB either way)
+    static constexpr int NBOX = D * ESIZE / 128;
+    static constexpr int KSTEPS = D * ESIZE / 32;   // MMA k-steps of 32 bytes over d
     static constexpr int THREADS = 384;
     static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 384;
     // shared memory carve-up (offsets from a 1024-byte aligned base)
@@ -74,11 +92,12 @@ struct FwdCfg {
     static constexpr int SMEM_BYTES = OFF_PREFIX + 2 * (kMaxVarlenSeqs + 1) * 4 + 1024;
 };
 
-template <int D>
-__global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
+template <int D, bool kF8 = false>
+__global__ void __launch_bounds__(FwdCfg<D, kF8>::THREADS, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
            const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-    using C = FwdCfg<D>;
+    using C = FwdCfg<D, kF8>;
+    static_assert(!kF8 || D == 128, "the FP8 variant is built for d = 128");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align_smem_1024(smem_raw);
     uint8_t* sQ = smem + C::OFF_Q;
@@ -165,7 +184,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 for (int t = 0; t < 2; ++t)
                     for (int b = 0; b < C::NBOX; ++b)
                         tma_load_3d(sQ + t * C::TILE_BYTES + b * C::BOX_BYTES, &tm_q, q_full,
-                                    b * 64, h, sp.start + r_lo + t * C::BM);
+                                    b * 128 / C::ESIZE, h, sp.start + r_lo + t * C::BM);
                 ++q_issued;
                 for (int j = jb; j < je && ok; ++j) {
                     for (int kv = 0; kv < 2; ++kv) {
@@ -179,10 +198,16 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                             skipped_at = cnt;
                         } else {
                             mbar_arrive_expect_tx(slot_full + slot, C::TILE_BYTES);
-                            const CUtensorMap* tm = kv == 0 ? &tm_k : &tm_v;
-                            for (int b = 0; b < C::NBOX; ++b)
-                                tma_load_3d(sKV + slot * C::TILE_BYTES + b * C::BOX_BYTES, tm,
-                                            slot_full + slot, b * 64, h, kp.start + j * C::BN);
+                            uint8_t* dst = sKV + slot * C::TILE_BYTES;
+                            if (kF8 && kv == 1) {
+                                // V^T tile: d rows of this (sequence, head), 128 keys
+                                tma_load_2d(dst, &tm_v, slot_full + slot, j * C::BN, (s * H + h) * D);
+                            } else {
+                                const CUtensorMap* tm = kv == 0 ? &tm_k : &tm_v;
+                                for (int b = 0; b < C::NBOX; ++b)
+                                    tma_load_3d(dst + b * C::BOX_BYTES, tm, slot_full + slot,
+                                                b * 128 / C::ESIZE, h, kp.start + j * C::BN);
+                            }
                         }
                         ++cnt;
                     }
@@ -200,8 +225,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             }
         } else if (warp == 1 && lane == 0) {
             // --------------------------------------------------- MMA issuer --
-            constexpr uint32_t IDESC_S = idesc_bf16(128, C::BN, false, false);
-            constexpr uint32_t IDESC_O = idesc_bf16(128, D, false, true);
+            constexpr uint32_t IDESC_S = kF8 ? idesc_e4m3(128, C::BN) : idesc_bf16(128, C::BN, false, false);
+            constexpr uint32_t IDESC_O = kF8 ? idesc_e4m3(128, D) : idesc_bf16(128, D, false, true);
             const uint32_t q_addr = smem_u32(sQ);
             const uint32_t kv_addr = smem_u32(sKV);
             uint32_t cnt = 0, step = 0, item_it = 0;
@@ -211,10 +236,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 const uint32_t a0 = q_addr + t * C::TILE_BYTES;
                 const uint32_t b0 = kv_addr + kslot * C::TILE_BYTES;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
+                for (int kk = 0; kk < C::KSTEPS; ++kk) {
                     const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
-                    umma_ss(d_tmem, sw128_desc(a0 + off, 16, 1024), sw128_desc(b0 + off, 16, 1024),
-                            IDESC_S, kk > 0);
+                    if constexpr (kF8)
+                        umma_ss_f8(d_tmem, sw128_desc(a0 + off, 16, 1024),
+                                   sw128_desc(b0 + off, 16, 1024), IDESC_S, kk > 0);
+                    else
+                        umma_ss(d_tmem, sw128_desc(a0 + off, 16, 1024),
+                                sw128_desc(b0 + off, 16, 1024), IDESC_S, kk > 0);
                 }
             };
             // O_t (+)= P_t[:, keys of half] V_j[keys of half, :]  (half = 64 keys)
@@ -222,11 +251,23 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 const uint32_t d_tmem = tmem + (t ? C::COL_O1 : C::COL_O0);
                 const uint32_t a_tmem = tmem + (t ? C::COL_S1 : C::COL_S0);
                 const uint32_t b0 = kv_addr + vslot * C::TILE_BYTES;
+                if constexpr (kF8) {
+                    // P: 4 e4m3 per TMEM column, 32 keys (8 columns) per k-step;
+                    // V^T K-major: 32 keys = 32 bytes along its 128-byte rows
 #pragma unroll
-                for (int k = 0; k < C::BN / 32; ++k) {
-                    const int kk = half * (C::BN / 32) + k;
-                    umma_ts(d_tmem, a_tmem + kk * 8, sw128_desc(b0 + kk * 2048, C::BOX_BYTES, 1024),
-                            IDESC_O, (accumulate | kk) != 0);
+                    for (int k = 0; k < C::BN / 64; ++k) {
+                        const int kk = half * (C::BN / 64) + k;
+                        umma_ts_f8(d_tmem, a_tmem + kk * 8, sw128_desc(b0 + kk * 32, 16, 1024),
+                                   IDESC_O, (accumulate | kk) != 0);
+                    }
+                } else {
+#pragma unroll
+                    for (int k = 0; k < C::BN / 32; ++k) {
+                        const int kk = half * (C::BN / 32) + k;
+                        umma_ts(d_tmem, a_tmem + kk * 8,
+                                sw128_desc(b0 + kk * 2048, C::BOX_BYTES, 1024), IDESC_O,
+                                (accumulate | kk) != 0);
+                    }
                 }
             };
             ItemIter<false> it;
@@ -327,7 +368,27 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             const int i = r0 + row_in_tile;             // this thread's row
             float m_ref = -INFINITY;
             float l = 0.f;
+            // FP8: the Q tile's scale, and the largest V block scale of the head
+            float sq_t = 1.f, sv_max = 1.f;
+            const float* skh = nullptr;
+            const float* svh = nullptr;
+            if constexpr (kF8) {
+                const size_t base = (static_cast<size_t>(s) * H + h) * p.nb;
+                skh = p.sk + base;
+                svh = p.sv + base;
+                sq_t = p.sq[base + min(r0 / C::BM, p.nb - 1)];
+                float mv = 0.f;
+                for (int b = lane; b < p.nb; b += 32) mv = fmaxf(mv, svh[b]);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) mv = fmaxf(mv, __shfl_xor_sync(0xffffffffu, mv, o));
+                sv_max = mv > 0.f ? mv : 1.f;
+            }
             for (int j = jb; j < je; ++j, ++step) {
+                float sl2j = sl2, r_j = 1.f;
+                if constexpr (kF8) {
+                    sl2j = sl2 * sq_t * skh[j];
+                    r_j = fminf(1.f, svh[j] / sv_max);
+                }
                 if (!mbar_wait(s_full + t, step & 1, wc)) { ok = false; break; }
                 tc_fence_after();
                 float sv[C::BN];
@@ -362,7 +423,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                                fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
                 }
-                const float m_new = fmaxf(m_ref, mx * sl2);
+                const float m_new = fmaxf(m_ref, mx * sl2j);
                 const bool resc = m_new > m_ref + kRescaleLog2;
                 float alpha = 1.f;
                 if (resc) {
@@ -377,17 +438,33 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 // exponentials of the second.  Masked keys hold -inf: ex2 gives 0.
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
-#pragma unroll
-                    for (int c = half * (C::BN / 64); c < (half + 1) * (C::BN / 64); ++c) {
+                    if constexpr (kF8) {
+                        // 64 keys -> 16 columns of four e4m3 values, scaled by r_j
                         uint32_t pk[16];
 #pragma unroll
                         for (int e = 0; e < 16; ++e) {
-                            const float p0 = ex2(fmaf(sv[c * 32 + 2 * e], sl2, neg_m));
-                            const float p1 = ex2(fmaf(sv[c * 32 + 2 * e + 1], sl2, neg_m));
-                            lsum += p0 + p1;
-                            pk[e] = pack_bf16(p0, p1);
+                            const int k = half * 64 + 4 * e;
+                            const float p0 = ex2(fmaf(sv[k], sl2j, neg_m));
+                            const float p1 = ex2(fmaf(sv[k + 1], sl2j, neg_m));
+                            const float p2 = ex2(fmaf(sv[k + 2], sl2j, neg_m));
+                            const float p3 = ex2(fmaf(sv[k + 3], sl2j, neg_m));
+                            lsum += (p0 + p1) + (p2 + p3);
+                            pk[e] = pack_e4m3x4(p0 * r_j, p1 * r_j, p2 * r_j, p3 * r_j);
                         }
-                        tmem_st16(tS + c * 16, pk);
+                        tmem_st16(tS + half * 16, pk);
+                    } else {
+#pragma unroll
+                        for (int c = half * (C::BN / 64); c < (half + 1) * (C::BN / 64); ++c) {
+                            uint32_t pk[16];
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                const float p0 = ex2(fmaf(sv[c * 32 + 2 * e], sl2, neg_m));
+                                const float p1 = ex2(fmaf(sv[c * 32 + 2 * e + 1], sl2, neg_m));
+                                lsum += p0 + p1;
+                                pk[e] = pack_bf16(p0, p1);
+                            }
+                            tmem_st16(tS + c * 16, pk);
+                        }
                     }
                     if (half == 0 && j > jb && __any_sync(0xffffffffu, resc)) {
                         // O_t *= alpha before the first O_t += P V of this step.  The
@@ -416,7 +493,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             if (!mbar_wait(o_final + t, item_it & 1, wc)) { ok = false; break; }
             tc_fence_after();
             const bool valid = i < n;
-            const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            const float inv_l = l > 0.f ? (kF8 ? sv_max : 1.f) / l : 0.f;
             __nv_bfloat16* orow = p.o + (static_cast<size_t>(sp.start) + i) * H * D +
                                   static_cast<size_t>(h) * D;
 #pragma unroll

@@ -140,6 +140,29 @@ def test_kvcache_workspace_size_and_splits():
     assert fa.fa_fwd_kvcache_num_splits(1, 1, 1, 300, 128) == 1
 
 
+def test_fp8_validation_on_host():
+    def quant(**kw):
+        a = dict(x=P, out=P, scales=P, B=1, N=128, H=1, d=128, transpose=0, signs=None, stream=0)
+        a.update(kw)
+        return fa.fa_quantize_fp8(**a)
+
+    def fwd8(**kw):
+        a = dict(q8=P, k8=P, vt8=P, sq=P, sk=P, sv=P, o=P, lse=P, B=1, H=1, N=128, d=128,
+                 scale=0.1, causal=0, window=0, stream=0)
+        a.update(kw)
+        return fa.fa_fwd_fp8(**a)
+
+    assert quant(x=None) == -1 and quant(d=64) == -2 and quant(N=-1) == -3
+    assert quant(transpose=1, signs=P) == -3          # no rotation for V
+    assert quant(out=P + 8) == -4 and quant(scales=P + 2) == -4
+    assert quant(N=0) == 0
+    assert fwd8(sv=None) == -1 and fwd8(d=64) == -2 and fwd8(window=5) == -5
+    assert fwd8(k8=P + 4) == -4 and fwd8(scale=-1.0) == -9 and fwd8(B=0) == 0
+    # V codes transposed to [B, H, 128, N rounded up to 16]
+    assert fa.fa_fp8_vt_bytes(2, 3, 200, 128) == 2 * 3 * 128 * 208
+    assert fa.fa_fp8_vt_bytes(2, 3, 200, 64) == 0
+
+
 def test_empty_problems_are_noops():
     assert kvcache(Nq=0) == 0
     assert kvcache(B=0) == 0

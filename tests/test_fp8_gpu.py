@@ -1,0 +1,124 @@
+"""FP8 path on the GPU: fa_quantize_fp8 against the oracle's quantiser (bit
+for bit: codes and scales are integer decisions taken in float32 on both
+sides), and fa_fwd_fp8 against the oracle's block-quantised forward and
+against exact attention.
+
+Tolerance of the forward against its oracle: both compute the scores from the
+same codes, but the GPU's fp32 scores and exponentials differ from the
+oracle's float64 ones by a few ulp, so an e4m3 code of P can fall on the other
+side of a rounding boundary (rarely: about one element in 10^5).  One such
+flip moves an output by at most 2^-3 p/l |v|; mean-abs stays at the bf16
+level (2e-3) and max-abs is bounded at 5e-2."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import io_aware_exact_21_b200 as fa
+from io_aware_exact_21_b200.inputs import fixed_inputs, fp8_signs
+from oracle import oracle as orc
+
+from helpers import to64
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+TOL_FP8_MAX = 5e-2
+TOL_FP8_MEAN = 2e-3
+TOL_FP8_LSE = 1e-3
+
+
+def e4m3_values(codes_u8):
+    return codes_u8.cpu().view(torch.float8_e4m3fn).float().numpy()
+
+
+def gpu_quantize(x, signs):
+    qz = fa.quantize_fp8(x["q"].to(DEV), x["k"].to(DEV), x["v"].to(DEV),
+                         None if signs is None else signs.to(DEV))
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_error() == 0
+    return qz
+
+
+def vt_to_tokens(vt8, B, N, H):
+    Np = (N + 15) // 16 * 16
+    a = vt8[:B * H * 128 * Np].view(B, H, 128, Np)
+    return a, a[..., :N].permute(0, 3, 1, 2)          # [B, N, H, 128]
+
+
+@pytest.mark.parametrize("B,N,H", [(1, 1, 1), (2, 200, 3), (1, 128, 2), (1, 300, 2), (2, 1000, 1)])
+@pytest.mark.parametrize("rotate", [False, True])
+def test_quantiser_bit_exact(B, N, H, rotate):
+    x = fixed_inputs(B, N, H, 128, seed=N + 3)
+    signs = fp8_signs(11) if rotate else None
+    qz = gpu_quantize(x, signs)
+    for name, src, sgn in (("q", x["q"], signs), ("k", x["k"], signs)):
+        codes, scales = orc.quantize_fp8(src, sgn)
+        assert np.array_equal(e4m3_values(qz[name + "8"]), codes), name
+        assert np.array_equal(qz["s" + name].cpu().numpy(), scales), name
+    codes, scales = orc.quantize_fp8(x["v"])
+    full, tok = vt_to_tokens(qz["vt8"], B, N, H)
+    assert np.array_equal(e4m3_values(tok.contiguous()), codes)
+    assert np.array_equal(qz["sv"].cpu().numpy(), scales)
+    assert torch.count_nonzero(full[..., N:]) == 0            # padding keys are zero
+
+
+def oracle_fp8(x, signs, causal, window):
+    qc, sq = orc.quantize_fp8(x["q"], signs)
+    kc, sk = orc.quantize_fp8(x["k"], signs)
+    vc, sv = orc.quantize_fp8(x["v"])
+    return orc.fwd_fp8(qc, kc, vc, sq, sk, sv, 1 / math.sqrt(128), causal, window)
+
+
+def check_close(o, lse, O, L):
+    g = to64(o)
+    err = np.abs(g - O)
+    assert np.isfinite(g).all()
+    assert err.max() <= TOL_FP8_MAX and err.mean() <= TOL_FP8_MEAN, \
+        "O: max %.3e mean %.3e" % (err.max(), err.mean())
+    el = np.abs(to64(lse) - L)
+    assert el.max() <= TOL_FP8_LSE, "lse: max %.3e" % el.max()
+
+
+@pytest.mark.parametrize("B,N,H", [(1, 128, 1), (2, 300, 2), (1, 1000, 2), (2, 17, 1), (1, 2048, 1)])
+@pytest.mark.parametrize("causal,window", [(False, 0), (True, 0), (True, 100)])
+@pytest.mark.parametrize("rotate", [False, True])
+def test_fwd_fp8_matches_its_oracle(B, N, H, causal, window, rotate):
+    x = fixed_inputs(B, N, H, 128, seed=N + 17)
+    signs = fp8_signs(12) if rotate else None
+    qz = gpu_quantize(x, signs)
+    o, lse = fa.forward_fp8(qz, B, N, H, causal=causal, window=window)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_error() == 0
+    O, L = oracle_fp8(x, signs, causal, window)
+    check_close(o, lse, O, L)
+
+
+def test_fwd_fp8_error_against_exact_attention():
+    # the GPU's FP8 result is as far from exact attention as the FP8 oracle is
+    x = fixed_inputs(1, 2048, 2, 128, seed=8)
+    qz = gpu_quantize(x, None)
+    o, lse = fa.forward_fp8(qz, 1, 2048, 2)
+    torch.cuda.synchronize()
+    Oe, Le = orc.fwd(x["q"], x["k"], x["v"], 1 / math.sqrt(128))
+    g = to64(o)
+    assert np.abs(g - Oe).mean() < 0.1 * np.abs(Oe).mean()
+    assert np.abs(to64(lse) - Le).max() < 0.05
+
+
+def test_fwd_fp8_workload_heads():
+    # the measured configuration, B4 H16 N8192 d128 non-causal with the
+    # rotation; two whole (sequence, head) slices against the oracle (the
+    # quantisation is per (sequence, head), so a slice is self-contained)
+    B, N, H = 4, 8192, 16
+    x = fixed_inputs(B, N, H, 128, seed=2)
+    signs = fp8_signs(1)
+    qz = gpu_quantize(x, signs)
+    o, lse = fa.forward_fp8(qz, B, N, H)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_error() == 0
+    for b, h in ((0, 0), (3, 9)):
+        sl = {n: x[n][b:b + 1, :, h:h + 1] for n in ("q", "k", "v")}
+        O, L = oracle_fp8(sl, signs, False, 0)
+        check_close(o[b:b + 1, :, h:h + 1], lse[b:b + 1, h:h + 1], O, L)
