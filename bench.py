@@ -19,6 +19,11 @@ workload on the host cores.
 tokens in an 8192-row buffer, d=128) in GB/s of cache read against the HBM
 roofline.
 
+--workload fp8 measures the block-quantised FP8 forward on the training
+shape (B=4, H=16, N=8192, d=128, non-causal, with the rotation): quantisation
+of Q, K, V plus the FP8 forward kernel per step.  It is a separate,
+lower-precision path, not exact attention.
+
 --workload prefill_kv measures the cached-KV prefill forward instead
 (fa_fwd_kv: B=4, H=16, 2048 new query tokens after 6144 cached ones, so
 Nk=8192, d=128, causal aligned bottom-right), with its own oracle sample.
@@ -660,6 +665,152 @@ def oracle_sample_decode():
     return nbytes / secs / 1e9, desc, orc.num_threads(), secs
 
 
+# --------------------------------------------------------------- FP8 arm ---
+
+FP8_METRIC = "attention FP8 (block-quantised e4m3) forward TFLOPs/s (d=128), % of B200 dense FP8 peak"
+
+
+def fp8_config(extra=None):
+    w = WORKLOAD
+    cfg = {"workload": "FP8 forward B%d H%d N%d d%d non-causal, e4m3 with 128-row block scales and "
+                       "the Hadamard rotation of Q and K; quantisation included" % (
+                           w["B"], w["H"], w["N"], w["d"]),
+           "B": w["B"], "H": w["H"], "N": w["N"], "d": w["d"], "causal": False, "seed": w["seed"],
+           "l2": "inputs larger than L2 (Q, K, V 128 MiB each in bf16); L2 not flushed"}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+def run_fp8(args, rank, world, device):
+    import io_aware_exact_21_b200 as fa
+    from io_aware_exact_21_b200.inputs import fp8_signs
+    w = WORKLOAD
+    B, H, N, d = w["B"], w["H"], w["N"], w["d"]
+    host = make_inputs(device, w["seed"] + rank)
+    q, k, v = (host[n].to(device) for n in ("q", "k", "v"))
+    signs = fp8_signs(1).to(device)
+    stream = torch.cuda.current_stream(device)
+    qz = fa.quantize_fp8(q, k, v, signs, stream=stream)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=device)
+
+    def step(qq, kk, vv, oo, ll):
+        fa.fa_quantize_fp8(qq, qz["q8"], qz["sq"], B, N, H, d, 0, signs, stream)
+        fa.fa_quantize_fp8(kk, qz["k8"], qz["sk"], B, N, H, d, 0, signs, stream)
+        fa.fa_quantize_fp8(vv, qz["vt8"], qz["sv"], B, N, H, d, 1, None, stream)
+        fa.forward_fp8(qz, B, N, H, d, out=oo, lse=ll, stream=stream)
+
+    for _ in range(args.warmup):
+        step(q, k, v, o, lse)
+    torch.cuda.synchronize(device)
+    assert fa.fa_get_device_error() == 0
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    clocks = ClockSampler(device)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize(device)
+    fa.fa_profile_begin()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step(q, k, v, o, lse)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    elapsed = e0.elapsed_time(e1)
+    prof = fa.fa_profile_end()
+    clk = clocks.stop()
+    assert fa.fa_get_device_error() == 0
+
+    pin = {n: host[n].pin_memory() for n in ("q", "k", "v")}
+    dev_in = {n: torch.empty_like(q) for n in pin}
+    host_o = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    host_l = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = host_o.numel() * host_o.element_size() + host_l.numel() * host_l.element_size()
+
+    def e2e_step():
+        for n in ("q", "k", "v"):
+            dev_in[n].copy_(pin[n], non_blocking=True)
+        step(dev_in["q"], dev_in["k"], dev_in["v"], o, lse)
+        host_o.copy_(o, non_blocking=True)
+        host_l.copy_(lse, non_blocking=True)
+
+    e2e_steps = max(2, min(args.steps, 10))
+    e2e_step()
+    torch.cuda.synchronize(device)
+    barrier()
+    e2 = torch.cuda.Event(enable_timing=True)
+    e3 = torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e3.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    e2e_elapsed = e2.elapsed_time(e3)
+    assert fa.fa_get_device_error() == 0
+
+    elapsed, e2e_elapsed = max_over_ranks([elapsed, e2e_elapsed], world, device)
+    if rank != 0:
+        return None
+    f, _ = flops(B, H, N, d, False)
+    value = job_throughput(f, world, args.steps, elapsed)
+    fwd_ms = prof["fwd_fp8"][0] / prof["fwd_fp8"][1]
+    quant_ms = prof["quant_fp8"][0] / max(1, prof["quant_fp8"][1]) * 3
+    peaks, peak_src = load_peaks()
+    burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    peak = 2.0 * burst
+    achieved = f / (fwd_ms * 1e-3) / 1e12
+    return {
+        "metric": FP8_METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(elapsed / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
+        "data": "synthetic: i.i.d. N(0,1) bf16 Q, K, V (seeded), no dataset",
+        "config": fp8_config({"parallelism": "replicas" if world > 1 else "single GPU"}),
+        "kernels_ms": {"quantise_q_k_v": round(quant_ms, 4), "fwd_fp8": round(fwd_ms, 4)},
+        "roofline": {"kernel": "fwd_fp8", "bound": "tensor", "achieved": round(achieved, 2),
+                     "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "peak_source": "%s bf16_tflops (burst) x 2, the nominal FP8:BF16 dense ratio"
+                                    % peak_src,
+                     "traffic": None,
+                     "traffic_unit": "bytes per launch (ncu dram read + write)"},
+        "e2e": {"value": round(job_throughput(f, world, e2e_steps, e2e_elapsed), 2), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "how": "pinned host -> device copy of bf16 Q, K, V, quantisation, FP8 forward, "
+                       "device -> host copy of O and LSE every step, in order on one stream"},
+        "gpu_launches": sum(c for (_, c) in prof.values()),
+        "clocks": clk,
+    }
+
+
+def oracle_sample_fp8(n_tokens=8192, seed=2):
+    """The oracle's FP8 path (quantise Q, K, V with the rotation, then the
+    block-quantised forward) on one (sequence, head) of the workload,
+    truncated to n_tokens."""
+    from oracle import oracle as orc
+    from io_aware_exact_21_b200.inputs import fixed_inputs, fp8_signs
+    d = WORKLOAD["d"]
+    x = fixed_inputs(1, n_tokens, 1, d, seed=seed)
+    signs = fp8_signs(1)
+    t0 = time.perf_counter()
+    qc, sq = orc.quantize_fp8(x["q"], signs)
+    kc, sk = orc.quantize_fp8(x["k"], signs)
+    vc, sv = orc.quantize_fp8(x["v"])
+    orc.fwd_fp8(qc, kc, vc, sq, sk, sv, 1.0 / math.sqrt(d))
+    secs = time.perf_counter() - t0
+    f, _ = flops(1, 1, n_tokens, d, False)
+    desc = ("FP8 path of one (sequence, head) of the workload truncated to %d tokens, d=%d: "
+            "%.1f s on %d threads" % (n_tokens, d, secs, orc.num_threads()))
+    return f / secs / 1e12, desc, orc.num_threads(), secs
+
+
 def oracle_sample_kv(n_q=None, seed=5):
     """Time the float64 oracle's cached-KV forward on one (sequence, head) of
     the prefill workload, optionally with fewer queries (the key length and
@@ -730,6 +881,27 @@ def run_reference(args):
                                  "kind": "oracle", "sample": desc},
                 "e2e": {"value": value, "unit": DECODE_UNIT, "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
+    if args.workload == "fp8":
+        for _ in range(args.warmup):
+            oracle_sample_fp8(n_tokens=256)
+        vals = []
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            val, desc, threads, _ = oracle_sample_fp8(n_tokens=1024)
+            vals.append(val)
+        elapsed = time.perf_counter() - t0
+        value = statistics.mean(vals)
+        return {"impl": "reference", "metric": FP8_METRIC, "value": value, "unit": UNIT,
+                "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": elapsed * 1e3 / max(1, args.steps),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic: i.i.d. N(0,1) bf16 inputs; codes emulated in float32, "
+                        "forward in float64",
+                "config": fp8_config({"parallelism": "host cores"}),
+                "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                 "sample": desc},
+                "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
     kv = args.workload == "prefill_kv"
     for _ in range(args.warmup):
         if kv:
@@ -766,9 +938,10 @@ def main():
     ap.add_argument("--shape", default=None,
                     help="B,H,N,d override of the workload (profiling of smaller cases)")
     ap.add_argument("--causal", action="store_true", help="causal mask (profiling)")
-    ap.add_argument("--workload", choices=["train", "prefill_kv", "decode"], default="train",
+    ap.add_argument("--workload", choices=["train", "prefill_kv", "decode", "fp8"], default="train",
                     help="train: forward+backward step (default); prefill_kv: cached-KV "
-                         "prefill forward; decode: decode against a K/V cache")
+                         "prefill forward; decode: decode against a K/V cache; fp8: the "
+                         "block-quantised FP8 forward")
     args = ap.parse_args()
     if args.shape:
         B, H, N, d = (int(x) for x in args.shape.split(","))
@@ -795,9 +968,10 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                              device_id=device)
-    runner = {"train": run_ours, "prefill_kv": run_prefill_kv, "decode": run_decode}[args.workload]
+    runner = {"train": run_ours, "prefill_kv": run_prefill_kv, "decode": run_decode,
+              "fp8": run_fp8}[args.workload]
     sampler = {"train": oracle_sample, "prefill_kv": oracle_sample_kv,
-               "decode": oracle_sample_decode}[args.workload]
+               "decode": oracle_sample_decode, "fp8": oracle_sample_fp8}[args.workload]
     try:
         out = runner(args, rank, world, device)
         if out is not None:

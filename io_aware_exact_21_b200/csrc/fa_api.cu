@@ -475,7 +475,8 @@ int fa_quantize_fp8(const void* x, void* out, float* scales, int B, int N, int H
     p.Np = static_cast<int>(fp8_vt_pitch(N));
     p.transpose = transpose ? 1 : 0;
     const int slot = prof_start(6, stream);
-    fa::quantize_fp8_kernel<<<static_cast<int>(static_cast<int64_t>(B) * H * nb), 128, 0, stream>>>(p);
+    fa::quantize_fp8_kernel<<<static_cast<int>(static_cast<int64_t>(B) * H * nb), 32 * fa::kQuantWarps, 0,
+                              stream>>>(p);
     prof_stop(6, slot, stream);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }

@@ -3,8 +3,8 @@
 // FP8 path quantises by blocks and adds a step that reduces quantisation
 // error).
 //
-// One CTA per (sequence, head, block of 128 rows), 128 threads: warp w takes
-// rows w, w + 4, ..., and lane l holds channels 4l .. 4l + 3 of each (d = 128).
+// One CTA per (sequence, head, block of 128 rows), 256 threads: warp w takes
+// rows w, w + 8, ..., and lane l holds channels 4l .. 4l + 3 of each (d = 128).
 //  * optional rotation (Q and K): multiply by a sign vector, then the
 //    orthonormal Walsh-Hadamard transform -- butterflies (a, b) -> (a + b,
 //    a - b) on channel pairs (j, j + h) for h = 1, 2, 4, ..., 64 in that
@@ -13,7 +13,8 @@
 //    operation, so the codes do not depend on how a compiler would contract
 //    them.  q.k is unchanged by the rotation.
 //  * scale s = amax / 448 over the block (1 for an all-zero block); codes are
-//    e4m3(x / s), round to nearest even, saturating.
+//    e4m3(x * inv), inv = 1 / s rounded to float32 once per block, round to
+//    nearest even, saturating.
 //  * layout: Q and K codes keep the token-major [B, N, H, 128] layout; V codes
 //    are written transposed, [B, H, 128, Np] with Np = N rounded up to 16 and
 //    zeros past N, so the forward's PV GEMM reads a K-major operand.
@@ -34,9 +35,12 @@ struct QuantParams {
 
 constexpr int kQuantRowPitch = 132;   // shared transpose tile: 128 keys + 4 bytes of padding
 
-__global__ void __launch_bounds__(128)
+constexpr int kQuantWarps = 8;
+constexpr int kQuantRows = 128 / kQuantWarps;   // rows per warp
+
+__global__ void __launch_bounds__(32 * kQuantWarps)
 quantize_fp8_kernel(const QuantParams p) {
-    __shared__ float s_amax[4];
+    __shared__ float s_amax[kQuantWarps];
     __shared__ __align__(16) uint8_t s_t[128 * kQuantRowPitch];
     const int item = blockIdx.x;
     const int blk = item % p.nb;
@@ -52,20 +56,25 @@ quantize_fp8_kernel(const QuantParams p) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) sg[e] = p.signs[4 * lane + e];
     }
-    float y[32][4];
+    // all row loads first, so they are in flight together
+    uint2 raw[kQuantRows];
+#pragma unroll
+    for (int k = 0; k < kQuantRows; ++k) {
+        const int r = r0 + warp + kQuantWarps * k;
+        raw[k] = make_uint2(0u, 0u);
+        if (r < p.N)
+            raw[k] = __ldg(reinterpret_cast<const uint2*>(
+                p.x + ((static_cast<size_t>(b) * p.N + r) * p.H + h) * 128 + 4 * lane));
+    }
+    float y[kQuantRows][4];
     float amax = 0.f;
 #pragma unroll
-    for (int k = 0; k < 32; ++k) {
-        const int r = r0 + warp + 4 * k;
-        float x4[4] = {0.f, 0.f, 0.f, 0.f};
-        if (r < p.N) {
-            const uint2 raw = *reinterpret_cast<const uint2*>(
-                p.x + ((static_cast<size_t>(b) * p.N + r) * p.H + h) * 128 + 4 * lane);
-            x4[0] = __uint_as_float(raw.x << 16);
-            x4[1] = __uint_as_float(raw.x & 0xffff0000u);
-            x4[2] = __uint_as_float(raw.y << 16);
-            x4[3] = __uint_as_float(raw.y & 0xffff0000u);
-        }
+    for (int k = 0; k < kQuantRows; ++k) {
+        float x4[4];
+        x4[0] = __uint_as_float(raw[k].x << 16);
+        x4[1] = __uint_as_float(raw[k].x & 0xffff0000u);
+        x4[2] = __uint_as_float(raw[k].y << 16);
+        x4[3] = __uint_as_float(raw[k].y & 0xffff0000u);
         if (p.signs) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) x4[e] = __fmul_rn(x4[e], sg[e]);
@@ -108,16 +117,19 @@ quantize_fp8_kernel(const QuantParams p) {
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     if (lane == 0) s_amax[warp] = amax;
     __syncthreads();
-    amax = fmaxf(fmaxf(s_amax[0], s_amax[1]), fmaxf(s_amax[2], s_amax[3]));
+    amax = s_amax[0];
+#pragma unroll
+    for (int w = 1; w < kQuantWarps; ++w) amax = fmaxf(amax, s_amax[w]);
     const float sc = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+    const float inv = __fdiv_rn(1.f, sc);
     if (threadIdx.x == 0) p.scales[static_cast<size_t>(bh) * p.nb + blk] = sc;
 
 #pragma unroll
-    for (int k = 0; k < 32; ++k) {
-        const int rr = warp + 4 * k;
+    for (int k = 0; k < kQuantRows; ++k) {
+        const int rr = warp + kQuantWarps * k;
         const int r = r0 + rr;
-        const uint32_t code = pack_e4m3x4(__fdiv_rn(y[k][0], sc), __fdiv_rn(y[k][1], sc),
-                                          __fdiv_rn(y[k][2], sc), __fdiv_rn(y[k][3], sc));
+        const uint32_t code = pack_e4m3x4(__fmul_rn(y[k][0], inv), __fmul_rn(y[k][1], inv),
+                                          __fmul_rn(y[k][2], inv), __fmul_rn(y[k][3], inv));
         if (!p.transpose) {
             if (r < p.N)
                 *reinterpret_cast<uint32_t*>(
@@ -131,12 +143,14 @@ quantize_fp8_kernel(const QuantParams p) {
     }
     if (p.transpose) {
         __syncthreads();
-        // thread c writes channel c's keys r0 .. r0 + 127 (those below Np)
-        const int c = threadIdx.x;
+        // two threads per channel c, each writing half of the keys r0 .. r0 + 127
+        // (those below Np)
+        const int c = threadIdx.x >> 1;
+        const int half = threadIdx.x & 1;
         const int nkeys = min(128, p.Np - r0);
         uint8_t* dst = p.out + (static_cast<size_t>(bh) * 128 + c) * p.Np + r0;
         const uint32_t* src = reinterpret_cast<const uint32_t*>(s_t + c * kQuantRowPitch);
-        for (int w = 0; w < nkeys / 16; ++w) {
+        for (int w = half; w < nkeys / 16; w += 2) {
             const uint4 v = make_uint4(src[4 * w], src[4 * w + 1], src[4 * w + 2], src[4 * w + 3]);
             *reinterpret_cast<uint4*>(dst + 16 * w) = v;
         }

@@ -21,7 +21,11 @@
  *     every q.k is unchanged while outliers are spread over all channels.
  *  2. Block scales: for every block of 128 rows of one head (rows past the
  *     sequence end excluded), s = amax / 448 (448 is the largest finite
- *     e4m3 value; s = 1 for an all-zero block), and codes c = e4m3(x / s).
+ *     e4m3 value; s = 1 for an all-zero block), and codes c = e4m3(x * inv)
+ *     with inv = 1 / s rounded to float32 once per block (one multiply per
+ *     element instead of a division; the two readings of "x over s" differ
+ *     only where x / s and x * inv fall on opposite sides of an e4m3
+ *     rounding boundary).
  *     Steps 1-2 decide integer codes, so they are taken in float32, the
  *     precision the CUDA kernel takes them in; every float operation here is
  *     a single IEEE-754 float32 operation (no fused multiply-add).
@@ -121,11 +125,12 @@ int oracle_quantize_fp8(const float *x, int B, int N, int H, int d, const float 
                     }
                 }
                 const float s = amax > 0.0f ? amax / 448.0f : 1.0f;
+                const float inv = 1.0f / s;
                 scales[((size_t)b * H + h) * nb + blk] = s;
                 for (int r = r0; r < r1; ++r) {
                     const float *yr = y + (size_t)(r - r0) * d;
                     float *cr = codes + (((size_t)b * N + r) * H + h) * d;
-                    for (int c = 0; c < d; ++c) cr[c] = oracle_e4m3_round(yr[c] / s);
+                    for (int c = 0; c < d; ++c) cr[c] = oracle_e4m3_round(yr[c] * inv);
                 }
             }
     free(y);

@@ -74,7 +74,8 @@ def test_quantiser_definition(rotate):
                 yb = y[b, rows, h]
                 sc = np.float32(np.abs(yb).max()) / np.float32(448.0)
                 assert scales[b, h, blk] == sc
-                ref = torch.from_numpy((yb / sc).astype(np.float32)).to(torch.float8_e4m3fn).float()
+                inv = np.float32(1.0) / sc
+                ref = torch.from_numpy((yb * inv).astype(np.float32)).to(torch.float8_e4m3fn).float()
                 assert np.array_equal(codes[b, rows, h], ref.numpy())
                 # e4m3 error bound: half a spacing (2^-4 relative, 2^-10 absolute below 2^-6)
                 err = np.abs(codes[b, rows, h].astype(np.float64) * sc - yb)
