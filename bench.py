@@ -52,23 +52,24 @@ WORKLOAD = dict(B=4, H=16, N=8192, d=128, causal=False, window=0, seed=2)
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
-# ncu captures.  Training step: the B=2 H=16 N=8192 d=128 non-causal case,
-# scaled by 2 to the B=4 workload (each kernel's traffic grows with the number
-# of heads it processes).  Decode: the decode workload itself.  Valid only for
+# ncu captures.  Training step and FP8 forward: the B=2 H=16 N=8192 d=128
+# non-causal case, scaled by 2 to the B=4 workload (each kernel's traffic grows
+# with the number of heads it processes).  Decode: the decode workload itself.  Valid only for
 # the kernel sources a capture was taken on: each entry carries a hash of them
 # and is reported as null once they change.  Summaries and commands:
 # profiles/*_kernel_*.md.
 TRAFFIC = {
-    "fwd": {"bytes_per_launch": 2 * (203.64e6 + 49.21e6), "workload": "train",
-            "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh"), "sha": "b41eb356c35423da"},
-    "dkdv": {"bytes_per_launch": 2 * (272.13e6 + 106.88e6), "workload": "train",
-             "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "81faa9db662491cc"},
-    "dq": {"bytes_per_launch": 2 * (271.25e6 + 53.68e6), "workload": "train",
-           "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "81faa9db662491cc"},
-    "decode": {"bytes_per_launch": 792.91e6 + 4.74e6, "workload": "decode",
-               "sources": ("decode_kernel.cuh", "sm100.cuh"), "sha": "beaec1c610a97f43"},
+    "fwd": {"bytes_per_launch": 2 * (206.98e6 + 48.87e6), "workload": "train",
+            "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh"), "sha": "546f242d1f9fa674"},
+    "dkdv": {"bytes_per_launch": 2 * (272.25e6 + 106.58e6), "workload": "train",
+             "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "a86cc198582432d1"},
+    "dq": {"bytes_per_launch": 2 * (271.42e6 + 53.35e6), "workload": "train",
+           "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "a86cc198582432d1"},
+    "decode": {"bytes_per_launch": 792.82e6 + 4.50e6, "workload": "decode",
+               "sources": ("decode_kernel.cuh", "sm100.cuh"), "sha": "21d2a30613f1e750"},
+    "fwd_fp8": {"bytes_per_launch": 2 * (101.02e6 + 31.42e6), "workload": "fp8",
+                "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh"), "sha": "546f242d1f9fa674"},
 }
-
 
 def traffic_for(kernel, workload="train"):
     """ncu traffic per launch if the kernel's sources still match the capture."""
@@ -85,7 +86,7 @@ def traffic_for(kernel, workload="train"):
         return None
     if h.hexdigest()[:16] != t["sha"]:
         return None
-    if workload == "train":
+    if workload in ("train", "fp8"):
         w = WORKLOAD
         if (w["B"], w["H"], w["N"], w["d"], w["causal"]) != (4, 16, 8192, 128, False):
             return None
@@ -779,7 +780,7 @@ def run_fp8(args, rank, world, device):
                      "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "peak_source": "%s bf16_tflops (burst) x 2, the nominal FP8:BF16 dense ratio"
                                     % peak_src,
-                     "traffic": None,
+                     "traffic": traffic_for("fwd_fp8", "fp8"),
                      "traffic_unit": "bytes per launch (ncu dram read + write)"},
         "e2e": {"value": round(job_throughput(f, world, e2e_steps, e2e_elapsed), 2), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
