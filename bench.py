@@ -25,8 +25,9 @@ of Q, K, V plus the FP8 forward kernel per step.  It is a separate,
 lower-precision path, not exact attention.
 
 --workload prefill_kv measures the cached-KV prefill forward instead
-(fa_fwd_kv: B=4, H=16, 2048 new query tokens after 6144 cached ones, so
-Nk=8192, d=128, causal aligned bottom-right), with its own oracle sample.
+(fa_fwd_kvcache with the library's key split: B=4, H=16, 2048 new query
+tokens after 6144 cached ones, so Nk=8192, d=128, causal aligned
+bottom-right), with its own oracle sample.
 """
 from __future__ import annotations
 
@@ -412,10 +413,14 @@ def run_prefill_kv(args, rank, world, device):
     o = torch.empty_like(q)
     lse = torch.empty((B, H, Nq), dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
+    # through the cache interface, split along the keys as the library chooses
+    ns = fa.fa_fwd_kvcache_num_splits(B, H, Nq, Nk, d)
+    ws = torch.empty(max(16, fa.fa_fwd_kvcache_workspace_size(B, H, Nq, d, ns)), dtype=torch.uint8,
+                     device=device)
 
     def step(qq, kk, vv, oo, ll):
-        fa.forward_kv(qq, kk, vv, causal=causal, window=window, scale=scale, out=oo, lse=ll,
-                      stream=stream)
+        fa.forward_kvcache(qq, kk, vv, causal=causal, window=window, scale=scale, num_splits=ns,
+                           out=oo, lse=ll, workspace=ws, stream=stream)
 
     for _ in range(args.warmup):
         step(q, k, v, o, lse)
@@ -482,6 +487,7 @@ def run_prefill_kv(args, rank, world, device):
     value = job_throughput(f, world, args.steps, elapsed)
     ms, cnt = prof["fwd"]
     kernel_ms = ms / cnt
+    merge_ms = prof["combine"][0] / prof["combine"][1] if prof["combine"][1] else 0.0
     peaks, peak_src = load_peaks()
     peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     achieved = f / (kernel_ms * 1e-3) / 1e12
@@ -490,7 +496,9 @@ def run_prefill_kv(args, rank, world, device):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(elapsed / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic: i.i.d. N(0,1) bf16 Q, K, V (seeded), no dataset",
-        "config": prefill_kv_config({"parallelism": "replicas" if world > 1 else "single GPU"}),
+        "config": prefill_kv_config({"parallelism": "replicas" if world > 1 else "single GPU",
+                                     "num_splits": ns, "api": "fa_fwd_kvcache"}),
+        "kernels_ms": {"fwd": round(kernel_ms, 4), "merge": round(merge_ms, 4)},
         "roofline": {"kernel": "fwd", "bound": "tensor", "achieved": round(achieved, 2),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "peak_source": "%s bf16_tflops (burst: the kernel is timed alone)" % peak_src,

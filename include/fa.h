@@ -130,12 +130,18 @@ int fa_fwd_kv(const void* q, const void* k, const void* v, void* o, float* lse,
  * scenario table), and they list inference with cached keys and values among
  * the interfaces (FlashAttention encyclopedia page, "software integration").
  *
- * q, o    : [B, Nq, H, d] bf16 (1 <= Nq <= 16; Nq = 0 is a no-op).
+ * q, o    : [B, Nq, H, d] bf16 (Nq = 0 is a no-op).  Up to 16 queries per
+ *           sequence run on a CUDA-core kernel built for the cache read;
+ *           longer chunks (prefill of new tokens after cached ones) run on the
+ *           tensor-core forward kernel, split along the keys the same way.
  * k_cache, v_cache : [B, Nk, H, d] bf16; sequence b uses rows 0 .. nk_b - 1
  *           of its slice, nk_b = seqlens_k[b] (device int32 [B], clamped to
- *           [0, Nk]) or Nk when seqlens_k is NULL.  Rows past nk_b are never
- *           used (they may hold anything).  k_cache and v_cache may be NULL
- *           when B * Nk = 0.
+ *           [0, Nk]) or Nk when seqlens_k is NULL.  Rows past nk_b never
+ *           reach a result; with Nq <= 16 they are never read and may hold
+ *           anything, with Nq > 16 the rows past nk_b that share a 128-row tile
+ *           with used ones are read and multiplied by zero, so they must hold
+ *           finite values (a zero-initialised cache does).  k_cache and v_cache
+ *           may be NULL when B * Nk = 0.
  * lse     : [B, H, Nq] fp32, natural log.
  * Masks   : as fa_fwd_kv with the queries at the last Nq positions of the
  *           nk_b keys: query i is at position nk_b - Nq + i.
@@ -149,8 +155,8 @@ int fa_fwd_kv(const void* q, const void* k, const void* v, void* o, float* lse,
  * workspace : device memory of at least fa_fwd_kvcache_workspace_size(B, H,
  *           Nq, d, splits) bytes, 16-byte aligned, for splits > 1 (NULL
  *           otherwise); contents on entry do not matter.
- * Errors as fa_fwd; Nq > 16 or num_splits outside [0, 32] is
- * FA_ERR_BAD_SHAPE, a missing or short workspace FA_ERR_WORKSPACE.
+ * Errors as fa_fwd; num_splits outside [0, 32] is FA_ERR_BAD_SHAPE, a
+ * missing or short workspace FA_ERR_WORKSPACE.
  */
 int fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, void* o,
                    float* lse, int B, int H, int Nq, int Nk, int d, float scale, int causal,

@@ -259,10 +259,10 @@ def forward_kv(q, k, v, causal=False, window=0, cu_seqlens_q=None, cu_seqlens_k=
 
 def forward_kvcache(q, k_cache, v_cache, seqlens_k=None, causal=False, window=0, scale=None,
                     num_splits=0, out=None, lse=None, workspace=None, stream=None):
-    """Decode: q [B, Nq, H, d] (Nq <= 16) against k_cache, v_cache [B, Nk, H, d],
-    of which sequence b uses its first seqlens_k[b] rows (int32 CUDA tensor, or
-    None for all Nk); queries are the last Nq of those positions.  Returns
-    (O, LSE)."""
+    """Attention against a K/V cache: q [B, Nq, H, d] (a few decode queries, or
+    a prefill chunk) against k_cache, v_cache [B, Nk, H, d], of which sequence
+    b uses its first seqlens_k[b] rows (int32 CUDA tensor, or None for all Nk);
+    queries are the last Nq of those positions.  Returns (O, LSE)."""
     import torch
     B, Nq, H, d = q.shape
     Nk = k_cache.shape[1]

@@ -111,6 +111,8 @@ int device_setup(DeviceState** out) {
             allow_smem(fa::fwd_kernel<128>, fa::FwdCfg<128>::SMEM_BYTES) != cudaSuccess ||
             decode_set_smem_limits() != cudaSuccess ||
             allow_smem(fa::fwd_kernel<128, true>, fa::FwdCfg<128, true>::SMEM_BYTES) != cudaSuccess ||
+            allow_smem(fa::fwd_kernel<64, false, true>, fa::FwdCfg<64>::SMEM_BYTES) != cudaSuccess ||
+            allow_smem(fa::fwd_kernel<128, false, true>, fa::FwdCfg<128>::SMEM_BYTES) != cudaSuccess ||
             fa::bwd_set_smem_limits() != cudaSuccess)
             return FA_ERR_CUDA;
         st.ready = true;
@@ -228,6 +230,25 @@ int decode_splits(int B, int H, int Nk, int num_sms) {
         }
     }
     return best;
+}
+
+// Split count for a prefill chunk (more than 16 queries) on the tensor-core
+// forward, whose work items are blocks of 256 queries: split only when there
+// are fewer blocks than SMs, into as many ranges as fill them, each keeping at
+// least 8 key tiles of 128.  (With enough blocks, splitting measured slower:
+// the extra Q loads and fp32 partial outputs cost more than the better
+// balance of the last wave gains.)
+int prefill_splits(int B, int H, int Nq, int Nk, int num_sms) {
+    const int64_t items = static_cast<int64_t>(B) * H * ((Nq + 255) / 256);
+    if (items >= num_sms) return 1;
+    const int tiles = (Nk + 127) / 128;
+    const int64_t want = (num_sms + items - 1) / items;
+    return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>({want, fa::kDecMaxSplits, tiles / 8})));
+}
+
+int kvcache_splits(int B, int H, int Nq, int Nk, int num_sms) {
+    return Nq <= fa::kDecMaxQ ? decode_splits(B, H, Nk, num_sms)
+                              : prefill_splits(B, H, Nq, Nk, num_sms);
 }
 
 size_t decode_workspace_bytes(int B, int H, int Nq, int d, int ns) {
@@ -364,14 +385,13 @@ int fa_fwd_kv(const void* q, const void* k, const void* v, void* o, float* lse, 
 }
 
 int fa_fwd_kvcache_num_splits(int B, int H, int Nq, int Nk, int d) {
-    (void)Nq;
     (void)d;
-    if (B <= 0 || H <= 0 || Nk <= 0) return 1;
+    if (B <= 0 || H <= 0 || Nk <= 0 || Nq <= 0) return 1;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (sms <= 0) sms = 148;
-    return decode_splits(B, H, Nk, sms);
+    return kvcache_splits(B, H, Nq, Nk, sms);
 }
 
 size_t fa_fwd_kvcache_workspace_size(int B, int H, int Nq, int d, int num_splits) {
@@ -385,7 +405,7 @@ int fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, void
                    cudaStream_t stream) {
     if (!q || !o || !lse) return FA_ERR_NULLPTR;
     if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED_D;
-    if (B < 0 || H <= 0 || Nq < 0 || Nk < 0 || Nq > fa::kDecMaxQ) return FA_ERR_BAD_SHAPE;
+    if (B < 0 || H <= 0 || Nq < 0 || Nk < 0) return FA_ERR_BAD_SHAPE;
     if (num_splits < 0 || num_splits > fa::kDecMaxSplits) return FA_ERR_BAD_SHAPE;
     if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_BAD_SCALE;
     if (window > 0 && !causal) return FA_ERR_BAD_MASK;
@@ -409,8 +429,68 @@ int fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, void
     if (rc != FA_OK) return rc;
     DeviceState* st = nullptr;
     if ((rc = device_setup(&st)) != FA_OK) return rc;
-    const int ns = num_splits > 0 ? num_splits : decode_splits(B, H, Nk, st->num_sms);
+    const int ns = num_splits > 0 ? num_splits : kvcache_splits(B, H, Nq, Nk, st->num_sms);
     if ((rc = check_ws(ns)) != FA_OK) return rc;
+    if (Nq > fa::kDecMaxQ) {
+        // a prefill chunk: the tensor-core forward, split along the keys when ns > 1
+        if (rows_q > (int64_t{1} << 31) - 1) return FA_ERR_BAD_SHAPE;
+        // with no cache rows at all the maps are pointed at q: every key is
+        // masked and nothing of q is used as a key
+        const void* kk = rows_k > 0 ? k_cache : q;
+        const void* vv = rows_k > 0 ? v_cache : q;
+        const int64_t map_rows_k = rows_k > 0 ? rows_k : rows_q;
+        CUtensorMap mq, mk, mv;
+        if (make_map(&mq, q, rows_q, H, d, 128) || make_map(&mk, kk, map_rows_k, H, d, 128) ||
+            make_map(&mv, vv, map_rows_k, H, d, 128))
+            return FA_ERR_CUDA;
+        fa::FwdParams p;
+        p.g.B = B;
+        p.g.H = H;
+        p.g.N = Nq;
+        p.g.T = static_cast<int>(rows_q);
+        p.g.cu_seqlens = nullptr;
+        p.g.causal = causal ? 1 : 0;
+        p.g.window = window > 0 ? window : 0;
+        p.g.Nk = Nk;
+        p.g.Tk = static_cast<int>(rows_k);
+        p.g.cu_seqlens_k = nullptr;
+        p.o = static_cast<__nv_bfloat16*>(o);
+        p.lse = lse;
+        p.scale_log2 = scale * 1.4426950408889634f;
+        p.error_word = st->error_word;
+        p.timeout_ns = g_fault_timeout_ns ? g_fault_timeout_ns : kDefaultTimeoutNs;
+        p.fault_skip_v = 0;
+        p.nsplit = ns;
+        p.kv.seqused_k = seqlens_k;
+        p.kv.o_part = ns > 1 ? static_cast<float*>(workspace) : nullptr;
+        p.kv.lse_part = ns > 1 ? static_cast<float*>(workspace) + static_cast<size_t>(ns) * rows_q * H * d
+                               : nullptr;
+        int grid = st->num_sms;
+        const int64_t items = static_cast<int64_t>(B) * H * ns * ((Nq + 255) / 256);
+        if (items < grid) grid = static_cast<int>(items);
+        const int slot = prof_start(0, stream);
+        if (d == 64) {
+            fa::fwd_kernel<64, false, true><<<grid, fa::FwdCfg<64>::THREADS, fa::FwdCfg<64>::SMEM_BYTES,
+                                              stream>>>(mq, mk, mv, p);
+            rc = cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+        } else {
+            fa::fwd_kernel<128, false, true><<<grid, fa::FwdCfg<128>::THREADS, fa::FwdCfg<128>::SMEM_BYTES,
+                                               stream>>>(mq, mk, mv, p);
+            rc = cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+        }
+        prof_stop(0, slot, stream);
+        if (rc != FA_OK || ns == 1) return rc;
+        const int64_t warps = rows_q * H;
+        const int slot2 = prof_start(5, stream);
+        if (d == 64)
+            fa::combine_kernel<64><<<static_cast<int>((warps + 7) / 8), 256, 0, stream>>>(
+                p.kv.o_part, p.kv.lse_part, p.o, lse, static_cast<int>(rows_q), H, Nq, ns);
+        else
+            fa::combine_kernel<128><<<static_cast<int>((warps + 7) / 8), 256, 0, stream>>>(
+                p.kv.o_part, p.kv.lse_part, p.o, lse, static_cast<int>(rows_q), H, Nq, ns);
+        prof_stop(5, slot2, stream);
+        return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+    }
     // With no cache rows every split is empty and no tile is loaded; the maps
     // still need a valid base, so they are pointed at q.
     const void* kk = rows_k > 0 ? k_cache : q;
@@ -508,9 +588,9 @@ int fa_fwd_fp8(const void* q8, const void* k8, const void* vt8, const float* sq,
     p.error_word = st->error_word;
     p.timeout_ns = g_fault_timeout_ns ? g_fault_timeout_ns : kDefaultTimeoutNs;
     p.fault_skip_v = 0;
-    p.sq = sq;
-    p.sk = sk;
-    p.sv = sv;
+    p.f8.sq = sq;
+    p.f8.sk = sk;
+    p.f8.sv = sv;
     p.nb = (N + 127) / 128;
     int grid = st->num_sms;
     const int64_t items = static_cast<int64_t>(B) * H * ((N + 255) / 256);

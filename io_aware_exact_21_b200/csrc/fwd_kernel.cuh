@@ -43,6 +43,16 @@
 // e4m3 after multiplying by r = s_v(block) / max s_v (so one accumulator
 // serves every V block; O is multiplied back by max s_v at the end).  The row
 // sum uses the unrounded P.  Fixed-length sequences and d = 128 only.
+//
+// kCache = true instantiates the padded K/V cache variant (fixed-length
+// queries; sequence s uses the first seqused_k[s] rows of its Nk-row cache
+// slice).  With nsplit > 1 it also cuts the key tiles of every block into
+// `nsplit` contiguous ranges that run as separate work items (the schedule
+// sees H * nsplit heads), so that few, long blocks still spread over all SMs;
+// each item then writes O / l as fp32 and the base-2 log-sum-exp of its range
+// to the split buffers ([nsplit, rows, H, D] and [nsplit, H, rows]), which
+// combine_kernel merges.  A split with no tiles writes -inf and is skipped by
+// the merge.
 #pragma once
 
 #include "schedule.cuh"
@@ -61,12 +71,40 @@ struct FwdParams {
     int* error_word;
     uint64_t timeout_ns;
     int fault_skip_v;       // test hook: producer skips the first V load
-    // FP8 variant: block scales [B, H, nb] of Q, K, V (nb = ceil(N / 128))
-    const float* sq;
-    const float* sk;
-    const float* sv;
-    int nb;
+    // Variant parameters; the FP8 and padded-cache variants never coexist, so
+    // they share storage (a larger parameter block changed the plain kernel's
+    // register allocation for the worse).
+    struct F8 {                 // FP8: block scales [B, H, nb] of Q, K, V, nb = ceil(N / 128)
+        const float* sq;
+        const float* sk;
+        const float* sv;
+    };
+    struct Cache {              // padded cache: used rows per sequence, split outputs
+        const int* seqused_k;   // or nullptr (all Nk rows in use)
+        float* o_part;          // [nsplit, B * N, H, D]
+        float* lse_part;        // [nsplit, H, B * N], base 2
+    };
+    union {
+        F8 f8;
+        Cache kv;
+    };
+    union {
+        int nb;                 // FP8
+        int nsplit;             // padded cache
+    };
 };
+
+// Tiles [jb, je) of split `split` out of `nsplit` for a block whose key range
+// is [jb, je); false when the split has none.
+__device__ __forceinline__ bool split_tile_range(int nsplit, int split, int& jb, int& je) {
+    const int n = je - jb;
+    const int ns = min(nsplit, n);
+    if (split >= ns) return false;
+    const int b0 = jb;
+    jb = b0 + split * n / ns;
+    je = b0 + (split + 1) * n / ns;
+    return true;
+}
 
 template <int D, bool kF8 = false>
 struct FwdCfg {
@@ -92,12 +130,13 @@ struct FwdCfg {
     static constexpr int SMEM_BYTES = OFF_PREFIX + 2 * (kMaxVarlenSeqs + 1) * 4 + 1024;
 };
 
-template <int D, bool kF8 = false>
+template <int D, bool kF8 = false, bool kCache = false>
 __global__ void __launch_bounds__(FwdCfg<D, kF8>::THREADS, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
            const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
     using C = FwdCfg<D, kF8>;
     static_assert(!kF8 || D == 128, "the FP8 variant is built for d = 128");
+    static_assert(!(kF8 && kCache), "no FP8 cache variant");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align_smem_1024(smem_raw);
     uint8_t* sQ = smem + C::OFF_Q;
@@ -151,8 +190,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     sch.order = 0;                              // pairs only (ItemIter<false>)
     sch.bprefix = prefix;
     sch.uprefix = prefix + kMaxVarlenSeqs + 1;
-    sch.total_units = build_schedule_prefix(p.g, C::ROWS, prefix, prefix + kMaxVarlenSeqs + 1,
-                                            scratch);  // has __syncthreads
+    if constexpr (kCache) {
+        sch.g.H = p.g.H * p.nsplit;             // (head, split) pairs
+        sch.total_units = build_schedule_prefix(sch.g, C::ROWS, prefix,
+                                                prefix + kMaxVarlenSeqs + 1, scratch);
+    } else {
+        sch.total_units = build_schedule_prefix(p.g, C::ROWS, prefix, prefix + kMaxVarlenSeqs + 1,
+                                                scratch);  // has __syncthreads
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -172,13 +217,24 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             ItemIter<false> it;
             int s, h, blk;
             for (; ok && it.next(sch, s, h, blk); ++item_it) {
+                [[maybe_unused]] int split = 0;
+                if constexpr (kCache) {
+                    split = h % p.nsplit;
+                    h /= p.nsplit;
+                }
                 const SeqSpan sp = sch.span(s);
-                const SeqSpan kp = sch.kspan(s);
+                const SeqSpan kp = kCache ? sch.kspan_used(s, p.kv.seqused_k) : sch.kspan(s);
                 const int off = kp.len - sp.len;        // key position of query row 0
                 const int r_lo = blk * C::ROWS;
                 const int r_hi = min(sp.len, r_lo + C::ROWS);
                 int jb, je;
                 key_tile_range(r_lo + off, r_hi + off, kp.len, p.g.causal, p.g.window, C::BN, jb, je);
+                if constexpr (kCache) {
+                    if (!split_tile_range(p.nsplit, split, jb, je)) {
+                        --item_it;          // no tiles: no barrier phase for this item
+                        continue;
+                    }
+                }
                 if (!mbar_wait(q_empty, (item_it & 1) ^ 1, wc)) { ok = false; break; }
                 mbar_arrive_expect_tx(q_full, 2 * C::TILE_BYTES);
                 for (int t = 0; t < 2; ++t)
@@ -273,13 +329,24 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             ItemIter<false> it;
             int s, h, blk;
             for (; ok && it.next(sch, s, h, blk); ++item_it) {
+                [[maybe_unused]] int split = 0;
+                if constexpr (kCache) {
+                    split = h % p.nsplit;
+                    h /= p.nsplit;
+                }
                 const SeqSpan sp = sch.span(s);
-                const SeqSpan kp = sch.kspan(s);
+                const SeqSpan kp = kCache ? sch.kspan_used(s, p.kv.seqused_k) : sch.kspan(s);
                 const int off = kp.len - sp.len;
                 const int r_lo = blk * C::ROWS;
                 const int r_hi = min(sp.len, r_lo + C::ROWS);
                 int jb, je;
                 key_tile_range(r_lo + off, r_hi + off, kp.len, p.g.causal, p.g.window, C::BN, jb, je);
+                if constexpr (kCache) {
+                    if (!split_tile_range(p.nsplit, split, jb, je)) {
+                        --item_it;          // no tiles: no barrier phase for this item
+                        continue;
+                    }
+                }
                 if (!mbar_wait(q_full, item_it & 1, wc)) { ok = false; break; }
                 // first key tile
                 uint32_t kslot = cnt % C::NSLOT;
@@ -355,8 +422,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         ItemIter<false> it;
         int s, h, blk;
         for (; ok && it.next(sch, s, h, blk); ++item_it) {
+            [[maybe_unused]] int split = 0;
+            if constexpr (kCache) {
+                split = h % p.nsplit;
+                h /= p.nsplit;
+            }
             const SeqSpan sp = sch.span(s);
-            const SeqSpan kp = sch.kspan(s);
+            const SeqSpan kp = kCache ? sch.kspan_used(s, p.kv.seqused_k) : sch.kspan(s);
             const int n = sp.len;
             const int nk = kp.len;
             const int off = nk - n;                     // key position of query row 0
@@ -366,6 +438,15 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             key_tile_range(r_lo + off, r_hi + off, nk, p.g.causal, p.g.window, C::BN, jb, je);
             const int r0 = r_lo + t * C::BM;            // first row of this tile
             const int i = r0 + row_in_tile;             // this thread's row
+            if constexpr (kCache) {
+                if (!split_tile_range(p.nsplit, split, jb, je)) {
+                    if (i < n)
+                        p.kv.lse_part[(static_cast<size_t>(split) * H + h) * p.g.T + sp.start + i] =
+                            -INFINITY;
+                    --item_it;
+                    continue;
+                }
+            }
             float m_ref = -INFINITY;
             float l = 0.f;
             // FP8: the Q tile's scale, and the largest V block scale of the head
@@ -374,9 +455,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             const float* svh = nullptr;
             if constexpr (kF8) {
                 const size_t base = (static_cast<size_t>(s) * H + h) * p.nb;
-                skh = p.sk + base;
-                svh = p.sv + base;
-                sq_t = p.sq[base + min(r0 / C::BM, p.nb - 1)];
+                skh = p.f8.sk + base;
+                svh = p.f8.sv + base;
+                sq_t = p.f8.sq[base + min(r0 / C::BM, p.nb - 1)];
                 float mv = 0.f;
                 for (int b = lane; b < p.nb; b += 32) mv = fmaxf(mv, svh[b]);
 #pragma unroll
@@ -494,6 +575,30 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             tc_fence_after();
             const bool valid = i < n;
             const float inv_l = l > 0.f ? (kF8 ? sv_max : 1.f) / l : 0.f;
+            if constexpr (kCache) if (p.nsplit > 1) {
+                // this split's O / l (fp32) and base-2 log-sum-exp
+                float* prow = p.kv.o_part + ((static_cast<size_t>(split) * p.g.T + sp.start + i) * H + h) * D;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tO + c * 32, r);
+                    tmem_wait_ld();
+                    if (valid) {
+                        float4* dst = reinterpret_cast<float4*>(prow + c * 32);
+#pragma unroll
+                        for (int v = 0; v < 8; ++v)
+                            dst[v] = make_float4(__uint_as_float(r[4 * v]) * inv_l,
+                                                 __uint_as_float(r[4 * v + 1]) * inv_l,
+                                                 __uint_as_float(r[4 * v + 2]) * inv_l,
+                                                 __uint_as_float(r[4 * v + 3]) * inv_l);
+                    }
+                }
+                if (valid)
+                    p.kv.lse_part[(static_cast<size_t>(split) * H + h) * p.g.T + sp.start + i] =
+                        l > 0.f ? m_ref + __log2f(l) : -INFINITY;
+                tc_fence_before();
+                continue;
+            }
             __nv_bfloat16* orow = p.o + (static_cast<size_t>(sp.start) + i) * H * D +
                                   static_cast<size_t>(h) * D;
 #pragma unroll

@@ -27,7 +27,7 @@ struct Geometry {
     // Key/value sequences (equal to the query ones for self-attention).  The
     // queries of a sequence are the last ones of its key sequence, so query
     // row i sits at key position i + (nk - nq).
-    int Nk;                 // fixed key length
+    int Nk;                 // fixed key length (the rows of each sequence's slice)
     int Tk;                 // token rows of the key/value buffers
     const int* cu_seqlens_k;
 };
@@ -130,6 +130,13 @@ struct Schedule {
             return SeqSpan{a, g.cu_seqlens_k[s + 1] - a};
         }
         return SeqSpan{s * g.Nk, g.Nk};
+    }
+
+    // Key/value span of sequence s in a padded cache (fixed length): the
+    // first seqused_k[s] rows of its Nk-row slice (all Nk when seqused_k is null).
+    __device__ __forceinline__ SeqSpan kspan_used(int s, const int* seqused_k) const {
+        const int used = seqused_k ? min(max(seqused_k[s], 0), g.Nk) : g.Nk;
+        return SeqSpan{s * g.Nk, used};
     }
 
     // Blocks of the sequences before s (packed batches; 0 for fixed length).

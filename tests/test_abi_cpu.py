@@ -116,7 +116,7 @@ def kvcache(**kw):
 @pytest.mark.parametrize("kw,code", [
     (dict(q=None), -1), (dict(v_cache=None), -1),
     (dict(d=96), -2),
-    (dict(Nq=17), -3), (dict(Nk=-1), -3), (dict(num_splits=33), -3), (dict(num_splits=-1), -3),
+    (dict(Nk=-1), -3), (dict(num_splits=33), -3), (dict(num_splits=-1), -3),
     (dict(seqlens_k=P + 2), -4), (dict(o=P + 8), -4),
     (dict(causal=0, window=4), -5),
     (dict(scale=0.0), -9),

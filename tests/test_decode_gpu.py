@@ -1,6 +1,8 @@
-"""Decode against a padded key/value cache on the GPU: fa_fwd_kvcache (few
-queries per sequence, split along the keys, partials merged by a second
-kernel) through the C ABI against the float64 oracle's fwd_kvcache."""
+"""Attention against a padded key/value cache on the GPU: fa_fwd_kvcache
+through the C ABI against the float64 oracle's fwd_kvcache -- decode (few
+queries per sequence, CUDA-core kernel) and prefill chunks (more than 16
+queries, the tensor-core forward), both split along the keys with the
+partials merged by a second kernel."""
 import math
 
 import numpy as np
@@ -109,5 +111,71 @@ def test_decode_workload_parity():
     x = wl.make()
     o, lse = run_decode(poison_unused_rows(x), wl.causal, wl.window, 0)
     O, L = oracle_decode(x, wl.causal, wl.window)
+    assert_close_bf16(o, O, "O")
+    assert_lse_with_empty_rows(lse, L)
+
+
+# ------------------------------------------- prefill chunks (Nq > 16) ---
+
+def fill_unused_rows(x, value):
+    """A finite value in the cache rows past each sequence's length (the
+    forward kernel multiplies those in a shared tile by zero)."""
+    lens = x["seqlens_k"]
+    if lens is None:
+        return x
+    k, v = x["k"].clone(), x["v"].clone()
+    for b, n in enumerate(lens.tolist()):
+        k[b, n:] = value
+        v[b, n:] = value
+    return dict(x, k=k, v=v)
+
+
+PREFILL = [(2, 17, 300, 2, 128), (1, 200, 1000, 2, 64), (2, 300, 300, 1, 128),
+           (1, 257, 4096, 2, 128), (3, 129, 2000, 1, 128)]
+
+
+@pytest.mark.parametrize("B,Nq,Nk,H,d", PREFILL)
+@pytest.mark.parametrize("causal,window", [(False, 0), (True, 0), (True, 100)])
+@pytest.mark.parametrize("num_splits", [1, 2, 5, 0])
+def test_prefill_chunk_elementwise(B, Nq, Nk, H, d, causal, window, num_splits):
+    # cache lengths drawn from [0, Nk]: includes empty caches and caches
+    # shorter than the chunk (its first queries then see no key when causal)
+    x = kvcache_inputs(B, Nq, Nk, H, d, seed=Nk + 7 * Nq, lens=(0, Nk))
+    o, lse = run_decode(fill_unused_rows(x, 3.0e4), causal, window, num_splits)
+    O, L = oracle_decode(x, causal, window)
+    assert_close_bf16(o, O, "O")
+    assert_lse_with_empty_rows(lse, L)
+
+
+def test_prefill_chunk_workload():
+    # the cached-KV prefill workload (B4 H16, 2048 queries after 6144 cached
+    # keys, d128, causal) through the cache interface: 512 blocks fill the
+    # GPU, so the library does not split; same kernel as fa_fwd_kv, so the
+    # results agree bit for bit; two heads against the oracle
+    wl = WORKLOADS["prefill_kv_causal"]
+    x = wl.make()
+    q, k, v = (x[n].to(DEV) for n in ("q", "k", "v"))
+    assert fa.fa_fwd_kvcache_num_splits(wl.B, wl.H, wl.N, wl.Nk, wl.d) == 1
+    o, lse = fa.forward_kvcache(q, k, v, causal=True)
+    o1, lse1 = fa.forward_kv(q, k, v, causal=True)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_error() == 0
+    assert torch.equal(o, o1) and torch.equal(lse, lse1)
+    for s, h in ((0, 3), (2, 11)):
+        sl = {n: x[n][s:s + 1, :, h:h + 1] for n in ("q", "k", "v")}
+        sl["seqlens_k"] = None
+        O, L = oracle_decode(sl, True, 0)
+        assert_close_bf16(o[s:s + 1, :, h:h + 1], O, "O")
+        assert_lse_with_empty_rows(lse[s:s + 1, h:h + 1], L)
+
+
+def test_prefill_chunk_few_blocks_split():
+    # few blocks (B1 H2, 512 queries: 4 blocks of 256) against 8192 cached
+    # keys: the library splits the keys so the blocks spread over the SMs
+    x = kvcache_inputs(1, 512, 8192, 2, 128, seed=9, lens=[8000])
+    ns = fa.fa_fwd_kvcache_num_splits(1, 2, 512, 8192, 128)
+    assert ns > 1
+    o, lse = run_decode(fill_unused_rows(x, 0.0), True, 0, 0)
+    O, L = oracle_decode(x, True, 0)
     assert_close_bf16(o, O, "O")
     assert_lse_with_empty_rows(lse, L)
