@@ -357,6 +357,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 issue_s(1, kslot);
                 umma_commit(s_full + 1);
                 umma_commit(slot_empty + kslot);
+                if (jb + 1 == je) umma_commit(q_empty);   // the item's last S: Q is free
                 ++cnt;
                 for (int j = jb; j < je; ++j, ++step) {
                     const bool last = (j + 1 == je);
@@ -391,9 +392,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                         issue_s(1, kslot_n);
                         umma_commit(s_full + 1);
                         umma_commit(slot_empty + kslot_n);
+                        if (j + 2 == je) umma_commit(q_empty);   // the item's last S: Q is free
                         cnt += 2;
                     } else {
-                        umma_commit(q_empty);
                         cnt += 1;
                     }
                 }
