@@ -94,13 +94,17 @@ quantize_fp8_kernel(const QuantParams p) {
             c = x4[3];
             x4[1] = __fadd_rn(a, c);
             x4[3] = __fsub_rn(a, c);
-            // h = 4 .. 64: partner lane l ^ (h / 4); the lower lane keeps a + b
+            // h = 4 .. 64: partner lane l ^ (h / 4); the lower lane keeps a + b,
+            // the upper a - b (a = the lower lane's value).  One fma with a
+            // +-1 factor: the product is exact, so the single rounding gives
+            // exactly the sum or the difference.
 #pragma unroll
             for (int m = 1; m < 32; m <<= 1) {
+                const float sgn = (lane & m) ? -1.f : 1.f;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float o = __shfl_xor_sync(0xffffffffu, x4[e], m);
-                    x4[e] = (lane & m) ? __fsub_rn(o, x4[e]) : __fadd_rn(x4[e], o);
+                    x4[e] = __fmaf_rn(sgn, x4[e], o);
                 }
             }
             const float cnorm = 0.08838834764831845f;   // 1/sqrt(128), rounded to float
