@@ -292,6 +292,8 @@ int fa_profile_end(double* ms, int* counts);
  * next fa_fwd launches make their load warp skip the first V tile, so the
  * consumer's bounded wait runs out after timeout_ns nanoseconds (0 keeps the
  * default of 2 s) and the kernel returns with FA_ERR_DEVICE_TIMEOUT recorded.
+ * mode 2: the same for the decode kernel of fa_fwd_kvcache (queries <= 16):
+ * each CTA's load thread leaves its first K/V stage unloaded.
  * Host-side setting, not thread safe; returns the previous mode.
  */
 int fa_debug_set_fault(int mode, unsigned long long timeout_ns);

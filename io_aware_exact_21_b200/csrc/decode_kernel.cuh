@@ -49,6 +49,7 @@ struct DecodeParams {
     float scale_log2;          // scale * log2(e)
     int* error_word;
     uint64_t timeout_ns;
+    int fault_skip;            // test hook: the producer leaves its first tile unloaded
 };
 
 template <int D>
@@ -189,11 +190,16 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             tma_prefetch_map(&tm_k);
             tma_prefetch_map(&tm_v);
             uint32_t cnt = 0;
+            uint32_t skipped_at = 0xffffffffu;
             bool ok = true;
             for (int t = tb; t < te; ++t, ++cnt) {
                 const int slot = cnt % C::NSTAGE;
                 if (!mbar_wait(empty + slot, ((cnt / C::NSTAGE) & 1) ^ 1, wc)) { ok = false; break; }
                 mbar_arrive_expect_tx(full + slot, C::STAGE_BYTES);
+                if (p.fault_skip && cnt == 0) {
+                    skipped_at = cnt;           // test hook: this stage never fills
+                    continue;
+                }
                 uint8_t* st = smem + C::OFF_ST + slot * C::STAGE_BYTES;
                 const int row = b * p.Nk + t * C::BN;
                 for (int bx = 0; bx < C::NBOX; ++bx) {
@@ -202,9 +208,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                                 row);
                 }
             }
-            if (!ok) {
+            if (!ok || skipped_at != 0xffffffffu) {
                 // let the copies in flight land before the CTA exits
                 for (uint32_t x = cnt > C::NSTAGE ? cnt - C::NSTAGE : 0; x < cnt; ++x) {
+                    if (x == skipped_at) continue;
                     volatile int no_abort = 0;
                     WaitCtl dw{&no_abort, p.error_word, 200000000ull};
                     mbar_wait(full + x % C::NSTAGE, (x / C::NSTAGE) & 1, dw);

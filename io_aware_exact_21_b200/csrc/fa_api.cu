@@ -518,6 +518,7 @@ int fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, void
     p.scale_log2 = scale * 1.4426950408889634f;
     p.error_word = st->error_word;
     p.timeout_ns = g_fault_timeout_ns ? g_fault_timeout_ns : kDefaultTimeoutNs;
+    p.fault_skip = g_fault_mode == 2 ? 1 : 0;
     return d == 64 ? launch_decode<64>(mk, mv, p, stream) : launch_decode<128>(mk, mv, p, stream);
 }
 
