@@ -52,6 +52,14 @@
  * Asynchrony: the forward and backward entry points enqueue kernels on
  *   `stream` and return without synchronising; outputs are valid once the
  *   stream reaches them.
+ *
+ * Threads and devices: calls run on the calling thread's current CUDA
+ *   device.  The first call on a device does a one-time set-up (SM count,
+ *   the tensor-map encoder, the kernels' shared-memory limits) under a
+ *   mutex; after it, calls from several host threads and on several streams
+ *   are independent, except fa_bwd_noalloc (see there) and the per-thread
+ *   profiling counters of fa_profile_begin/end.  The device error word is
+ *   shared by all calls on a device.
  */
 #ifndef FA_B200_H
 #define FA_B200_H

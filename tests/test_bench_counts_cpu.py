@@ -1,0 +1,69 @@
+"""The bench's counted work and its traffic bookkeeping, on the CPU: the FLOP
+counts of the training step and the cached-KV prefill against a direct count
+of allowed (query, key) pairs, the decode byte count against the used cache
+rows, and the rule that a stored ncu traffic figure is dropped once the
+kernel sources it was captured on change."""
+import hashlib
+import os
+
+import numpy as np
+
+import bench
+from io_aware_exact_21_b200.inputs import WORKLOADS
+
+
+def _pairs(nq, nk, causal):
+    i = np.arange(nq)[:, None] + (nk - nq)
+    j = np.arange(nk)[None, :]
+    allowed = np.ones((nq, nk), bool)
+    if causal:
+        allowed &= j <= i
+    return int(allowed.sum())
+
+
+def test_training_flops_are_the_dense_convention():
+    # forward 4*d per (query, key) pair of the full square, halved when causal;
+    # backward 2.5 x forward (five GEMMs)
+    f, b = bench.flops(4, 16, 8192, 128, False)
+    assert f == 4.0 * 4 * 16 * 8192 * 8192 * 128 and b == 2.5 * f
+    fc, bc = bench.flops(4, 16, 8192, 128, True)
+    assert fc == f / 2 and bc == b / 2
+    # the halved count is within 1/N of the exact causal pair count
+    n = 512
+    exact = 4.0 * _pairs(n, n, True) * 64
+    assert abs(bench.flops(1, 1, n, 64, True)[0] - exact) / exact < 1.0 / n
+
+
+def test_cached_kv_flops_count_the_allowed_pairs():
+    # Nq*Nk - Nq^2/2 pairs under the bottom-right causal mask (the triangle of
+    # the last Nq positions halved, as in the self-attention count)
+    for nq, nk in ((64, 256), (128, 128), (100, 1000)):
+        exact = 4.0 * _pairs(nq, nk, True) * 128
+        got = bench.flops_kv(1, 1, nq, nk, 128, True)
+        assert abs(got - exact) / exact < 1.0 / nq
+        assert bench.flops_kv(1, 1, nq, nk, 128, False) == 4.0 * nq * nk * 128
+
+
+def test_decode_bytes_are_the_used_cache_rows():
+    wl = WORKLOADS["decode"]
+    lens = [4096, 5000, 8192] + [6000] * (wl.B - 3)
+    kv = 2 * sum(lens) * wl.H * wl.d * 2
+    qo = 2 * wl.B * wl.N * wl.H * wl.d * 2 + wl.B * wl.H * wl.N * 4
+    assert bench.decode_bytes(wl, lens) == kv + qo
+
+
+def test_traffic_figure_is_dropped_when_its_sources_change(monkeypatch, tmp_path):
+    # a stored figure is reported only while the hash of its sources matches
+    entry = bench.TRAFFIC["dkdv"]
+    h = hashlib.sha256()
+    for f in entry["sources"]:
+        with open(os.path.join(bench.ROOT, "io_aware_exact_21_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    current = h.hexdigest()[:16]
+    monkeypatch.setitem(bench.TRAFFIC, "dkdv", dict(entry, sha=current))
+    assert bench.traffic_for("dkdv") == entry["bytes_per_launch"]
+    monkeypatch.setitem(bench.TRAFFIC, "dkdv", dict(entry, sha="0" * 16))
+    assert bench.traffic_for("dkdv") is None
+    # and only for the workload it was captured on
+    monkeypatch.setitem(bench.TRAFFIC, "dkdv", dict(entry, sha=current))
+    assert bench.traffic_for("dkdv", "decode") is None
