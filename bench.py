@@ -667,11 +667,13 @@ def run_decode(args, rank, world, device):
     }
 
 
-def oracle_sample_decode():
-    """The float64 oracle's decode on the whole decode workload."""
+def oracle_sample_decode(x=None):
+    """The float64 oracle's decode on the whole decode workload (its inputs
+    made here unless given)."""
     from oracle import oracle as orc
     wl = decode_workload()
-    x = wl.make()
+    if x is None:
+        x = wl.make()
     t0 = time.perf_counter()
     orc.fwd_kvcache(x["q"], x["k"], x["v"], wl.scale, seqlens_k=x["seqlens_k"],
                     causal=wl.causal, window=wl.window)
@@ -873,6 +875,37 @@ def oracle_sample(n_tokens=None, seed=2):
     return (f_fwd + f_bwd) / secs / 1e12, desc, orc.num_threads(), secs
 
 
+CPU_SAMPLE_MIN_S = 10.0
+
+
+def cpu_baseline_sample(workload, min_secs=CPU_SAMPLE_MIN_S, max_reps=64):
+    """The cpu_baseline leg: the workload's oracle sample, repeated (a new
+    input seed each time, where the sample takes one) until at least
+    min_secs of host time have been spent.  Returns (rate over all samples,
+    description, threads)."""
+    work = total = 0.0
+    reps = 0
+    first = threads = None
+    dec_inputs = decode_workload().make() if workload == "decode" else None
+    while reps < max_reps and (reps == 0 or total < min_secs):
+        if workload == "train":
+            val, desc, threads, secs = oracle_sample(seed=2 + reps)
+        elif workload == "prefill_kv":
+            val, desc, threads, secs = oracle_sample_kv(seed=5 + reps)
+        elif workload == "fp8":
+            val, desc, threads, secs = oracle_sample_fp8(seed=2 + reps)
+        else:
+            val, desc, threads, secs = oracle_sample_decode(dec_inputs)
+        work += val * secs
+        total += secs
+        reps += 1
+        first = first or desc
+    desc = "%s; %d such sample%s%s, %.1f s in total" % (
+        first, reps, "s" if reps > 1 else "",
+        "" if workload == "decode" else " (input seed +1 each)", total)
+    return work / total, desc, threads
+
+
 def run_reference(args):
     """Reference arm: the float64 CPU oracle as it stands, timed on the host
     cores, one bounded sample of the workload per step."""
@@ -988,13 +1021,11 @@ def main():
                                              device_id=device)
     runner = {"train": run_ours, "prefill_kv": run_prefill_kv, "decode": run_decode,
               "fp8": run_fp8}[args.workload]
-    sampler = {"train": oracle_sample, "prefill_kv": oracle_sample_kv,
-               "decode": oracle_sample_decode, "fp8": oracle_sample_fp8}[args.workload]
     try:
         out = runner(args, rank, world, device)
         if out is not None:
             if not args.no_cpu_baseline and world == 1:
-                val, desc, threads, secs = sampler()
+                val, desc, threads = cpu_baseline_sample(args.workload)
                 out["cpu_baseline"] = {"value": val, "unit": out["unit"], "cores": threads,
                                        "kind": "oracle", "sample": desc}
             else:

@@ -67,3 +67,19 @@ def test_traffic_figure_is_dropped_when_its_sources_change(monkeypatch, tmp_path
     # and only for the workload it was captured on
     monkeypatch.setitem(bench.TRAFFIC, "dkdv", dict(entry, sha=current))
     assert bench.traffic_for("dkdv", "decode") is None
+
+
+def test_cpu_baseline_repeats_until_the_time_floor(monkeypatch):
+    # the cpu_baseline leg repeats the oracle sample with a new seed each
+    # time and reports the rate over all samples
+    calls = []
+
+    def fake(seed=5):
+        calls.append(seed)
+        return 2.0 * len(calls), "one sample", 4, 1.0     # rate, description, threads, seconds
+
+    monkeypatch.setattr(bench, "oracle_sample_kv", fake)
+    rate, desc, threads = bench.cpu_baseline_sample("prefill_kv", min_secs=3.0)
+    assert calls == [5, 6, 7]
+    assert rate == (2.0 + 4.0 + 6.0) / 3.0 and threads == 4
+    assert "3 such samples" in desc and "3.0 s in total" in desc
