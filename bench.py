@@ -59,37 +59,77 @@ NOMINAL_BF16_DENSE_TFLOPS = 2250.0
 # ncu captures.  Training step and FP8 forward: the B=2 H=16 N=8192 d=128
 # non-causal case, scaled by 2 to the B=4 workload (each kernel's traffic grows
 # with the number of heads it processes).  Decode: the decode workload itself.  Valid only for
-# the kernel sources a capture was taken on: each entry carries a hash of them
-# and is reported as null once they change.  Summaries and commands:
+# the kernel sources a capture was taken on: each entry carries a hash of their
+# comment-free text and is reported as null once that changes.  Summaries and commands:
 # profiles/*_kernel_*.md.
 TRAFFIC = {
     "fwd": {"bytes_per_launch": 2 * (207.10e6 + 48.93e6), "workload": "train",
-            "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh"), "sha": "24296b4dd9e32e50"},
+            "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh"), "sha": "db7381e1f845ff58"},
     "dkdv": {"bytes_per_launch": 2 * (271.87e6 + 107.11e6), "workload": "train",
-             "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "2cc387b6c0427932"},
+             "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "eac9bf149dae49e0"},
     "dq": {"bytes_per_launch": 2 * (271.07e6 + 53.35e6), "workload": "train",
-           "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "2cc387b6c0427932"},
+           "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "eac9bf149dae49e0"},
     "decode": {"bytes_per_launch": 792.82e6 + 5.62e6, "workload": "decode",
-               "sources": ("decode_kernel.cuh", "sm100.cuh"), "sha": "52c6df8de384d880"},
+               "sources": ("decode_kernel.cuh", "sm100.cuh"), "sha": "5424c1188ad151db"},
     "fwd_fp8": {"bytes_per_launch": 2 * (101.02e6 + 32.14e6), "workload": "fp8",
-                "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh"), "sha": "24296b4dd9e32e50"},
+                "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh"), "sha": "db7381e1f845ff58"},
 }
+
+
+def strip_comments(text):
+    """C/C++ source without its comments and blank lines, trailing spaces
+    removed: what the compiler sees, so that a comment edit does not count as
+    a kernel change."""
+    out, i, n = [], 0, len(text)
+    in_str = False
+    while i < n:
+        c = text[i]
+        if in_str:
+            out.append(c)
+            if c == "\\" and i + 1 < n:
+                out.append(text[i + 1])
+                i += 2
+                continue
+            if c == '"':
+                in_str = False
+            i += 1
+        elif c == '"':
+            in_str = True
+            out.append(c)
+            i += 1
+        elif text.startswith("//", i):
+            while i < n and text[i] != "\n":
+                i += 1
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = (ln.rstrip() for ln in "".join(out).split("\n"))
+    return "\n".join(ln for ln in lines if ln)
+
+
+def source_hash(files):
+    """Hash of the comment-free text of kernel sources under csrc/, or None
+    if one is missing."""
+    import hashlib
+    h = hashlib.sha256()
+    try:
+        for f in files:
+            with open(os.path.join(ROOT, "io_aware_exact_21_b200", "csrc", f), encoding="utf-8") as fh:
+                h.update(strip_comments(fh.read()).encode())
+    except OSError:
+        return None
+    return h.hexdigest()[:16]
 
 
 def traffic_for(kernel, workload="train"):
     """ncu traffic per launch if the kernel's sources still match the capture."""
-    import hashlib
     t = TRAFFIC.get(kernel)
     if not t or t["workload"] != workload:
         return None
-    h = hashlib.sha256()
-    try:
-        for f in t["sources"]:
-            with open(os.path.join(ROOT, "io_aware_exact_21_b200", "csrc", f), "rb") as fh:
-                h.update(fh.read())
-    except OSError:
-        return None
-    if h.hexdigest()[:16] != t["sha"]:
+    if source_hash(t["sources"]) != t["sha"]:
         return None
     if workload in ("train", "fp8"):
         w = WORKLOAD

@@ -104,7 +104,7 @@ __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* map) {
 }
 
 // 3-D tiled load, box coordinates (c0 innermost).  Completion is signalled on
-// `bar` through its transaction count.  No multicast.
+// `bar` through its transaction count.  Into this CTA's shared memory only.
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
                                             int c0, int c1, int c2) {
     asm volatile(
@@ -115,7 +115,7 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
         : "memory");
 }
 
-// 2-D tiled load, box coordinates (c0 innermost).  No multicast.
+// 2-D tiled load, box coordinates (c0 innermost), into this CTA's shared memory.
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
                                             int c0, int c1) {
     asm volatile(
@@ -128,7 +128,7 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
 
 // Contiguous global -> shared copy of `bytes` (multiple of 16, both
 // addresses 16-byte aligned), completion on `bar` through its transaction
-// count.  No multicast.
+// count.  Into this CTA's shared memory only.
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes,
                                           uint64_t* bar) {
     asm volatile(

@@ -3,9 +3,6 @@ counts of the training step and the cached-KV prefill against a direct count
 of allowed (query, key) pairs, the decode byte count against the used cache
 rows, and the rule that a stored ncu traffic figure is dropped once the
 kernel sources it was captured on change."""
-import hashlib
-import os
-
 import numpy as np
 
 import bench
@@ -55,11 +52,7 @@ def test_decode_bytes_are_the_used_cache_rows():
 def test_traffic_figure_is_dropped_when_its_sources_change(monkeypatch, tmp_path):
     # a stored figure is reported only while the hash of its sources matches
     entry = bench.TRAFFIC["dkdv"]
-    h = hashlib.sha256()
-    for f in entry["sources"]:
-        with open(os.path.join(bench.ROOT, "io_aware_exact_21_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
-    current = h.hexdigest()[:16]
+    current = bench.source_hash(entry["sources"])
     monkeypatch.setitem(bench.TRAFFIC, "dkdv", dict(entry, sha=current))
     assert bench.traffic_for("dkdv") == entry["bytes_per_launch"]
     monkeypatch.setitem(bench.TRAFFIC, "dkdv", dict(entry, sha="0" * 16))
@@ -83,3 +76,14 @@ def test_cpu_baseline_repeats_until_the_time_floor(monkeypatch):
     assert calls == [5, 6, 7]
     assert rate == (2.0 + 4.0 + 6.0) / 3.0 and threads == 4
     assert "3 such samples" in desc and "3.0 s in total" in desc
+
+
+def test_source_hash_ignores_comments_only():
+    # a comment or blank-line edit keeps the hash (the compiler sees the same
+    # code); any change to code, including inside a string, does not
+    base = 'int a = 1;  // the count\nconst char* s = "x // y";\n'
+    assert bench.strip_comments(base) == bench.strip_comments(
+        '/* header */\nint a = 1;\n\nconst char* s = "x // y";  // note\n')
+    assert bench.strip_comments(base) != bench.strip_comments(base.replace("1;", "2;"))
+    assert bench.strip_comments(base) != bench.strip_comments(base.replace("x // y", "x // z"))
+
