@@ -207,11 +207,57 @@ def fa_profile_end():
 
 
 # ------------------------------------------------------ tensor helpers ---
+#
+# The library reads and writes exactly the elements its size arguments imply,
+# from each base pointer, in the documented dtype and dense layout.  The
+# wrappers below derive those sizes from the tensors and refuse any tensor
+# that does not match them (dtype, shape, contiguity, device), so that a
+# mismatch raises here instead of making a kernel touch memory outside a
+# tensor.  The raw fa_* functions above take pointers and do no such check.
+
+def _require_cuda(t, name):
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+
+
+def _expect(t, name, shape, dtype, device):
+    if t is None:
+        raise ValueError("%s is required" % name)
+    _require_cuda(t, name)
+    if t.device != device:
+        raise ValueError("%s is on %s, expected %s" % (name, t.device, device))
+    if t.dtype != dtype:
+        raise TypeError("%s has dtype %s, expected %s" % (name, t.dtype, dtype))
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), tuple(shape)))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+def _expect_bytes(t, name, nbytes, device):
+    """A byte buffer (workspace): uint8, dense, at least nbytes long."""
+    import torch
+    _require_cuda(t, name)
+    if t.device != device:
+        raise ValueError("%s is on %s, expected %s" % (name, t.device, device))
+    if t.dtype != torch.uint8 or not t.is_contiguous():
+        raise TypeError("%s must be a contiguous uint8 tensor" % name)
+    if t.numel() < nbytes:
+        raise ValueError("%s holds %d bytes, %d needed" % (name, t.numel(), nbytes))
+
+
+def _rank(t, name, ranks):
+    if t is None or t.dim() not in ranks:
+        raise ValueError("%s must have %s dimensions" % (name, " or ".join(map(str, ranks))))
+
 
 def _shape(q, cu_seqlens):
     if cu_seqlens is None:
+        _rank(q, "q", (4,))
         B, N, H, d = q.shape
         return B, H, N, d
+    _rank(q, "q (packed)", (3,))
+    _rank(cu_seqlens, "cu_seqlens", (1,))
     T, H, d = q.shape
     return cu_seqlens.numel() - 1, H, T, d
 
@@ -222,13 +268,20 @@ def forward(q, k, v, causal=False, window=0, cu_seqlens=None, scale=None, out=No
     int32 ``cu_seqlens``).  Outputs are allocated with torch when not given."""
     import torch
     B, H, N, d = _shape(q, cu_seqlens)
+    dev = q.device
+    lse_shape = (B, H, N) if cu_seqlens is None else (H, N)
+    for t, name in ((q, "q"), (k, "k"), (v, "v")):
+        _expect(t, name, q.shape, torch.bfloat16, dev)
+    if cu_seqlens is not None:
+        _expect(cu_seqlens, "cu_seqlens", (B + 1,), torch.int32, dev)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
-        lse = torch.empty((B, H, N) if cu_seqlens is None else (H, N), dtype=torch.float32,
-                          device=q.device)
+        lse = torch.empty(lse_shape, dtype=torch.float32, device=dev)
+    _expect(out, "out", q.shape, torch.bfloat16, dev)
+    _expect(lse, "lse", lse_shape, torch.float32, dev)
     _check(fa_fwd(q, k, v, out, lse, B, H, N, d, scale, causal, window, cu_seqlens, stream),
            "fa_fwd")
     return out, lse
@@ -240,18 +293,32 @@ def forward_kv(q, k, v, causal=False, window=0, cu_seqlens_q=None, cu_seqlens_k=
     [B, Nk, H, d] (or packed [Tq, H, d] / [Tk, H, d] with int32 cu_seqlens_q
     and cu_seqlens_k); queries are the last positions of their key sequence."""
     import torch
+    if (cu_seqlens_q is None) != (cu_seqlens_k is None):
+        raise ValueError("cu_seqlens_q and cu_seqlens_k go together")
     B, H, Nq, d = _shape(q, cu_seqlens_q)
+    dev = q.device
+    _expect(q, "q", q.shape, torch.bfloat16, dev)
     if cu_seqlens_q is None:
+        _rank(k, "k", (4,))
         Nk = k.shape[1]
+        kv_shape = (B, Nk, H, d)
     else:
+        _rank(k, "k (packed)", (3,))
         Nk = k.shape[0]
+        kv_shape = (Nk, H, d)
+        _expect(cu_seqlens_q, "cu_seqlens_q", (B + 1,), torch.int32, dev)
+        _expect(cu_seqlens_k, "cu_seqlens_k", (B + 1,), torch.int32, dev)
+    _expect(k, "k", kv_shape, torch.bfloat16, dev)
+    _expect(v, "v", kv_shape, torch.bfloat16, dev)
+    lse_shape = (B, H, Nq) if cu_seqlens_q is None else (H, Nq)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
-        lse = torch.empty((B, H, Nq) if cu_seqlens_q is None else (H, Nq), dtype=torch.float32,
-                          device=q.device)
+        lse = torch.empty(lse_shape, dtype=torch.float32, device=dev)
+    _expect(out, "out", q.shape, torch.bfloat16, dev)
+    _expect(lse, "lse", lse_shape, torch.float32, dev)
     _check(fa_fwd_kv(q, k, v, out, lse, B, H, Nq, Nk, d, scale, causal, window, cu_seqlens_q,
                      cu_seqlens_k, stream), "fa_fwd_kv")
     return out, lse
@@ -264,18 +331,30 @@ def forward_kvcache(q, k_cache, v_cache, seqlens_k=None, causal=False, window=0,
     b uses its first seqlens_k[b] rows (int32 CUDA tensor, or None for all Nk);
     queries are the last Nq of those positions.  Returns (O, LSE)."""
     import torch
+    _rank(q, "q", (4,))
+    _rank(k_cache, "k_cache", (4,))
     B, Nq, H, d = q.shape
     Nk = k_cache.shape[1]
+    dev = q.device
+    _expect(q, "q", q.shape, torch.bfloat16, dev)
+    _expect(k_cache, "k_cache", (B, Nk, H, d), torch.bfloat16, dev)
+    _expect(v_cache, "v_cache", (B, Nk, H, d), torch.bfloat16, dev)
+    if seqlens_k is not None:
+        _expect(seqlens_k, "seqlens_k", (B,), torch.int32, dev)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
-        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=dev)
+    _expect(out, "out", q.shape, torch.bfloat16, dev)
+    _expect(lse, "lse", (B, H, Nq), torch.float32, dev)
     ns = num_splits if num_splits > 0 else fa_fwd_kvcache_num_splits(B, H, Nq, Nk, d)
     need = fa_fwd_kvcache_workspace_size(B, H, Nq, d, ns)
     if need and workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if workspace is not None:
+        _expect_bytes(workspace, "workspace", need, dev)
     _check(fa_fwd_kvcache(q, k_cache, v_cache, out, lse, B, H, Nq, Nk, d, scale, causal, window,
                           seqlens_k, ns, workspace,
                           0 if workspace is None else workspace.numel(), stream),
@@ -289,9 +368,14 @@ def quantize_fp8(q, k, v, signs=None, stream=None):
     128, Np]) and their scales sq, sk, sv [B, H, ceil(N / 128)].  signs (128
     floats of +-1 on the device) rotates Q and K first."""
     import torch
+    _rank(q, "q", (4,))
     B, N, H, d = q.shape
     nb = (N + 127) // 128
     dev = q.device
+    for t, name in ((q, "q"), (k, "k"), (v, "v")):
+        _expect(t, name, q.shape, torch.bfloat16, dev)
+    if signs is not None:
+        _expect(signs, "signs", (d,), torch.float32, dev)
     out = {"q8": torch.empty((B, N, H, d), dtype=torch.uint8, device=dev),
            "k8": torch.empty((B, N, H, d), dtype=torch.uint8, device=dev),
            "vt8": torch.empty(max(1, fa_fp8_vt_bytes(B, H, N, d)), dtype=torch.uint8, device=dev),
@@ -311,10 +395,18 @@ def forward_fp8(qz, B, N, H, d=128, causal=False, window=0, scale=None, out=None
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     dev = qz["q8"].device
+    nb = (N + 127) // 128
+    _expect(qz["q8"], "q8", (B, N, H, d), torch.uint8, dev)
+    _expect(qz["k8"], "k8", (B, N, H, d), torch.uint8, dev)
+    _expect_bytes(qz["vt8"], "vt8", fa_fp8_vt_bytes(B, H, N, d), dev)
+    for name in ("sq", "sk", "sv"):
+        _expect(qz[name], name, (B, H, nb), torch.float32, dev)
     if out is None:
         out = torch.empty((B, N, H, d), dtype=torch.bfloat16, device=dev)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    _expect(out, "out", (B, N, H, d), torch.bfloat16, dev)
+    _expect(lse, "lse", (B, H, N), torch.float32, dev)
     _check(fa_fwd_fp8(qz["q8"], qz["k8"], qz["vt8"], qz["sq"], qz["sk"], qz["sv"], out, lse, B, H,
                       N, d, scale, causal, window, stream), "fa_fwd_fp8")
     return out, lse
@@ -325,14 +417,23 @@ def backward(q, k, v, o, lse, dout, causal=False, window=0, cu_seqlens=None, sca
     """dQ, dK, dV for the forward's (O, LSE) and the output gradient dO."""
     import torch
     B, H, N, d = _shape(q, cu_seqlens)
+    dev = q.device
+    for t, name in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _expect(t, name, q.shape, torch.bfloat16, dev)
+    _expect(lse, "lse", (B, H, N) if cu_seqlens is None else (H, N), torch.float32, dev)
+    if cu_seqlens is not None:
+        _expect(cu_seqlens, "cu_seqlens", (B + 1,), torch.int32, dev)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if grads is None:
         grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
     dq, dk, dv = grads
+    for t, name in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _expect(t, name, q.shape, torch.bfloat16, dev)
     ws_bytes = fa_bwd_workspace_size(B, H, N, d, N if cu_seqlens is not None else 0)
     if workspace is None:
-        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    _expect_bytes(workspace, "workspace", ws_bytes, dev)
     _check(fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, window,
                   cu_seqlens, workspace, workspace.numel(), stream), "fa_bwd")
     return dq, dk, dv
