@@ -1,0 +1,179 @@
+// Host build of the kernels' tile schedule and mask classification
+// (io_aware_exact_21_b200/csrc/schedule.cuh), checked for the invariants the
+// kernels rely on:
+//   1. every (sequence, head, row block) is visited by exactly one CTA, for
+//      the pair walk and the pair + snake-tail walk, for fixed-length and
+//      packed batches and for several grid sizes;
+//   2. the key-tile range of a block holds every key any of its rows may see,
+//      and the tiles outside it hold none;
+//   3. a tile classified as needing no mask has every (row, key) pair of the
+//      block allowed.
+// The CUDA built-ins the header reads (blockIdx, gridDim, threadIdx,
+// blockDim, __syncthreads) are host variables here; the packed-batch prefix
+// is built by one emulated thread.  Prints "ok" and exits 0, or names the
+// first violation and exits 1.
+#include <algorithm>
+#include <cstdio>
+#include <cstdlib>
+#include <map>
+#include <random>
+#include <tuple>
+#include <vector>
+
+#define __device__
+#define __forceinline__ inline
+using std::max;
+using std::min;
+struct Dim3 {
+    unsigned x = 0, y = 1, z = 1;
+};
+static Dim3 blockIdx, gridDim, threadIdx, blockDim;
+static inline void __syncthreads() {}
+
+#include "schedule.cuh"
+
+namespace {
+
+int failures = 0;
+
+void fail(const char* what, int a, int b, int c, int d) {
+    if (failures++ < 10) std::printf("FAIL %s (%d %d %d %d)\n", what, a, b, c, d);
+}
+
+// Visit every CTA's walk and count the (s, h, blk) it yields.
+template <bool kTail>
+void check_cover(const fa::Geometry& g, const std::vector<int>& lens, int rows_per_item, int order,
+                 int G) {
+    std::vector<int> bpre(fa::kMaxVarlenSeqs + 1), upre(fa::kMaxVarlenSeqs + 1);
+    std::vector<int> scratch(2);
+    fa::Schedule sch;
+    sch.g = g;
+    sch.rows_per_item = rows_per_item;
+    sch.order = order;
+    sch.bprefix = bpre.data();
+    sch.uprefix = upre.data();
+    blockDim.x = 1;
+    threadIdx.x = 0;
+    gridDim.x = G;
+    sch.total_units = fa::build_schedule_prefix(g, rows_per_item, bpre.data(), upre.data(),
+                                                scratch.data());
+    fa::schedule_split_tail(sch);
+    std::map<std::tuple<int, int, int>, int> seen;
+    for (int c = 0; c < G; ++c) {
+        blockIdx.x = c;
+        fa::ItemIter<kTail> it;
+        int s, h, blk, guard = 0;
+        while (it.next(sch, s, h, blk)) {
+            if (++guard > 1000000) {
+                fail("walk does not end", c, G, rows_per_item, order);
+                return;
+            }
+            ++seen[std::make_tuple(s, h, blk)];
+        }
+    }
+    size_t expected = 0;
+    for (int s = 0; s < g.B; ++s) {
+        const int n = lens[s];
+        const int nb = (n + rows_per_item - 1) / rows_per_item;
+        for (int h = 0; h < g.H; ++h)
+            for (int b = 0; b < nb; ++b) {
+                ++expected;
+                auto f = seen.find(std::make_tuple(s, h, b));
+                const int cnt = f == seen.end() ? 0 : f->second;
+                if (cnt != 1) fail("block visited != once", s, h, b, cnt);
+            }
+    }
+    if (seen.size() != expected) fail("walk yields blocks outside the batch", (int)seen.size(),
+                                      (int)expected, G, order);
+}
+
+void check_masks(std::mt19937& rng) {
+    const int BN = 128;
+    for (int trial = 0; trial < 400; ++trial) {
+        const int nk = 1 + rng() % 1500;
+        const int nq = 1 + rng() % nk;              // queries: the last nq key positions
+        const int off = nk - nq;
+        const int causal = rng() % 4 != 0;
+        const int window = causal && rng() % 2 ? 1 + rng() % 300 : 0;
+        const int rows = rng() % 2 ? 128 : 256;
+        for (int r_lo = 0; r_lo < nq; r_lo += rows) {
+            const int r_hi = min(nq, r_lo + rows);
+            int jb, je;
+            fa::key_tile_range(r_lo + off, r_hi + off, nk, causal, window, BN, jb, je);
+            if (jb < 0 || je <= jb) fail("empty or negative tile range", jb, je, nk, nq);
+            const int ntiles = (nk + BN - 1) / BN;
+            for (int t = 0; t < max(ntiles, je); ++t) {
+                bool any = false, all = true;
+                for (int i = r_lo; i < r_hi; ++i)
+                    for (int k = t * BN; k < (t + 1) * BN; ++k) {
+                        const bool a = fa::key_allowed(i + off, k, nk, causal, window);
+                        any = any || a;
+                        all = all && a;
+                    }
+                const bool inside = t >= jb && t < je;
+                if (any && !inside) fail("allowed key outside the tile range", t, jb, je, nk);
+                if (inside && !fa::tile_needs_mask_pos(r_lo + off, r_hi + off, t * BN, BN, nk,
+                                                       causal, window) && !all)
+                    fail("unmasked tile holds a disallowed pair", t, r_lo, nk, window);
+            }
+        }
+    }
+}
+
+}  // namespace
+
+int main() {
+    std::mt19937 rng(12345);
+    // fixed length: pairs, and pairs + snake tail in both cost directions
+    const int grids[] = {1, 7, 148, 300};
+    const int shapes[][3] = {{4, 16, 8192}, {4, 16, 2048}, {2, 16, 4096}, {1, 1, 128},
+                             {3, 5, 1000}, {1, 2, 65536}, {64, 32, 128}, {2, 3, 257}};
+    for (auto& sh : shapes) {
+        for (int causal = 0; causal < 2; ++causal) {
+            fa::Geometry g{};
+            g.B = sh[0];
+            g.H = sh[1];
+            g.N = sh[2];
+            g.T = sh[0] * sh[2];
+            g.causal = causal;
+            g.Nk = sh[2];
+            g.Tk = g.T;
+            std::vector<int> lens(g.B, g.N);
+            for (int G : grids)
+                for (int rows : {128, 256}) {
+                    check_cover<false>(g, lens, rows, 0, G);
+                    const int order = fa::schedule_order(g, 1);
+                    check_cover<true>(g, lens, rows, order, G);
+                    check_cover<true>(g, lens, rows, -order, G);
+                }
+        }
+    }
+    // packed batches (pairs only): random lengths, including empty sequences
+    for (int trial = 0; trial < 30; ++trial) {
+        const int B = 1 + rng() % 40;
+        std::vector<int> lens(B), cu(B + 1, 0);
+        for (int s = 0; s < B; ++s) {
+            lens[s] = rng() % 5 == 0 ? 0 : 1 + rng() % 3000;
+            cu[s + 1] = cu[s] + lens[s];
+        }
+        fa::Geometry g{};
+        g.B = B;
+        g.H = 1 + rng() % 8;
+        g.N = 0;
+        g.T = cu[B];
+        g.cu_seqlens = cu.data();
+        g.causal = rng() % 2;
+        g.Nk = 0;
+        g.Tk = g.T;
+        g.cu_seqlens_k = cu.data();
+        for (int G : grids) check_cover<false>(g, lens, 256, 0, G);
+        for (int G : grids) check_cover<true>(g, lens, 128, fa::schedule_order(g, 1), G);
+    }
+    check_masks(rng);
+    if (failures) {
+        std::printf("%d violations\n", failures);
+        return 1;
+    }
+    std::printf("ok\n");
+    return 0;
+}
