@@ -1,8 +1,9 @@
 """Python face of the float64 CPU oracle (``attn_oracle.c``).
 
 TEST INFRASTRUCTURE ONLY: imported by ``tests/``, by ``__graft_entry__.smoke``
-and by the CPU-baseline leg of ``bench.py``.  The CUDA library never imports
-it, and it imports nothing from the CUDA package.
+and by ``bench.py``'s CPU-baseline leg and its ``--impl reference`` arm (the
+oracle timed on the host cores).  The CUDA library never imports it, and it
+imports nothing from the CUDA package.
 
 The oracle computes, in float64 from exact upcasts of the (bf16) inputs, the
 definition of scaled-dot-product attention, ``O = softmax(scale * Q K^T) V``
