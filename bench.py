@@ -60,8 +60,7 @@ NOMINAL_BF16_DENSE_TFLOPS = 2250.0
 # non-causal case, scaled by 2 to the B=4 workload (each kernel's traffic grows
 # with the number of heads it processes).  Decode: the decode workload itself.  Valid only for
 # the kernel sources a capture was taken on: each entry carries a hash of their
-# comment-free text and is reported as null once that changes.  Summaries and commands:
-# profiles/*_kernel_*.md.
+# comment-free text and is reported as null once that changes.
 TRAFFIC = {
     "fwd": {"bytes_per_launch": 2 * (207.10e6 + 48.93e6), "workload": "train",
             "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh"), "sha": "db7381e1f845ff58"},
@@ -376,6 +375,11 @@ def run_ours(args, rank, world, device):
     assert fa.fa_get_device_error() == 0
 
     elapsed, e2e_elapsed = max_over_ranks([elapsed, e2e_elapsed], world, device)
+    configs = None
+    if not args.no_configs:
+        del sets, pin
+        torch.cuda.empty_cache()
+        configs = sweep_configs(device)
     if rank != 0:
         return None
 
@@ -388,19 +392,40 @@ def run_ours(args, rank, world, device):
     per_kernel = {}
     for kind, (ms, cnt) in prof.items():
         per_kernel[kind] = {"ms_per_launch": ms / cnt if cnt else None, "launches": cnt}
-    # dominant kernel by total device time
-    dom = max(prof, key=lambda kk: prof[kk][0])
-    dom_ms = per_kernel[dom]["ms_per_launch"]
-    # algorithmic FLOPs per launch: forward 4BHN^2d; dK/dV kernel = the dV and dK
-    # GEMMs plus the S and dP recomputation it needs (4 x 2BHN^2d, of which the
-    # counted backward work assigns it 2 + 2 ... reported below as executed).
-    kernel_flops = {"fwd": f_fwd, "dkdv": 2.0 * f_fwd, "dq": 1.5 * f_fwd, "dot": 0.0}
-    peak_key = "bf16_tflops_sustained" if peak_src == "measured" else "bf16_tflops"
-    peak = peaks.get(peak_key, FALLBACK_PEAKS["bf16_tflops"])
-    achieved = kernel_flops[dom] / (dom_ms * 1e-3) / 1e12 if dom_ms else None
+    # Per-kernel rooflines.  Algorithmic FLOPs per launch are the GEMMs each
+    # kernel executes: forward 4BHN^2d (S and PV); dK/dV kernel 4 GEMMs of
+    # 2BHN^2d (S^T, dP^T, dV, dK); dQ kernel 3 (S, dP, dQ); halved under a causal
+    # mask.  The pre-pass is HBM-bound: it reads dO, O and LSE and writes the
+    # 8-byte statistics, 4d + 12 bytes per (row, head).  The kernels are timed
+    # inside a sub-second loop, so the denominator is the measured burst peak.
+    kernel_flops = {"fwd": f_fwd, "dkdv": 2.0 * f_fwd, "dq": 1.5 * f_fwd}
+    peak_key = "bf16_tflops"
+    peak = peaks.get(peak_key, FALLBACK_PEAKS[peak_key])
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    stats_bytes = float(B) * N * H * (4 * d + 12)
+    rooflines = {}
+    for kk in ("fwd", "dkdv", "dq", "dot"):
+        ms = per_kernel[kk]["ms_per_launch"]
+        if not ms:
+            continue
+        if kk == "dot":
+            ach = stats_bytes / (ms * 1e-3) / 1e9
+            rooflines[kk] = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm,
+                             "unit": "GB/s", "frac": round(ach / hbm, 4),
+                             "algorithmic": stats_bytes, "ms": round(ms, 4),
+                             "traffic": traffic_for(kk)}
+        else:
+            ach = kernel_flops[kk] / (ms * 1e-3) / 1e12
+            rooflines[kk] = {"bound": "tensor", "achieved": round(ach, 2), "peak": peak,
+                             "unit": "TFLOP/s", "frac": round(ach / peak, 4),
+                             "algorithmic": kernel_flops[kk], "ms": round(ms, 4),
+                             "traffic": traffic_for(kk)}
+    # dominant kernel: the largest device time per step
+    dom = max(("fwd", "dkdv", "dq"), key=lambda kk: prof[kk][0])
+    achieved = rooflines[dom]["achieved"]
     t_fwd = per_kernel["fwd"]["ms_per_launch"]
     t_bwd = sum(per_kernel[kk]["ms_per_launch"] or 0.0 for kk in ("dot", "dkdv", "dq"))
-    burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    burst = peak
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
@@ -418,12 +443,13 @@ def run_ours(args, rank, world, device):
                 "kernels_ms": {kk: round(per_kernel[kk]["ms_per_launch"] or 0.0, 4)
                                for kk in ("dot", "dkdv", "dq")}},
         "roofline": {"kernel": dom, "bound": "tensor",
-                     "achieved": round(achieved, 2) if achieved else None,
-                     "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4) if achieved else None,
-                     "peak_source": "%s %s" % (peak_src, peak_key),
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4),
+                     "peak_source": "%s %s (burst: kernels timed inside a sub-second loop)"
+                                    % (peak_src, peak_key),
                      "traffic": traffic_for(dom),
                      "traffic_unit": "bytes per launch (ncu dram read + write)"},
+        "roofline_kernels": rooflines,
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "how": "pinned host -> device copy of Q, K, V, dO and device -> host copy of O, LSE, "
@@ -431,7 +457,102 @@ def run_ours(args, rank, world, device):
                        "compute (two device buffer sets)"},
         "gpu_launches": sum(c for (_, c) in prof.values()),
         "clocks": clk,
+        "configs": configs,
     }
+    return out
+
+
+# ------------------------------------------- the other parity workloads ---
+
+# Device-timed throughput of the other workloads of the parity contract, on the
+# same line as the headline: (label, workload name, mask override).
+SWEEP = [
+    ("2 training B4 H16 N2048 non-causal", "train"),
+    ("2 training B4 H16 N2048 causal", "train_causal"),
+    ("3a prefill B2 H16 N8192 causal", "prefill_b2_causal"),
+    ("3b prefill B4 H16 N8192 causal", "prefill_b4_causal"),
+    ("4 packed 16 seqs H32 causal", "varlen_causal"),
+    ("4 packed 16 seqs H32 causal window 1024", "varlen_window"),
+    ("5 backward B2 H16 N4096 causal", "bwd_causal"),
+]
+
+
+def allowed_pairs(n, causal, window):
+    """(query, key) pairs the mask keeps in one sequence of n tokens.  Causal
+    without a window uses n^2 / 2, the convention of the fixed-length count;
+    a window counts the pairs exactly, sum over rows r of min(r + 1, W)."""
+    n = int(n)
+    if not causal:
+        return float(n) * n
+    if window <= 0:
+        return 0.5 * n * n
+    w = int(window)
+    if n <= w:
+        return n * (n + 1) / 2.0
+    return w * (w + 1) / 2.0 + float(n - w) * w
+
+
+def workload_flops(wl, lens):
+    """Forward FLOPs (4d per allowed pair) and backward FLOPs (2.5x)."""
+    pairs = sum(allowed_pairs(n, wl.causal, wl.window) for n in lens)
+    f = 4.0 * wl.H * wl.d * pairs
+    return f, 2.5 * f
+
+
+def sweep_configs(device, reps=10, warmup=3):
+    """fwd and bwd TFLOP/s of each SWEEP workload: per-kernel CUDA events
+    (fa_profile) around every launch, mean over `reps` calls after `warmup`."""
+    import io_aware_exact_21_b200 as fa
+    from io_aware_exact_21_b200.inputs import WORKLOADS, fixed_inputs, varlen_inputs
+    peaks, _ = load_peaks()
+    burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    stream = torch.cuda.current_stream(device)
+    out = {}
+    for label, name in SWEEP:
+        wl = WORKLOADS[name]
+        if wl.varlen is not None:
+            nseq, lo, hi = wl.varlen
+            host = varlen_inputs(nseq, lo, hi, wl.H, wl.d, wl.seed, with_dout=True)
+            cu_h = host["cu_seqlens"]
+            lens = [int(x) for x in (cu_h[1:] - cu_h[:-1])]
+            cu = cu_h.to(device)
+        else:
+            host = fixed_inputs(wl.B, wl.N, wl.H, wl.d, wl.seed, with_dout=True)
+            lens = [wl.N] * wl.B
+            cu = None
+        q, k, v, do = (host[n].to(device) for n in ("q", "k", "v", "dout"))
+        o, lse = fa.forward(q, k, v, causal=wl.causal, window=wl.window, cu_seqlens=cu,
+                            stream=stream)
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+
+        def step():
+            fa.forward(q, k, v, causal=wl.causal, window=wl.window, cu_seqlens=cu, out=o, lse=lse,
+                       stream=stream)
+            fa.backward(q, k, v, o, lse, do, causal=wl.causal, window=wl.window, cu_seqlens=cu,
+                        grads=grads, stream=stream)
+
+        for _ in range(warmup):
+            step()
+        torch.cuda.synchronize(device)
+        fa.fa_profile_begin()
+        for _ in range(reps):
+            step()
+        torch.cuda.synchronize(device)
+        prof = fa.fa_profile_end()
+        assert fa.fa_get_device_error() == 0
+        ms = {kk: prof[kk][0] / prof[kk][1] for kk in ("fwd", "dot", "dkdv", "dq")}
+        f_fwd, f_bwd = workload_flops(wl, lens)
+        t_bwd = ms["dot"] + ms["dkdv"] + ms["dq"]
+        tf_f = f_fwd / (ms["fwd"] * 1e-3) / 1e12
+        tf_b = f_bwd / (t_bwd * 1e-3) / 1e12
+        out[label] = {"fwd_ms": round(ms["fwd"], 4), "fwd_tflops": round(tf_f, 1),
+                      "fwd_frac_of_measured_burst": round(tf_f / burst, 4),
+                      "bwd_ms": round(t_bwd, 4), "bwd_tflops": round(tf_b, 1),
+                      "bwd_frac_of_measured_burst": round(tf_b / burst, 4),
+                      "kernels_ms": {kk: round(v, 4) for kk, v in ms.items()},
+                      "fwd_flops": f_fwd, "tokens": sum(lens)}
+        del q, k, v, do, o, lse, grads, host
+        torch.cuda.empty_cache()
     return out
 
 
@@ -1026,6 +1147,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the oracle timing (used for profiling runs)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the sweep of the other parity workloads (train workload)")
     ap.add_argument("--shape", default=None,
                     help="B,H,N,d override of the workload (profiling of smaller cases)")
     ap.add_argument("--causal", action="store_true", help="causal mask (profiling)")

@@ -249,9 +249,13 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
  * that loads the library until the process exits).  The pages have no
  * counterpart of this entry point; it only changes where the scratch lives.
  *
- * - Problems whose workspace (fa_bwd_workspace_size) exceeds
- *   8 * FA_NOALLOC_MAX_ROWS bytes return FA_ERR_SCRATCH_LIMIT and launch
- *   nothing; use fa_bwd for them.
+ * - The limit is on the workspace, not on H * N alone: a call fits when
+ *   fa_bwd_workspace_size(B, H, N, d, packed ? N : 0) <= 8 * FA_NOALLOC_MAX_ROWS,
+ *   where each sequence counts its length rounded up to a multiple of 128
+ *   rows, once per head (fixed length: B * H * ceil(N / 128) * 128 entries;
+ *   packed: H * (N + 127 * B) rounded up to 128).  So H = 16, N = 65536
+ *   fits, H = 16, N = 65537 does not.  Larger problems return
+ *   FA_ERR_SCRATCH_LIMIT and launch nothing; use fa_bwd for them.
  * - It calls no cudaMalloc / cudaFree and no allocating library routine.
  * - The first call on a device looks up the array's device address (a
  *   one-time set-up with that device current); make that first call before

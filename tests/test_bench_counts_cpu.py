@@ -41,6 +41,26 @@ def test_cached_kv_flops_count_the_allowed_pairs():
         assert bench.flops_kv(1, 1, nq, nk, 128, False) == 4.0 * nq * nk * 128
 
 
+def _window_pairs(n, w):
+    i = np.arange(n)[:, None]
+    j = np.arange(n)[None, :]
+    return int(((j <= i) & (j > i - w)).sum())
+
+
+def test_packed_workload_flops_from_the_drawn_lengths():
+    # a window counts its pairs exactly; causal alone uses n^2 / 2 per sequence
+    for n in (1, 5, 127, 1024, 1025, 3000):
+        assert bench.allowed_pairs(n, True, 1024) == _window_pairs(n, 1024)
+        assert bench.allowed_pairs(n, True, 0) == 0.5 * n * n
+        assert bench.allowed_pairs(n, False, 0) == n * n
+    wl = WORKLOADS["varlen_window"]
+    lens = [130, 2000, 4096]
+    f, b = bench.workload_flops(wl, lens)
+    assert f == 4.0 * wl.H * wl.d * sum(_window_pairs(n, 1024) for n in lens) and b == 2.5 * f
+    wc = WORKLOADS["varlen_causal"]
+    assert bench.workload_flops(wc, lens)[0] == 4.0 * wc.H * wc.d * sum(n * n / 2 for n in lens)
+
+
 def test_decode_bytes_are_the_used_cache_rows():
     wl = WORKLOADS["decode"]
     lens = [4096, 5000, 8192] + [6000] * (wl.B - 3)

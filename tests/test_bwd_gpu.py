@@ -58,18 +58,20 @@ def test_bwd_varlen_elementwise(lens, causal, window):
     check((dq, dk, dv), ref)
 
 
-def test_bwd_workload_parity_sampled_heads():
-    """B=2, H=16, N=4096, d=128, causal: full gradients of two heads."""
+def test_bwd_workload_parity_all_heads():
+    """B=2, H=16, N=4096, d=128, causal: the gradients of all 32 (sequence,
+    head) slices, element by element.  Under a causal mask the backward kernels
+    deal the heads of the last round block by block (the snake tail), so this
+    covers both kinds of schedule."""
     wl = WORKLOADS["bwd_causal"]
     x = wl.make()
     o, lse, dq, dk, dv = run(x, wl.causal, wl.window)
-    heads = [(0, 0), (1, 15)]
-    ref = orc.bwd(x["q"], x["k"], x["v"], x["dout"], wl.scale, causal=True, heads=heads)
-    for s, h in heads:
-        for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
-            assert_close_bf16(t[s, :, h], ref[name][s, :, h], "%s[%d,:,%d]" % (name, s, h))
+    ref = orc.bwd(x["q"], x["k"], x["v"], x["dout"], wl.scale, causal=True)
     for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
         assert torch.isfinite(t).all(), name
+        for s in range(wl.B):
+            for h in range(wl.H):
+                assert_close_bf16(t[s, :, h], ref[name][s, :, h], "%s[%d,:,%d]" % (name, s, h))
 
 
 def test_bwd_invariants_and_determinism():
@@ -124,7 +126,9 @@ def test_bwd_training_shape_causal_sampled_heads():
     wl = WORKLOADS["train_causal"]
     x = fixed_inputs(wl.B, wl.N, wl.H, wl.d, seed=wl.seed, with_dout=True)
     o, lse, dq, dk, dv = run(x, True, 0)
-    heads = [(0, 3), (3, 12)]
+    # heads 37..63 in (sequence, head) order, e.g. (2, 7), (3, 12) and (3, 15),
+    # are dealt block by block by the snake tail of the last round
+    heads = [(0, 3), (2, 7), (3, 12), (3, 15)]
     ref = orc.bwd(x["q"], x["k"], x["v"], x["dout"], wl.scale, causal=True, heads=heads)
     for s, h in heads:
         for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
@@ -143,7 +147,8 @@ def test_bwd_packed_batch_sampled_sequences(window):
     o, lse, dq, dk, dv = run(x, True, window, cu)
     lens = np.diff(cu.numpy())
     order = np.argsort(lens)
-    heads = [(int(order[0]), 0), (int(order[nseq // 2]), wl.H - 1)]
+    heads = [(int(order[0]), 0), (int(order[nseq // 2]), wl.H - 1), (int(order[-1]), 5),
+             (nseq - 1, wl.H - 1)]
     ref = orc.bwd(x["q"], x["k"], x["v"], x["dout"], wl.scale, causal=True, window=window,
                   cu_seqlens=cu, heads=heads)
     for s, h in heads:

@@ -10,7 +10,8 @@ import pytest
 import torch
 
 import io_aware_exact_21_b200 as fa
-from io_aware_exact_21_b200.inputs import fixed_inputs
+from io_aware_exact_21_b200.inputs import fixed_inputs, varlen_inputs
+from oracle import oracle as orc
 
 from helpers import assert_close_bf16, to64
 
@@ -47,6 +48,38 @@ def test_noalloc_backward_matches_fa_bwd_on_two_calls_in_a_row():
         assert fa.fa_get_device_error() == 0
         for name, got, want in zip(("dq", "dk", "dv"), grads, ref):
             assert_close_bf16(got, to64(want), name)
+
+
+def test_noalloc_packed_batch_after_a_larger_call():
+    """A packed batch (its statistics sit at per-sequence offsets rounded up to
+    128 rows in the scratch) right after a larger fixed-length call that left
+    other values there; checked against fa_bwd and the float64 oracle."""
+    big = dict(B=2, N=1500, H=4, d=128, causal=False, window=0, seed=43)
+    q, k, v, do, o, lse = _problem(big)
+    grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    rc = fa.fa_bwd_noalloc(q, k, v, o, lse, do, *grads, big["B"], big["H"], big["N"], big["d"],
+                           1 / math.sqrt(big["d"]), 0, 0, None, None)
+    assert rc == 0, fa.fa_status_string(rc)
+    lens = [130, 1, 517]
+    H, d, window = 3, 128, 200
+    x = varlen_inputs(len(lens), 0, 0, H, d, seed=44, with_dout=True, lengths=lens)
+    cu = x["cu_seqlens"].to(DEV)
+    q, k, v, do = (x[n].to(DEV) for n in ("q", "k", "v", "dout"))
+    o, lse = fa.forward(q, k, v, causal=True, window=window, cu_seqlens=cu)
+    want = fa.backward(q, k, v, o, lse, do, causal=True, window=window, cu_seqlens=cu)
+    T = sum(lens)
+    ref = orc.bwd(x["q"], x["k"], x["v"], x["dout"], 1 / math.sqrt(d), causal=True,
+                  window=window, cu_seqlens=x["cu_seqlens"])
+    for _ in range(2):
+        got = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+        rc = fa.fa_bwd_noalloc(q, k, v, o, lse, do, *got, len(lens), H, T, d, 1 / math.sqrt(d), 1,
+                               window, cu, None)
+        assert rc == 0, fa.fa_status_string(rc)
+        torch.cuda.synchronize()
+        assert fa.fa_get_device_error() == 0
+        for name, g, w in zip(("dq", "dk", "dv"), got, want):
+            assert_close_bf16(g, to64(w), name + " vs fa_bwd")
+            assert_close_bf16(g, ref[name], name + " vs oracle")
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
