@@ -190,8 +190,8 @@ size_t fa_fwd_kvcache_workspace_size(int B, int H, int Nq, int d, int num_splits
  *
  * fa_quantize_fp8: x bf16 [B, N, H, 128] -> e4m3 codes and one float scale per
  *   block of 128 rows of a head, scales [B, H, ceil(N/128)]: s = amax / 448
- *   (1 for an all-zero block), code = e4m3(x / s), round to nearest even,
- *   saturating.  signs (128 floats of +-1, or NULL) selects the
+ *   (1 for an all-zero block), code = e4m3(x / s): the real quotient rounded
+ *   once to the nearest e4m3 value, ties to even, saturating.  signs (128 floats of +-1, or NULL) selects the
  *   error-reducing rotation of each row before quantising: multiply by the
  *   signs, then the orthonormal Walsh-Hadamard transform (q.k is unchanged;
  *   use the same signs for Q and K).  transpose = 0 writes codes as
@@ -199,9 +199,14 @@ size_t fa_fwd_kvcache_workspace_size(int B, int H, int Nq, int d, int num_splits
  *   Np = N rounded up to 16, zeros past N (use for V; signs must be NULL,
  *   else FA_ERR_BAD_SHAPE).  fa_fp8_vt_bytes gives that buffer's size.
  * fa_fwd_fp8: O (bf16 [B, N, H, 128]) and LSE ([B, H, N]) from the codes and
- *   scales: scores use the block scales of Q and K, P is rounded to e4m3
- *   (after folding in the V block scale relative to the head's largest) for
- *   the PV GEMM, the row sums use the unrounded P.  Masks as fa_fwd.
+ *   scales: the softmax of the quantised scores (codes times block scales),
+ *   with the probabilities rounded to e4m3 before they multiply the quantised
+ *   V and the row sums taken from the unrounded ones.  Which reference the
+ *   probabilities are rounded against is the kernel's: a running maximum
+ *   raised only when it grows by more than 2^3 (base 2), with the V block
+ *   scale folded in relative to the head's largest; the result lies within
+ *   one e4m3 step of P per key of rounding against the row's final maximum.
+ *   Masks as fa_fwd.
  * Errors as fa_fwd; d != 128 is FA_ERR_UNSUPPORTED_D.
  */
 size_t fa_fp8_vt_bytes(int B, int H, int N, int d);

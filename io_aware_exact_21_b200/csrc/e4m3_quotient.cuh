@@ -1,0 +1,57 @@
+// e4m3_quotient.cuh -- the float32 value whose e4m3 conversion (round to
+// nearest, ties to even) is the real quotient x / s rounded once to e4m3.
+//
+// The float32 quotient q = RN(x / s) rounds to the same e4m3 value as x / s
+// unless q itself lies exactly halfway between two e4m3 values while x / s
+// does not (double rounding).  Only then the residual r = x - q s, which one
+// fused multiply-add computes exactly for a correctly rounded quotient (the
+// exact-remainder property of IEEE division), says on which side of that
+// midpoint x / s lies, and q moves one float32 step towards it.  e4m3
+// midpoints: in the normal range (|q| >= 2^-6) four significant bits with the
+// fourth one set; below it the odd multiples of 2^-10.  Requires s > 0.
+//
+// Self-contained (no CUDA headers) so that the host test can build it.
+#pragma once
+
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+namespace fa {
+
+__host__ __device__ __forceinline__ float e4m3_quotient(float x, float s) {
+#ifdef __CUDA_ARCH__
+    float q = __fdiv_rn(x, s);
+#else
+    float q = x / s;
+#endif
+    const float a = fabsf(q);
+    bool mid;
+    if (a >= 0.015625f) {
+        uint32_t bits;
+        memcpy(&bits, &a, 4);
+        mid = (bits & 0x7FFFFu) == 0u && (bits & 0x80000u) != 0u;
+    } else {
+        const float t = a * 1024.f;          // exact: a power-of-two scaling, t < 16
+        mid = t == floorf(t) && (static_cast<int>(t) & 1) == 1;
+    }
+    if (mid) {
+#ifdef __CUDA_ARCH__
+        const float r = __fmaf_rn(-q, s, x);
+#else
+        const float r = fmaf(-q, s, x);
+#endif
+        if (r != 0.f) {
+            // one float32 step towards x / s: up when r > 0 (s > 0)
+            uint32_t qb;
+            memcpy(&qb, &q, 4);
+            const bool up = r > 0.f;
+            const bool neg = (qb >> 31) != 0u;
+            qb = (up != neg) ? qb + 1u : qb - 1u;   // the magnitude grows iff moving away from 0
+            memcpy(&q, &qb, 4);
+        }
+    }
+    return q;
+}
+
+}  // namespace fa

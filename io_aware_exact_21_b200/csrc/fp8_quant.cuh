@@ -13,13 +13,14 @@
 //    operation, so the codes do not depend on how a compiler would contract
 //    them.  q.k is unchanged by the rotation.
 //  * scale s = amax / 448 over the block (1 for an all-zero block); codes are
-//    e4m3(x * inv), inv = 1 / s rounded to float32 once per block, round to
-//    nearest even, saturating.
+//    e4m3(x / s), the real quotient rounded once to the nearest e4m3 value
+//    (ties to even, saturating at +-448): see e4m3_quotient below.
 //  * layout: Q and K codes keep the token-major [B, N, H, 128] layout; V codes
 //    are written transposed, [B, H, 128, Np] with Np = N rounded up to 16 and
 //    zeros past N, so the forward's PV GEMM reads a K-major operand.
 #pragma once
 
+#include "e4m3_quotient.cuh"
 #include "sm100.cuh"
 
 namespace fa {
@@ -125,15 +126,14 @@ quantize_fp8_kernel(const QuantParams p) {
 #pragma unroll
     for (int w = 1; w < kQuantWarps; ++w) amax = fmaxf(amax, s_amax[w]);
     const float sc = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
-    const float inv = __fdiv_rn(1.f, sc);
     if (threadIdx.x == 0) p.scales[static_cast<size_t>(bh) * p.nb + blk] = sc;
 
 #pragma unroll
     for (int k = 0; k < kQuantRows; ++k) {
         const int rr = warp + kQuantWarps * k;
         const int r = r0 + rr;
-        const uint32_t code = pack_e4m3x4(__fmul_rn(y[k][0], inv), __fmul_rn(y[k][1], inv),
-                                          __fmul_rn(y[k][2], inv), __fmul_rn(y[k][3], inv));
+        const uint32_t code = pack_e4m3x4(e4m3_quotient(y[k][0], sc), e4m3_quotient(y[k][1], sc),
+                                          e4m3_quotient(y[k][2], sc), e4m3_quotient(y[k][3], sc));
         if (!p.transpose) {
             if (r < p.N)
                 *reinterpret_cast<uint32_t*>(

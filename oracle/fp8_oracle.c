@@ -10,8 +10,8 @@
  * FlashAttention-3 paragraph) says that the FP8 path adds block quantisation
  * and a processing step that reduces quantisation error, and that such
  * low-precision execution is to be kept apart from exact dense attention at
- * higher precision.  It prints no formulas.  This file writes out, step by
- * step, the reading the CUDA path implements:
+ * higher precision.  It prints no formulas.  This file writes out the plain
+ * reading of block-quantised attention, step by step:
  *
  *  1. Error-reducing rotation (optional) of every q and k row, d = 128:
  *     multiply element-wise by a random sign vector, then apply the
@@ -19,29 +19,27 @@
  *     (a + b, a - b) on element pairs (j, j + h) for h = 1, 2, 4, ..., 64 in
  *     that order, then a factor 1/sqrt(128).  The rotation is orthogonal, so
  *     every q.k is unchanged while outliers are spread over all channels.
+ *     Its values are the inputs of integer decisions (the codes), so they are
+ *     taken in float32, one IEEE-754 operation at a time (no fused
+ *     multiply-add).
  *  2. Block scales: for every block of 128 rows of one head (rows past the
- *     sequence end excluded), s = amax / 448 (448 is the largest finite
- *     e4m3 value; s = 1 for an all-zero block), and codes c = e4m3(x * inv)
- *     with inv = 1 / s rounded to float32 once per block (one multiply per
- *     element instead of a division; the two readings of "x over s" differ
- *     only where x / s and x * inv fall on opposite sides of an e4m3
- *     rounding boundary).
- *     Steps 1-2 decide integer codes, so they are taken in float32, the
- *     precision the CUDA kernel takes them in; every float operation here is
- *     a single IEEE-754 float32 operation (no fused multiply-add).
- *  3. Forward, in float64 from the codes: for each query row the 128-key
- *     blocks are visited in order with the online normalisation of the
- *     encyclopedia page, section "tiled computation and online
- *     normalisation", in base 2 and with the reference maximum raised only
- *     when a block's maximum exceeds it by more than 8 (the exponentials
- *     then stay <= 2^8, inside e4m3's range):
- *        x_j = (c_q . c_k_j) * scale * log2(e) * s_q * s_k(block of j)
- *        p_j = 2^(x_j - m),  l += p_j
- *        P_j = e4m3(p_j * r_b),  r_b = min(1, s_v(b) / max_b' s_v(b'))
- *        acc += P_j * c_v_j
- *     and O = acc * max_b s_v(b) / l, LSE = ln 2 * (m + log2 l).  The V
- *     block scales are folded into P relative to the head's largest one so
- *     that a single fp32 accumulator serves all blocks.
+ *     sequence end excluded), s = amax / 448 in float32 (448 is the largest
+ *     finite e4m3 value; s = 1 for an all-zero block), and codes
+ *     c = e4m3(x / s): the real quotient rounded once to the nearest e4m3
+ *     value, ties to even, saturating at +-448.  (The quotient of two float32
+ *     numbers is taken in float64; no float64 quotient lies on an e4m3
+ *     rounding boundary unless the real one does, so this is the exactly
+ *     rounded code.)
+ *  3. Forward from the codes, in float64: the codes times their block scales
+ *     are the quantised operands q^, k^, v^; per query row the scores
+ *     x_j = scale q^.k^_j over the allowed keys, the row maximum m, the
+ *     exponentials p_j = exp(x_j - m) and their sum l (the softmax statistics
+ *     are not matmul operands and keep full precision), and the output
+ *        O = sum_j e4m3(p_j) v^_j / l,     LSE = m + ln l,
+ *     i.e. the probabilities are quantised to e4m3 against the row maximum
+ *     (p <= 1) before they multiply V.  This is the exact softmax of the
+ *     quantised scores, with no tiling: how a kernel walks the keys is not
+ *     part of what the method computes.
  *
  * Return value 0 = ok, -3 = bad shape, -5 = window without causal.
  */
@@ -125,12 +123,12 @@ int oracle_quantize_fp8(const float *x, int B, int N, int H, int d, const float 
                     }
                 }
                 const float s = amax > 0.0f ? amax / 448.0f : 1.0f;
-                const float inv = 1.0f / s;
                 scales[((size_t)b * H + h) * nb + blk] = s;
                 for (int r = r0; r < r1; ++r) {
                     const float *yr = y + (size_t)(r - r0) * d;
                     float *cr = codes + (((size_t)b * N + r) * H + h) * d;
-                    for (int c = 0; c < d; ++c) cr[c] = oracle_e4m3_round(yr[c] * inv);
+                    for (int c = 0; c < d; ++c)
+                        cr[c] = (float)e4m3_round_d((double)yr[c] / (double)s);
                 }
             }
     free(y);
@@ -145,65 +143,93 @@ static int allowed(int i, int j, int causal, int window)
 }
 
 /* Step 3.  qc, kc, vc: [B * N, H, d] code values; sq, sk, sv: [B, H, nb].
- * quantize_p = 0 skips the e4m3 rounding of P (with unit scales and exact
- * values this is then the exact forward).  o: [B * N, H, d]; lse: [B, H, N]. */
+ * quantize_p = 0 skips the e4m3 rounding of p (with unit scales and exact
+ * values this is then the exact forward).  o: [B * N, H, d]; lse: [B, H, N].
+ *
+ * Optional outputs (NULL to skip), [B * N, H, d] like o, the sums an error
+ * bound on the rounding of p needs, per output element (row i, channel c):
+ *   wa  = sum_j p_j |v^_jc| / l        wa2 = sum_j (p_j v^_jc)^2 / l^2
+ *   wz  = sum_j |cv_jc| / l            wz2 = sum_j cv_jc^2 / l^2
+ * (cv: the V codes, p_j = exp(x_j - m) as above, j over the allowed keys). */
 int oracle_fwd_fp8(const float *qc, const float *kc, const float *vc, const float *sq,
                    const float *sk, const float *sv, int B, int N, int H, int d, double scale,
-                   int causal, int window, int quantize_p, double *o, double *lse)
+                   int causal, int window, int quantize_p, double *o, double *lse,
+                   double *wa, double *wa2, double *wz, double *wz2)
 {
     if (B < 0 || N < 0 || H <= 0 || d <= 0) return -3;
     if (window > 0 && !causal) return -5;
     const int nb = (N + BLK - 1) / BLK;
-    const double log2e = 1.4426950408889634;
-    #pragma omp parallel for collapse(3) schedule(dynamic, 16)
-    for (int b = 0; b < B; ++b)
-        for (int h = 0; h < H; ++h)
-            for (int i = 0; i < N; ++i) {
-                const float *sv_bh = sv + ((size_t)b * H + h) * nb;
-                double svmax = 0.0;
-                for (int j = 0; j < nb; ++j)
-                    if (sv_bh[j] > svmax) svmax = sv_bh[j];
-                const float *qr = qc + (((size_t)b * N + i) * H + h) * d;
-                const double sqi = sq[((size_t)b * H + h) * nb + i / BLK];
-                double *acc = o + (((size_t)b * N + i) * H + h) * d;
-                for (int c = 0; c < d; ++c) acc[c] = 0.0;
-                double m = -INFINITY, l = 0.0;
-                double xs[BLK];
-                for (int kb = 0; kb < nb; ++kb) {
-                    const double skb = sk[((size_t)b * H + h) * nb + kb];
-                    const int j0 = kb * BLK, j1 = (j0 + BLK < N) ? j0 + BLK : N;
-                    double mx = -INFINITY;
-                    for (int j = j0; j < j1; ++j) {
-                        xs[j - j0] = -INFINITY;
+    int bad = 0;
+    #pragma omp parallel
+    {
+        double *x = (double *)malloc(sizeof(double) * (N > 0 ? N : 1));
+        double *qh = (double *)malloc(sizeof(double) * d);
+        if (!x || !qh) {
+            #pragma omp atomic write
+            bad = 1;
+        }
+        #pragma omp for collapse(3) schedule(dynamic, 16)
+        for (int b = 0; b < B; ++b)
+            for (int h = 0; h < H; ++h)
+                for (int i = 0; i < N; ++i) {
+                    if (!x || !qh) continue;
+                    const size_t sb = ((size_t)b * H + h) * nb;
+                    const size_t oi = (((size_t)b * N + i) * H + h) * d;
+                    const float *qr = qc + oi;
+                    for (int c = 0; c < d; ++c) qh[c] = (double)qr[c] * sq[sb + i / BLK];
+                    /* scores of the quantised operands and their maximum */
+                    double m = -INFINITY;
+                    for (int j = 0; j < N; ++j) {
+                        x[j] = -INFINITY;
                         if (!allowed(i, j, causal, window)) continue;
                         const float *kr = kc + (((size_t)b * N + j) * H + h) * d;
-                        double s = 0.0;
-                        for (int c = 0; c < d; ++c) s += (double)qr[c] * (double)kr[c];
-                        xs[j - j0] = s * scale * log2e * sqi * skb;
-                        if (xs[j - j0] > mx) mx = xs[j - j0];
+                        const double skj = sk[sb + j / BLK];
+                        double acc = 0.0;
+                        for (int c = 0; c < d; ++c) acc += qh[c] * ((double)kr[c] * skj);
+                        x[j] = scale * acc;
+                        if (x[j] > m) m = x[j];
                     }
-                    if (mx == -INFINITY) continue;          /* nothing allowed in this block */
-                    const double m_new = mx > m ? mx : m;
-                    if (m_new > m + 8.0) {
-                        const double alpha = exp2(m - m_new);   /* 0 on the first block */
-                        l *= alpha;
-                        for (int c = 0; c < d; ++c) acc[c] *= alpha;
-                        m = m_new;
+                    double *orow = o + oi;
+                    for (int c = 0; c < d; ++c) orow[c] = 0.0;
+                    if (wa) for (int c = 0; c < d; ++c) wa[oi + c] = 0.0;
+                    if (wa2) for (int c = 0; c < d; ++c) wa2[oi + c] = 0.0;
+                    if (wz) for (int c = 0; c < d; ++c) wz[oi + c] = 0.0;
+                    if (wz2) for (int c = 0; c < d; ++c) wz2[oi + c] = 0.0;
+                    if (m == -INFINITY) {               /* no allowed key */
+                        lse[sb / nb * N + i] = -INFINITY;
+                        continue;
                     }
-                    double r = svmax > 0.0 ? sv_bh[kb] / svmax : 1.0;
-                    if (r > 1.0) r = 1.0;
-                    for (int j = j0; j < j1; ++j) {
-                        if (xs[j - j0] == -INFINITY) continue;
-                        const double p = exp2(xs[j - j0] - m);
-                        l += p;
-                        const double pq = quantize_p ? e4m3_round_d(p * r) : p * r;
+                    /* exponentials and their sum */
+                    double l = 0.0;
+                    for (int j = 0; j < N; ++j)
+                        if (x[j] != -INFINITY) l += exp(x[j] - m);
+                    /* output: quantised p times the quantised V rows */
+                    for (int j = 0; j < N; ++j) {
+                        if (x[j] == -INFINITY) continue;
+                        const double p = exp(x[j] - m);
+                        const double pq = quantize_p ? e4m3_round_d(p) : p;
                         const float *vr = vc + (((size_t)b * N + j) * H + h) * d;
-                        for (int c = 0; c < d; ++c) acc[c] += pq * (double)vr[c];
+                        const double svj = sv[sb + j / BLK];
+                        for (int c = 0; c < d; ++c) {
+                            const double vh = (double)vr[c] * svj;
+                            orow[c] += pq * vh;
+                            if (wa) wa[oi + c] += p * fabs(vh);
+                            if (wa2) wa2[oi + c] += (p * vh) * (p * vh);
+                            if (wz) wz[oi + c] += fabs((double)vr[c]);
+                            if (wz2) wz2[oi + c] += (double)vr[c] * (double)vr[c];
+                        }
                     }
+                    for (int c = 0; c < d; ++c) {
+                        orow[c] /= l;
+                        if (wa) wa[oi + c] /= l;
+                        if (wa2) wa2[oi + c] /= l * l;
+                        if (wz) wz[oi + c] /= l;
+                        if (wz2) wz2[oi + c] /= l * l;
+                    }
+                    lse[sb / nb * N + i] = m + log(l);
                 }
-                const double f = l > 0.0 ? svmax / l : 0.0;
-                for (int c = 0; c < d; ++c) acc[c] *= f;
-                lse[((size_t)b * H + h) * N + i] = l > 0.0 ? log(2.0) * (m + log2(l)) : -INFINITY;
-            }
-    return 0;
+        free(x);
+        free(qh);
+    }
+    return bad ? -3 : 0;
 }

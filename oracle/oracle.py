@@ -81,7 +81,7 @@ def _load():
         lib.oracle_quantize_fp8.restype = ctypes.c_int
         lib.oracle_fwd_fp8.argtypes = [fp, fp, fp, fp, fp, fp, ctypes.c_int, ctypes.c_int,
                                        ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int,
-                                       ctypes.c_int, ctypes.c_int, dp, dp]
+                                       ctypes.c_int, ctypes.c_int, dp, dp, dp, dp, dp, dp]
         lib.oracle_fwd_fp8.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -315,14 +315,22 @@ def quantize_fp8(x, signs=None):
     return codes, scales
 
 
-def fwd_fp8(qc, kc, vc, sq, sk, sv, scale, causal=False, window=0, quantize_p=True):
-    """FP8 forward from codes and block scales (fixed length [B, N, H, d]).
-    Returns O [B, N, H, d] and LSE [B, H, N] in float64."""
+def fwd_fp8(qc, kc, vc, sq, sk, sv, scale, causal=False, window=0, quantize_p=True,
+            terms=False):
+    """FP8 forward from codes and block scales (fixed length [B, N, H, d]):
+    the exact softmax of the dequantised scores, with the probabilities
+    rounded to e4m3 against the row maximum before they multiply the
+    dequantised V.  Returns O [B, N, H, d] and LSE [B, H, N] in float64; with
+    ``terms`` also a dict of the per-element sums an error bound needs
+    (``wa``, ``wa2``, ``wz``, ``wz2``; see fp8_oracle.c)."""
     q, k, v = _f32(qc), _f32(kc), _f32(vc)
     B, N, H, d = q.shape
     o = np.zeros(q.shape, dtype=np.float64)
     lse = np.zeros((B, H, N), dtype=np.float64)
+    t = {n: np.zeros(q.shape, dtype=np.float64) for n in ("wa", "wa2", "wz", "wz2")} if terms \
+        else None
+    tp = [_dp(t[n]) if terms else None for n in ("wa", "wa2", "wz", "wz2")]
     _check(_load().oracle_fwd_fp8(_fp(q), _fp(k), _fp(v), _fp(_f32(sq)), _fp(_f32(sk)),
                                   _fp(_f32(sv)), B, N, H, d, float(scale), int(bool(causal)),
-                                  int(window), int(bool(quantize_p)), _dp(o), _dp(lse)))
-    return o, lse
+                                  int(window), int(bool(quantize_p)), _dp(o), _dp(lse), *tp))
+    return (o, lse, t) if terms else (o, lse)
