@@ -309,6 +309,7 @@ def run_ours(args, rank, world, device):
     barrier()
     elapsed = e0.elapsed_time(e1)
     prof = fa.fa_profile_end()
+    fwd_balance, fwd_ctas = fa.fa_profile_cta_balance()
     clk = clocks.stop()
     assert fa.fa_get_device_error() == 0
 
@@ -376,10 +377,13 @@ def run_ours(args, rank, world, device):
 
     elapsed, e2e_elapsed = max_over_ranks([elapsed, e2e_elapsed], world, device)
     configs = None
+    fused = None
     if not args.no_configs:
         del sets, pin
         torch.cuda.empty_cache()
         configs = sweep_configs(device)
+        if d == 128:
+            fused = time_fused_backward(q, k, v, o, lse, do, causal, window, scale, device)
     if rank != 0:
         return None
 
@@ -433,6 +437,7 @@ def run_ours(args, rank, world, device):
         "data": "synthetic: i.i.d. N(0,1) bf16 Q, K, V, dO (seeded), no dataset",
         "config": workload_config({"parallelism": "replicas" if world > 1 else "single GPU"}),
         "fwd": {"ms": round(t_fwd, 4), "tflops": round(f_fwd / (t_fwd * 1e-3) / 1e12, 2),
+                "cta_balance": round(fwd_balance, 4),
                 "frac_of_measured_burst_peak": round(f_fwd / (t_fwd * 1e-3) / 1e12 / burst, 4),
                 "frac_of_nominal_dense_peak": round(f_fwd / (t_fwd * 1e-3) / 1e12
                                                     / NOMINAL_BF16_DENSE_TFLOPS, 4)},
@@ -458,7 +463,11 @@ def run_ours(args, rank, world, device):
         "gpu_launches": sum(c for (_, c) in prof.values()),
         "clocks": clk,
         "configs": configs,
+        "bwd_fused_prototype": fused,
     }
+    if fused:
+        fused["tflops"] = round(f_bwd / (fused["ms"] * 1e-3) / 1e12, 2)
+        fused["vs_two_kernel_backward"] = round(t_bwd / fused["ms"], 4)
     return out
 
 
@@ -497,6 +506,35 @@ def workload_flops(wl, lens):
     pairs = sum(allowed_pairs(n, wl.causal, wl.window) for n in lens)
     f = 4.0 * wl.H * wl.d * pairs
     return f, 2.5 * f
+
+
+def time_fused_backward(q, k, v, o, lse, do, causal, window, scale, device, reps=10, warmup=3):
+    """The single-kernel backward (fa_bwd_fused) on the same inputs: pre-pass,
+    fused kernel and dQ conversion, per-kernel CUDA events, mean over reps."""
+    import io_aware_exact_21_b200 as fa
+    stream = torch.cuda.current_stream(device)
+    B, N, H, d = q.shape
+    ws = torch.empty(fa.fa_bwd_fused_workspace_size(B, H, N, d, 0), dtype=torch.uint8, device=device)
+    grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+
+    def step():
+        fa.backward(q, k, v, o, lse, do, causal=causal, window=window, scale=scale, grads=grads,
+                    workspace=ws, stream=stream, fused=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(device)
+    fa.fa_profile_begin()
+    for _ in range(reps):
+        step()
+    torch.cuda.synchronize(device)
+    prof = fa.fa_profile_end()
+    assert fa.fa_get_device_error() == 0
+    ms = {kk: prof[kk][0] / prof[kk][1] for kk in ("dot", "bwd_fused", "dq_convert")}
+    return {"ms": round(sum(ms.values()), 4), "kernels_ms": {kk: round(v, 4) for kk, v in ms.items()},
+            "how": "fa_bwd_fused: pre-pass (statistics, zeroed fp32 dQ accumulator), one kernel for "
+                   "dK, dV and the dQ parts (five GEMMs per tile pair, dQ parts added by bulk fp32 "
+                   "reductions), dQ conversion; same inputs as the timed step"}
 
 
 def sweep_configs(device, reps=10, warmup=3):
@@ -539,6 +577,7 @@ def sweep_configs(device, reps=10, warmup=3):
             step()
         torch.cuda.synchronize(device)
         prof = fa.fa_profile_end()
+        balance, ctas = fa.fa_profile_cta_balance()
         assert fa.fa_get_device_error() == 0
         ms = {kk: prof[kk][0] / prof[kk][1] for kk in ("fwd", "dot", "dkdv", "dq")}
         f_fwd, f_bwd = workload_flops(wl, lens)
@@ -550,6 +589,7 @@ def sweep_configs(device, reps=10, warmup=3):
                       "bwd_ms": round(t_bwd, 4), "bwd_tflops": round(tf_b, 1),
                       "bwd_frac_of_measured_burst": round(tf_b / burst, 4),
                       "kernels_ms": {kk: round(v, 4) for kk, v in ms.items()},
+                      "fwd_cta_balance": round(balance, 4), "fwd_ctas": ctas,
                       "fwd_flops": f_fwd, "tokens": sum(lens)}
         del q, k, v, do, o, lse, grads, host
         torch.cuda.empty_cache()

@@ -244,6 +244,32 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
            const int* cu_seqlens, void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Single-kernel backward (d = 128 only): the same gradients as fa_bwd, with
+ * dK, dV and the dQ contributions computed in one kernel that recomputes each
+ * score and gradient tile once (five GEMMs per key tile x query tile pair
+ * instead of fa_bwd's seven).  The pages say only that the backward pass
+ * recomputes attention blocks from compact normalisation statistics
+ * (FlashAttention encyclopedia page, "training and complexity"); this entry
+ * point is the variant that trades fa_bwd's second recomputation for an fp32
+ * reduction of every tile's dQ part into an accumulator in the workspace
+ * (through the L2's reduction units), then a scaling kernel writes bf16 dQ.
+ * Results equal fa_bwd's up to the order of the fp32 additions into dQ, which
+ * is not fixed (the reductions of different key tiles land in any order), so
+ * dQ is not bit-reproducible from run to run; dK and dV are.
+ *
+ * Arguments as fa_bwd; `workspace` must hold fa_bwd_fused_workspace_size(...)
+ * bytes (the statistics array plus rows x H x 128 floats) and be 256-byte
+ * aligned; its contents on entry do not matter.  d != 128 returns
+ * FA_ERR_UNSUPPORTED_D; fa_bwd_fused_workspace_size returns 0 for it.
+ */
+size_t fa_bwd_fused_workspace_size(int B, int H, int N, int d, int varlen_total);
+int fa_bwd_fused(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dO, void* dq, void* dk, void* dv,
+                 int B, int H, int N, int d, float scale, int causal, int window,
+                 const int* cu_seqlens, void* workspace, size_t workspace_bytes,
+                 cudaStream_t stream);
+
+/*
  * fa_bwd_noalloc: the backward pass for callers that cannot allocate device
  * memory -- for example a plugin inside a framework or runtime that owns every
  * device allocation and has no way to hand this library a workspace, or a
@@ -294,15 +320,28 @@ int fa_get_device_error(cudaStream_t stream);
  * (up to 1024 launches per kernel kind; later ones are not recorded).
  * fa_profile_end() waits for the recorded events, stops recording, and writes
  * for each kind k (0 forward, 1 D pre-pass, 2 dK/dV, 3 dQ, 4 decode, 5 decode
- * split merge, 6 FP8 quantisation, 7 FP8 forward) the summed device
+ * split merge, 6 FP8 quantisation, 7 FP8 forward, 8 single-kernel backward,
+ * 9 its dQ conversion) the summed device
  * milliseconds ms[k] and the number of recorded launches counts[k] (arrays of
  * FA_PROFILE_KINDS entries).
  * Either output pointer may be NULL.  The events are created once per device
  * on the first fa_profile_begin() call.
  */
-#define FA_PROFILE_KINDS 8
+#define FA_PROFILE_KINDS 10
 int fa_profile_begin(void);
 int fa_profile_end(double* ms, int* counts);
+
+/*
+ * While profiling is on, each forward launch (fa_fwd, fa_fwd_kv and the
+ * prefill path of fa_fwd_kvcache) also records the start and end time of
+ * every CTA of its persistent grid.  fa_profile_cta_balance() synchronises
+ * the device and reports, for the last such launch, the mean CTA busy time
+ * over the largest one (1 = every SM busy until the last one finishes) and
+ * the grid size.  The first fa_profile_begin() on a device allocates the
+ * small timing buffer this needs (profiling only; no other entry point
+ * allocates).
+ */
+int fa_profile_cta_balance(double* balance, int* ctas);
 
 /*
  * Test hook for the failure path.  mode 0: normal operation.  mode 1: the

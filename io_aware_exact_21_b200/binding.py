@@ -38,15 +38,19 @@ SIGNATURES = {
                     _VP, _VP, _SZ, _VP]),
     "fa_bwd_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I,
                             _I, _VP, _VP]),
+    "fa_bwd_fused_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "fa_bwd_fused": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _I,
+                          _VP, _VP, _SZ, _VP]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_get_device_error": (_I, [_VP]),
     "fa_debug_set_fault": (_I, [_I, ctypes.c_ulonglong]),
     "fa_profile_begin": (_I, []),
     "fa_profile_end": (_I, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]),
+    "fa_profile_cta_balance": (_I, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]),
 }
 
 PROFILE_KINDS = ("fwd", "dot", "dkdv", "dq", "decode", "combine", "quant_fp8",
-                 "fwd_fp8")   # FA_PROFILE_KINDS order
+                 "fwd_fp8", "bwd_fused", "dq_convert")   # FA_PROFILE_KINDS order
 
 
 class FaError(RuntimeError):
@@ -171,6 +175,20 @@ def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, window,
                                  _ptr(workspace), int(workspace_bytes), _stream(stream))
 
 
+def fa_bwd_fused_workspace_size(B, H, N, d, varlen_total=0) -> int:
+    return int(load_library().fa_bwd_fused_workspace_size(int(B), int(H), int(N), int(d),
+                                                          int(varlen_total)))
+
+
+def fa_bwd_fused(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, window, cu_seqlens,
+                 workspace, workspace_bytes, stream=None) -> int:
+    return load_library().fa_bwd_fused(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+                                       _ptr(dq), _ptr(dk), _ptr(dv), int(B), int(H), int(N),
+                                       int(d), float(scale), int(causal), int(window),
+                                       _ptr(cu_seqlens), _ptr(workspace), int(workspace_bytes),
+                                       _stream(stream))
+
+
 def fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, window,
                    cu_seqlens, stream=None) -> int:
     """fa_bwd without a workspace argument: for callers that cannot allocate
@@ -195,6 +213,16 @@ def fa_debug_set_fault(mode: int, timeout_ns: int = 0) -> int:
 
 def fa_profile_begin() -> int:
     return load_library().fa_profile_begin()
+
+
+def fa_profile_cta_balance():
+    """(mean CTA busy time / largest, grid size) of the last forward launch
+    recorded while profiling was on."""
+    b = ctypes.c_double()
+    n = ctypes.c_int()
+    _check(load_library().fa_profile_cta_balance(ctypes.byref(b), ctypes.byref(n)),
+           "fa_profile_cta_balance")
+    return b.value, n.value
 
 
 def fa_profile_end():
@@ -413,8 +441,9 @@ def forward_fp8(qz, B, N, H, d=128, causal=False, window=0, scale=None, out=None
 
 
 def backward(q, k, v, o, lse, dout, causal=False, window=0, cu_seqlens=None, scale=None,
-             grads=None, workspace=None, stream=None):
-    """dQ, dK, dV for the forward's (O, LSE) and the output gradient dO."""
+             grads=None, workspace=None, stream=None, fused=False):
+    """dQ, dK, dV for the forward's (O, LSE) and the output gradient dO.
+    fused=True runs the single-kernel backward (fa_bwd_fused, d = 128)."""
     import torch
     B, H, N, d = _shape(q, cu_seqlens)
     dev = q.device
@@ -430,10 +459,12 @@ def backward(q, k, v, o, lse, dout, causal=False, window=0, cu_seqlens=None, sca
     dq, dk, dv = grads
     for t, name in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
         _expect(t, name, q.shape, torch.bfloat16, dev)
-    ws_bytes = fa_bwd_workspace_size(B, H, N, d, N if cu_seqlens is not None else 0)
+    size_fn = fa_bwd_fused_workspace_size if fused else fa_bwd_workspace_size
+    ws_bytes = size_fn(B, H, N, d, N if cu_seqlens is not None else 0)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
     _expect_bytes(workspace, "workspace", ws_bytes, dev)
-    _check(fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, window,
-                  cu_seqlens, workspace, workspace.numel(), stream), "fa_bwd")
+    fn = fa_bwd_fused if fused else fa_bwd
+    _check(fn(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, window,
+              cu_seqlens, workspace, workspace.numel(), stream), fn.__name__)
     return dq, dk, dv

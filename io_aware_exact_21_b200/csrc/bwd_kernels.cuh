@@ -82,11 +82,13 @@ __device__ __forceinline__ size_t stats_index(const Geometry& g, int64_t stride,
 // lanes reading 16-byte vectors, the dot product reduced with warp shuffles.
 // Packed batches: each CTA first builds the per-sequence block prefix and a
 // copy of cu_seqlens in shared memory to place each token.
+// With dq_acc non-null (the fused backward) it also zeroes that fp32 [rows, d]
+// accumulator, row by row.
 template <int D>
 __global__ void __launch_bounds__(256)
 stats_kernel(const __nv_bfloat16* __restrict__ dO, const __nv_bfloat16* __restrict__ O,
              const float* __restrict__ lse, float2* __restrict__ stats, int64_t stride,
-             Geometry g) {
+             Geometry g, float* __restrict__ dq_acc) {
     constexpr int LPR = D / 8;                 // lanes per row (16-byte vectors)
     constexpr int RPW = 32 / LPR;              // rows per warp per iteration
     extern __shared__ int pre_smem[];
@@ -107,6 +109,11 @@ stats_kernel(const __nv_bfloat16* __restrict__ dO, const __nv_bfloat16* __restri
     for (int64_t base = warp_global * RPW; base < rows; base += nwarps * RPW) {
         const int64_t r = base + sub;
         float acc = 0.f;
+        if (r < rows && dq_acc) {
+            float4* z = reinterpret_cast<float4*>(dq_acc + r * D + part * 8);
+            z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+            z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
         if (r < rows) {
             const uint4 a = *reinterpret_cast<const uint4*>(dO + r * D + part * 8);
             const uint4 b = *reinterpret_cast<const uint4*>(O + r * D + part * 8);
@@ -168,7 +175,8 @@ struct BwdCfg {
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int OFF_SCRATCH = OFF_MISC + 16;
     static constexpr int OFF_PREFIX = OFF_SCRATCH + 2 * THREADS * 4;   // block and unit prefixes
-    static constexpr int SMEM_BYTES = OFF_PREFIX + 2 * (kMaxVarlenSeqs + 1) * 4 + 1024;
+    static constexpr int OFF_RANK = OFF_PREFIX + 2 * (kMaxVarlenSeqs + 1) * 4;   // short[kMaxSortedSeqs]
+    static constexpr int SMEM_BYTES = OFF_RANK + kMaxSortedSeqs * 2 + 1024;
 };
 
 // Query-tile range [ib, ie) (tiles of BS rows) whose rows can see some key of
@@ -332,8 +340,11 @@ __device__ __forceinline__ uint32_t bwd_prologue(uint8_t* smem, const BwdBarrier
     sch.order = schedule_order(p.g, 0);     // key blocks: fewer queries see later keys
     sch.bprefix = prefix;
     sch.uprefix = prefix + kMaxVarlenSeqs + 1;
+    short* rank_seq = reinterpret_cast<short*>(smem + C::OFF_RANK);
+    bool ranked = false;
     sch.total_units = build_schedule_prefix(p.g, C::BM, prefix, prefix + kMaxVarlenSeqs + 1,
-                                            scratch);   // __syncthreads inside
+                                            scratch, rank_seq, &ranked);   // __syncthreads inside
+    sch.rank_seq = ranked ? rank_seq : nullptr;
     schedule_split_tail(sch);
     tc_fence_before();
     __syncthreads();
@@ -641,7 +652,8 @@ struct DqCfg {
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int OFF_SCRATCH = OFF_MISC + 16;
     static constexpr int OFF_PREFIX = OFF_SCRATCH + 2 * THREADS * 4;
-    static constexpr int SMEM_BYTES = OFF_PREFIX + 2 * (kMaxVarlenSeqs + 1) * 4 + 1024;
+    static constexpr int OFF_RANK = OFF_PREFIX + 2 * (kMaxVarlenSeqs + 1) * 4;   // short[kMaxSortedSeqs]
+    static constexpr int SMEM_BYTES = OFF_RANK + kMaxSortedSeqs * 2 + 1024;
 };
 
 struct DqBarriers {
@@ -717,8 +729,11 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
     sch.order = schedule_order(p.g, 1);     // query blocks: later queries see more keys
     sch.bprefix = prefix;
     sch.uprefix = prefix + kMaxVarlenSeqs + 1;
+    short* rank_seq = reinterpret_cast<short*>(smem + C::OFF_RANK);
+    bool ranked = false;
     sch.total_units = build_schedule_prefix(p.g, C::BM, prefix, prefix + kMaxVarlenSeqs + 1,
-                                            scratch);   // __syncthreads inside
+                                            scratch, rank_seq, &ranked);   // __syncthreads inside
+    sch.rank_seq = ranked ? rank_seq : nullptr;
     schedule_split_tail(sch);
     tc_fence_before();
     __syncthreads();
@@ -1018,7 +1033,7 @@ cudaError_t bwd_launch_d(const BwdArgs& a, const BwdMaps& m, cudaStream_t stream
         if (blocks < 1) blocks = 1;
         stats_kernel<D><<<static_cast<int>(blocks), 256, a.g.cu_seqlens ? kStatsSmem : 0, stream>>>(
             static_cast<const __nv_bfloat16*>(a.dO), static_cast<const __nv_bfloat16*>(a.o), a.lse,
-            a.stats, a.stats_stride, a.g);
+            a.stats, a.stats_stride, a.g, nullptr);
         hk.stop(1, slot, stream);
     }
     BwdParams p;

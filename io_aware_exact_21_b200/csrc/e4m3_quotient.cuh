@@ -1,14 +1,23 @@
 // e4m3_quotient.cuh -- the float32 value whose e4m3 conversion (round to
 // nearest, ties to even) is the real quotient x / s rounded once to e4m3.
 //
-// The float32 quotient q = RN(x / s) rounds to the same e4m3 value as x / s
-// unless q itself lies exactly halfway between two e4m3 values while x / s
-// does not (double rounding).  Only then the residual r = x - q s, which one
-// fused multiply-add computes exactly for a correctly rounded quotient (the
-// exact-remainder property of IEEE division), says on which side of that
-// midpoint x / s lies, and q moves one float32 step towards it.  e4m3
-// midpoints: in the normal range (|q| >= 2^-6) four significant bits with the
-// fourth one set; below it the odd multiples of 2^-10.  Requires s > 0.
+// Fast path: the product q1 = x * inv with inv = RN(1 / s) is within two
+// float32 steps of x / s (two roundings of relative size 2^-24 each), so when
+// q1 lies more than 8 steps from every e4m3 rounding boundary, x / s lies on
+// the same side and e4m3(q1) is the answer.  e4m3 midpoints in the normal
+// range (|q| >= 2^-6) have four significant bits with the fourth one set, so
+// the distance in float32 steps is the low 20 mantissa bits' distance from
+// 0x80000.  Values below 2^-6 (the subnormal range, rare for block-scaled
+// data) and values near a midpoint take the exact path.
+//
+// Exact path: the float32 quotient q = RN(x / s) rounds to the same e4m3
+// value as x / s unless q itself lies exactly halfway between two e4m3 values
+// while x / s does not (double rounding).  Only then the residual
+// r = x - q s, which one fused multiply-add computes exactly for a correctly
+// rounded quotient (the exact-remainder property of IEEE division), says on
+// which side of that midpoint x / s lies, and q moves one float32 step
+// towards it.  Below 2^-6 the midpoints are the odd multiples of 2^-10.
+// Requires s > 0.
 //
 // Self-contained (no CUDA headers) so that the host test can build it.
 #pragma once
@@ -19,7 +28,14 @@
 
 namespace fa {
 
-__host__ __device__ __forceinline__ float e4m3_quotient(float x, float s) {
+// Out of line: the kernel reaches it rarely, and one copy keeps the unrolled
+// quantiser loop small.
+#ifdef __CUDA_ARCH__
+__device__ __noinline__
+#else
+inline
+#endif
+float e4m3_quotient_exact(float x, float s) {
 #ifdef __CUDA_ARCH__
     float q = __fdiv_rn(x, s);
 #else
@@ -52,6 +68,21 @@ __host__ __device__ __forceinline__ float e4m3_quotient(float x, float s) {
         }
     }
     return q;
+}
+
+// inv must be RN(1 / s).
+__host__ __device__ __forceinline__ float e4m3_quotient(float x, float s, float inv) {
+#ifdef __CUDA_ARCH__
+    const float q1 = __fmul_rn(x, inv);
+#else
+    const float q1 = x * inv;
+#endif
+    uint32_t bits;
+    memcpy(&bits, &q1, 4);
+    bits &= 0x7FFFFFFFu;
+    const int dist = static_cast<int>(bits & 0xFFFFFu) - 0x80000;
+    const bool safe = bits >= 0x3C800000u /* 2^-6 */ && (dist > 8 || dist < -8);
+    return safe ? q1 : e4m3_quotient_exact(x, s);
 }
 
 }  // namespace fa

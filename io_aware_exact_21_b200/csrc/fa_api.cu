@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "../../include/fa.h"
+#include "bwd_fused.cuh"
 #include "bwd_kernels.cuh"
 #include "decode_kernel.cuh"
 #include "fp8_quant.cuh"
@@ -23,14 +24,18 @@ constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;
 
 // ----------------------------------------------------------- profiling --
 // Event pairs recorded around each launch while profiling is on.
-constexpr int kProfKinds = 8;   // forward, D pre-pass, dK/dV, dQ, decode, merge, FP8 quantise, FP8 forward
+// forward, D pre-pass, dK/dV, dQ, decode, merge, FP8 quantise, FP8 forward,
+// fused backward kernel, fused backward's dQ conversion
+constexpr int kProfKinds = 10;
 constexpr int kProfCap = 1024;
+constexpr int kClockCtas = 4096;   // CTA timing entries of the profiled forward launch
 struct Profiler {
     bool created = false;
     bool on = false;
     int device = -1;
     cudaEvent_t ev[kProfKinds][kProfCap][2];
     int n[kProfKinds] = {};
+    unsigned long long* cta_clock = nullptr;   // device: 1 + 2 * kClockCtas entries
 };
 thread_local Profiler g_prof;
 
@@ -113,7 +118,7 @@ int device_setup(DeviceState** out) {
             allow_smem(fa::fwd_kernel<128, true>, fa::FwdCfg<128, true>::SMEM_BYTES) != cudaSuccess ||
             allow_smem(fa::fwd_kernel<64, false, true>, fa::FwdCfg<64>::SMEM_BYTES) != cudaSuccess ||
             allow_smem(fa::fwd_kernel<128, false, true>, fa::FwdCfg<128>::SMEM_BYTES) != cudaSuccess ||
-            fa::bwd_set_smem_limits() != cudaSuccess)
+            fa::bwd_set_smem_limits() != cudaSuccess || fa::fused_set_smem_limit() != cudaSuccess)
             return FA_ERR_CUDA;
         st.ready = true;
     }
@@ -655,6 +660,64 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
     return fa::bwd_launch(a, m, stream, hooks) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+size_t fa_bwd_fused_workspace_size(int B, int H, int N, int d, int varlen_total) {
+    if (H <= 0 || B <= 0 || d != 128) return 0;
+    const bool packed = varlen_total > 0;
+    if (!packed && N <= 0) return 0;
+    const int64_t rows = packed ? static_cast<int64_t>(varlen_total) : static_cast<int64_t>(B) * N;
+    return fa::fused_workspace_bytes(B, H, fa::bwd_stats_stride(B, N, varlen_total, packed), packed,
+                                     rows);
+}
+
+int fa_bwd_fused(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                 float scale, int causal, int window, const int* cu_seqlens, void* workspace,
+                 size_t workspace_bytes, cudaStream_t stream) {
+    if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return FA_ERR_NULLPTR;
+    Common c;
+    int rc = validate_common(B, H, N, d, scale, causal, window, cu_seqlens, &c);
+    if (rc != FA_OK) return rc;
+    if (d != 128) return FA_ERR_UNSUPPORTED_D;
+    if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(o) || misaligned(lse) ||
+        misaligned(dO) || misaligned(dq) || misaligned(dk) || misaligned(dv))
+        return FA_ERR_MISALIGNED;
+    if (B == 0 || c.rows == 0) return FA_OK;
+    const bool packed = cu_seqlens != nullptr;
+    const int64_t stride = fa::bwd_stats_stride(B, N, c.rows, packed);
+    const size_t need = fa::fused_workspace_bytes(B, H, stride, packed, c.rows);
+    if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FA_ERR_MISALIGNED;
+    DeviceState* st = nullptr;
+    if ((rc = device_setup(&st)) != FA_OK) return rc;
+
+    fa::BwdArgs a;
+    a.g = c.g;
+    a.d = d;
+    a.q = q;
+    a.o = o;
+    a.dO = dO;
+    a.lse = lse;
+    a.dq = dq;
+    a.dk = dk;
+    a.dv = dv;
+    a.stats = static_cast<float2*>(workspace);
+    a.stats_stride = stride;
+    a.scale = scale;
+    a.num_sms = st->num_sms;
+    a.error_word = st->error_word;
+    a.timeout_ns = g_fault_timeout_ns ? g_fault_timeout_ns : kDefaultTimeoutNs;
+    float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                             fa::fused_stats_bytes(B, H, stride, packed));
+    fa::BwdMaps m;
+    if (make_map(&m.q, q, c.rows, H, d, 128) || make_map(&m.k, k, c.rows, H, d, 128) ||
+        make_map(&m.v, v, c.rows, H, d, 128) || make_map(&m.dO, dO, c.rows, H, d, 128))
+        return FA_ERR_CUDA;
+    fa::BwdHooks hooks{
+        [](int kind, cudaStream_t s) { return prof_start(kind == 1 ? 1 : kind == 2 ? 8 : 9, s); },
+        [](int kind, int slot, cudaStream_t s) { prof_stop(kind == 1 ? 1 : kind == 2 ? 8 : 9, slot, s); }};
+    return fa::bwd_fused_launch(a, m, dq_acc, stream, hooks) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
                    const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d,
                    float scale, int causal, int window, const int* cu_seqlens,
@@ -745,6 +808,8 @@ int fa_profile_begin(void) {
                 cudaEventDestroy(P.ev[k][i][0]);
                 cudaEventDestroy(P.ev[k][i][1]);
             }
+        cudaFree(P.cta_clock);
+        P.cta_clock = nullptr;
         P.created = false;
     }
     if (!P.created) {
@@ -753,10 +818,16 @@ int fa_profile_begin(void) {
                 if (cudaEventCreate(&P.ev[k][i][0]) != cudaSuccess ||
                     cudaEventCreate(&P.ev[k][i][1]) != cudaSuccess)
                     return FA_ERR_CUDA;
+        // profiling only: the per-CTA timing buffer of the forward kernel
+        if (cudaMalloc(&P.cta_clock, sizeof(unsigned long long) * (1 + 2 * kClockCtas)) != cudaSuccess ||
+            cudaMemset(P.cta_clock, 0, sizeof(unsigned long long) * (1 + 2 * kClockCtas)) != cudaSuccess)
+            return FA_ERR_CUDA;
         P.created = true;
         P.device = dev;
     }
     for (int k = 0; k < kProfKinds; ++k) P.n[k] = 0;
+    if (cudaMemcpyToSymbol(fa::g_cta_clock, &P.cta_clock, sizeof(P.cta_clock)) != cudaSuccess)
+        return FA_ERR_CUDA;
     P.on = true;
     return FA_OK;
 }
@@ -764,6 +835,9 @@ int fa_profile_begin(void) {
 int fa_profile_end(double* ms, int* counts) {
     Profiler& P = g_prof;
     P.on = false;
+    unsigned long long* none = nullptr;
+    if (P.created && cudaMemcpyToSymbol(fa::g_cta_clock, &none, sizeof(none)) != cudaSuccess)
+        return FA_ERR_CUDA;
     for (int k = 0; k < kProfKinds; ++k) {
         double total = 0.0;
         for (int i = 0; i < P.n[k]; ++i) {
@@ -776,6 +850,25 @@ int fa_profile_end(double* ms, int* counts) {
         if (ms) ms[k] = total;
         if (counts) counts[k] = P.n[k];
     }
+    return FA_OK;
+}
+
+int fa_profile_cta_balance(double* balance, int* ctas) {
+    Profiler& P = g_prof;
+    if (!P.created || !P.cta_clock) return FA_ERR_CUDA;
+    static unsigned long long h[1 + 2 * kClockCtas];
+    if (cudaDeviceSynchronize() != cudaSuccess ||
+        cudaMemcpy(h, P.cta_clock, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return FA_ERR_CUDA;
+    const int G = static_cast<int>(h[0] < static_cast<unsigned long long>(kClockCtas) ? h[0] : kClockCtas);
+    double sum = 0.0, mx = 0.0;
+    for (int c = 0; c < G; ++c) {
+        const double busy = static_cast<double>(h[2 + 2 * c] - h[1 + 2 * c]);
+        sum += busy;
+        if (busy > mx) mx = busy;
+    }
+    if (balance) *balance = (G > 0 && mx > 0.0) ? sum / G / mx : 0.0;
+    if (ctas) *ctas = G;
     return FA_OK;
 }
 

@@ -126,14 +126,16 @@ quantize_fp8_kernel(const QuantParams p) {
 #pragma unroll
     for (int w = 1; w < kQuantWarps; ++w) amax = fmaxf(amax, s_amax[w]);
     const float sc = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+    const float inv = __fdiv_rn(1.f, sc);
     if (threadIdx.x == 0) p.scales[static_cast<size_t>(bh) * p.nb + blk] = sc;
 
 #pragma unroll
     for (int k = 0; k < kQuantRows; ++k) {
         const int rr = warp + kQuantWarps * k;
         const int r = r0 + rr;
-        const uint32_t code = pack_e4m3x4(e4m3_quotient(y[k][0], sc), e4m3_quotient(y[k][1], sc),
-                                          e4m3_quotient(y[k][2], sc), e4m3_quotient(y[k][3], sc));
+        const uint32_t code =
+            pack_e4m3x4(e4m3_quotient(y[k][0], sc, inv), e4m3_quotient(y[k][1], sc, inv),
+                        e4m3_quotient(y[k][2], sc, inv), e4m3_quotient(y[k][3], sc, inv));
         if (!p.transpose) {
             if (r < p.N)
                 *reinterpret_cast<uint32_t*>(

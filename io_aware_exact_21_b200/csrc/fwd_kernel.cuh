@@ -127,7 +127,8 @@ struct FwdCfg {
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int OFF_SCRATCH = OFF_MISC + 16;
     static constexpr int OFF_PREFIX = OFF_SCRATCH + 2 * THREADS * 4;   // block and unit prefixes
-    static constexpr int SMEM_BYTES = OFF_PREFIX + 2 * (kMaxVarlenSeqs + 1) * 4 + 1024;
+    static constexpr int OFF_RANK = OFF_PREFIX + 2 * (kMaxVarlenSeqs + 1) * 4;   // short[kMaxSortedSeqs]
+    static constexpr int SMEM_BYTES = OFF_RANK + kMaxSortedSeqs * 2 + 1024;
 };
 
 template <int D, bool kF8 = false, bool kCache = false>
@@ -157,8 +158,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
 
     const int warp = threadIdx.x >> 5;
     const int lane = lane_id();
+    unsigned long long* t_start = reinterpret_cast<unsigned long long*>(smem + C::OFF_MISC + 8);
 
     if (threadIdx.x == 0) {
+        *t_start = global_timer_ns();         // this CTA's start (profiling: CTA balance)
         mbar_init(q_full, 1);
         mbar_init(q_empty, 1);
         for (int s = 0; s < C::NSLOT; ++s) {
@@ -187,17 +190,24 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     Schedule sch;
     sch.g = p.g;
     sch.rows_per_item = C::ROWS;
-    sch.order = 0;                              // pairs only (ItemIter<false>)
+    // fixed length under a causal or window mask: pairs, then the last
+    // round's blocks one by one, heaviest first (query blocks grow in cost
+    // with their index); pairs alone otherwise
+    sch.order = kCache ? 0 : schedule_order(p.g, 1);
     sch.bprefix = prefix;
     sch.uprefix = prefix + kMaxVarlenSeqs + 1;
+    short* rank_seq = reinterpret_cast<short*>(smem + C::OFF_RANK);
+    bool ranked = false;
     if constexpr (kCache) {
         sch.g.H = p.g.H * p.nsplit;             // (head, split) pairs
         sch.total_units = build_schedule_prefix(sch.g, C::ROWS, prefix,
                                                 prefix + kMaxVarlenSeqs + 1, scratch);
     } else {
         sch.total_units = build_schedule_prefix(p.g, C::ROWS, prefix, prefix + kMaxVarlenSeqs + 1,
-                                                scratch);  // has __syncthreads
+                                                scratch, rank_seq, &ranked);  // has __syncthreads
     }
+    sch.rank_seq = ranked ? rank_seq : nullptr;
+    schedule_split_tail(sch);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -214,7 +224,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             bool ok = true;
             bool skipped = false;
             uint32_t skipped_at = 0xffffffffu;
-            ItemIter<false> it;
+            ItemIter<true> it;
             int s, h, blk;
             for (; ok && it.next(sch, s, h, blk); ++item_it) {
                 [[maybe_unused]] int split = 0;
@@ -326,7 +336,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     }
                 }
             };
-            ItemIter<false> it;
+            ItemIter<true> it;
             int s, h, blk;
             for (; ok && it.next(sch, s, h, blk); ++item_it) {
                 [[maybe_unused]] int split = 0;
@@ -420,7 +430,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         const float sl2 = p.scale_log2;
         uint32_t step = 0, item_it = 0;
         bool ok = true;
-        ItemIter<false> it;
+        ItemIter<true> it;
         int s, h, blk;
         for (; ok && it.next(sch, s, h, blk); ++item_it) {
             [[maybe_unused]] int split = 0;
@@ -491,20 +501,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     for (int c = 0; c < C::BN; ++c)
                         if (!key_allowed(i + off, k0 + c, nk, p.g.causal, p.g.window)) sv[c] = -INFINITY;
                 }
-                // row maximum as a tree (the max is exact in any order), so the
-                // 127 compares are not one dependent chain
-                float mx;
-                {
-                    float m8[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) m8[e] = sv[e];
-#pragma unroll
-                    for (int c = 8; c < C::BN; c += 8)
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) m8[e] = fmaxf(m8[e], sv[c + e]);
-                    mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-                }
+                // row maximum as a tree of three-input maxima (the max is exact
+                // in any order), so the compares are not one dependent chain
+                const float mx = row_max<C::BN>(sv);
                 const float m_new = fmaxf(m_ref, mx * sl2j);
                 const bool resc = m_new > m_ref + kRescaleLog2;
                 float alpha = 1.f;
@@ -535,18 +534,24 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                         }
                         tmem_st16(tS + half * 16, pk);
                     } else {
+                        // pairs of keys: the argument and the row sum in packed
+                        // float32x2 arithmetic (two sums, added at the end)
+                        float2 ls = make_float2(0.f, 0.f);
 #pragma unroll
                         for (int c = half * (C::BN / 64); c < (half + 1) * (C::BN / 64); ++c) {
                             uint32_t pk[16];
 #pragma unroll
                             for (int e = 0; e < 16; ++e) {
-                                const float p0 = ex2(fmaf(sv[c * 32 + 2 * e], sl2, neg_m));
-                                const float p1 = ex2(fmaf(sv[c * 32 + 2 * e + 1], sl2, neg_m));
-                                lsum += p0 + p1;
+                                const float2 a = ffma2(make_float2(sv[c * 32 + 2 * e], sv[c * 32 + 2 * e + 1]),
+                                                       make_float2(sl2, sl2), make_float2(neg_m, neg_m));
+                                const float p0 = ex2(a.x);
+                                const float p1 = ex2(a.y);
+                                ls = fadd2(ls, make_float2(p0, p1));
                                 pk[e] = pack_bf16(p0, p1);
                             }
                             tmem_st16(tS + c * 16, pk);
                         }
+                        lsum += ls.x + ls.y;
                     }
                     if (half == 0 && j > jb && __any_sync(0xffffffffu, resc)) {
                         // O_t *= alpha before the first O_t += P V of this step.  The
@@ -635,6 +640,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
+    }
+    if (threadIdx.x == 0) {
+        unsigned long long* const cta_clock = g_cta_clock;
+        if (cta_clock && blockIdx.x < 4096) {
+            if (blockIdx.x == 0) cta_clock[0] = gridDim.x;
+            cta_clock[1 + 2 * blockIdx.x] = *t_start;
+            cta_clock[2 + 2 * blockIdx.x] = global_timer_ns();
+        }
     }
 }
 

@@ -15,6 +15,7 @@
 namespace fa {
 
 constexpr int kMaxVarlenSeqs = 2048;   // sequences a packed batch may hold
+constexpr int kMaxSortedSeqs = 256;    // packed batches up to this size are dealt longest first
 
 struct Geometry {
     int B;                  // sequences
@@ -84,10 +85,18 @@ __device__ __forceinline__ bool tile_needs_mask(int r0, int BM, int k0, int BN, 
 // Pairs: a work unit is the pair of blocks p and nb-1-p of one (sequence,
 // head) (the middle block alone when nb is odd), so that under a causal mask
 // -- where a block's cost grows or shrinks linearly with its index -- every
-// unit costs the same.  Units are ordered sequence-major, then head, then p,
-// so the CTAs running at the same time share K/V of few heads in L2; unit w
-// goes to CTA w % gridDim.x.  This is the whole schedule for packed batches
-// and for fixed length without a causal or window mask.
+// unit of a sequence costs the same.  Units are ordered sequence-major, then
+// head, then p, so the CTAs running at the same time share K/V of few heads
+// in L2; unit w goes to CTA w % gridDim.x.  This is the whole schedule for
+// fixed length without a causal or window mask.
+//
+// Packed batches, longest first: a unit's cost grows with its sequence's
+// length, so with up to kMaxSortedSeqs sequences the sequences are ranked by
+// length (longest first, ties by index) and the units follow that order;
+// they are dealt in rounds of gridDim.x, forwards in even rounds and
+// backwards in odd ones (a "snake"), so that every CTA's list runs from
+// costly units to cheap ones and the costs even out across CTAs (a greedy
+// longest-first assignment in the usual sense).
 //
 // Pairs + snake tail (the backward kernels, for fixed length with a causal or
 // window mask, where a block's cost is monotone in its index; the forward
@@ -108,7 +117,8 @@ struct Schedule {
     int tail_heads;         //   (sequence, head)s in the tail
     int tail_c0;            //   CTA that takes the tail's first block
     const int* bprefix;     // shared memory: blocks of the sequences before s (packed only)
-    const int* uprefix;     // shared memory: units of the sequences before s (packed only)
+    const int* uprefix;     // shared memory: units of the sequences ranked before r (packed only)
+    const short* rank_seq;  // shared memory: the sequence at each rank, or nullptr (rank = index)
     int total_units;
 
     __device__ __forceinline__ int blocks_of(int len) const {
@@ -153,16 +163,16 @@ struct Schedule {
             s = w / (g.H * nu);
             local = w - s * g.H * nu;
         } else {
-            // binary search: largest s with uprefix[s] * H <= w
+            // binary search: largest rank r with uprefix[r] * H <= w
             int lo = 0, hi = g.B - 1;
             while (lo < hi) {
                 int mid = (lo + hi + 1) >> 1;
                 if (uprefix[mid] * g.H <= w) lo = mid; else hi = mid - 1;
             }
-            s = lo;
-            nu = uprefix[s + 1] - uprefix[s];
+            s = rank_seq ? rank_seq[lo] : lo;
+            nu = uprefix[lo + 1] - uprefix[lo];
             nb = bprefix[s + 1] - bprefix[s];
-            local = w - uprefix[s] * g.H;
+            local = w - uprefix[lo] * g.H;
         }
         h = local / nu;
         p = local - h * nu;
@@ -177,8 +187,9 @@ template <bool kTail>
 struct ItemIter {
     int w;        // pairs: next unit
     int half;
-    int round;    // snake: next round
-    __device__ __forceinline__ ItemIter() : w(blockIdx.x), half(0), round(0) {}
+    int pround;   // pairs: round of the next unit
+    int round;    // snake tail: next round
+    __device__ __forceinline__ ItemIter() : w(blockIdx.x), half(0), pround(0), round(0) {}
     __device__ __forceinline__ bool next(const Schedule& sch, int& s, int& h, int& blk) {
         const int limit = (kTail && sch.order != 0) ? sch.bulk_units : sch.total_units;
         while (w < limit) {
@@ -190,7 +201,12 @@ struct ItemIter {
                 return true;
             }
             half = 0;
-            w += gridDim.x;
+            // the next round's unit: forwards in even rounds, backwards in odd
+            // ones when the units run longest first, else w + gridDim.x
+            ++pround;
+            const int G = gridDim.x;
+            w = pround * G + ((sch.rank_seq && (pround & 1)) ? G - 1 - static_cast<int>(blockIdx.x)
+                                                             : static_cast<int>(blockIdx.x));
             if (nb - 1 - p != p) {
                 blk = nb - 1 - p;
                 return true;
@@ -236,27 +252,51 @@ __device__ __forceinline__ int schedule_order(const Geometry& g, int cost_grows_
     return cost_grows_with_index ? 1 : -1;
 }
 
-// Build the per-sequence block and unit prefixes in shared memory (packed
-// batches only) and return the number of work units.  All threads of the CTA
-// call it.
+// Build the per-sequence block prefix (in sequence order) and the unit prefix
+// (in rank order) in shared memory (packed batches only) and return the number
+// of work units.  With `rank_seq` non-null and at most kMaxSortedSeqs
+// sequences, the ranks are by length, longest first (ties by index), and
+// rank_seq[r] receives the sequence of rank r; the caller then sets the
+// schedule's rank_seq to it, else to nullptr (rank = index).  Returns the rank
+// order's use through *ranked.  All threads of the CTA call it.
 __device__ __forceinline__ int build_schedule_prefix(const Geometry& g, int rows_per_item,
                                                      int* bprefix, int* uprefix,
-                                                     int* scratch /* 2 * blockDim */) {
+                                                     int* scratch /* 2 * blockDim */,
+                                                     short* rank_seq = nullptr,
+                                                     bool* ranked = nullptr) {
+    if (ranked) *ranked = false;
     if (!g.cu_seqlens) {
         const int nb = (g.N + rows_per_item - 1) / rows_per_item;
         return g.B * g.H * ((nb + 1) >> 1);
     }
+    const bool sort = rank_seq != nullptr && g.B <= kMaxSortedSeqs;
     const int tid = threadIdx.x, nt = blockDim.x;
     const int per = (g.B + nt - 1) / nt;
     const int s0 = min(g.B, tid * per), s1 = min(g.B, s0 + per);
-    int runb = 0, runu = 0;
+    // raw per-sequence counts: blocks at the sequence's index, units at its rank
     for (int s = s0; s < s1; ++s) {
         const int len = g.cu_seqlens[s + 1] - g.cu_seqlens[s];
         const int nb = (len + rows_per_item - 1) / rows_per_item;
-        runb += nb;
-        runu += (nb + 1) >> 1;
-        bprefix[s + 1] = runb;          // local inclusive prefixes for now
-        uprefix[s + 1] = runu;
+        bprefix[s + 1] = nb;
+        int r = s;
+        if (sort) {
+            r = 0;
+            for (int o = 0; o < g.B; ++o) {
+                const int lo = g.cu_seqlens[o + 1] - g.cu_seqlens[o];
+                r += (lo > len) || (lo == len && o < s);
+            }
+            rank_seq[r] = static_cast<short>(s);
+        }
+        uprefix[r + 1] = (nb + 1) >> 1;
+    }
+    __syncthreads();
+    // inclusive prefix sums over [1, B]: per-thread chunks, then chunk offsets
+    int runb = 0, runu = 0;
+    for (int x = s0; x < s1; ++x) {
+        runb += bprefix[x + 1];
+        bprefix[x + 1] = runb;
+        runu += uprefix[x + 1];
+        uprefix[x + 1] = runu;
     }
     scratch[tid] = runb;
     scratch[nt + tid] = runu;
@@ -275,11 +315,12 @@ __device__ __forceinline__ int build_schedule_prefix(const Geometry& g, int rows
     }
     __syncthreads();
     const int ob = scratch[tid], ou = scratch[nt + tid];
-    for (int s = s0; s < s1; ++s) {
-        bprefix[s + 1] += ob;
-        uprefix[s + 1] += ou;
+    for (int x = s0; x < s1; ++x) {
+        bprefix[x + 1] += ob;
+        uprefix[x + 1] += ou;
     }
     __syncthreads();
+    if (ranked) *ranked = sort;
     return uprefix[g.B] * g.H;
 }
 

@@ -28,6 +28,11 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
+// Per-CTA busy times of the last profiled forward launch: {start, end} in
+// nanoseconds per CTA, entry 0 preceded by the grid size.  Null unless the
+// host's profiling is on (fa_profile_begin / fa_profile_end).
+__device__ unsigned long long* g_cta_clock;
+
 // First 1024-byte aligned byte of the dynamic shared memory (swizzled TMA
 // tiles need 1024-byte alignment).  Offsetting the __shared__ array itself,
 // rather than rebuilding a pointer from an integer, keeps the shared address
@@ -136,6 +141,30 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint
         ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes),
           "r"(smem_u32(bar))
         : "memory");
+}
+
+// Make this thread's generic-proxy shared-memory writes visible to the async
+// proxy (tensor-core operand reads, bulk copies) that is signalled afterwards.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// global[gdst .. + bytes) += shared[ssrc .. + bytes) as float32, element-wise,
+// performed by the bulk-copy unit (bytes a multiple of 16, both addresses
+// 16-byte aligned).  Tracked by this thread's bulk async-group.
+__device__ __forceinline__ void bulk_reduce_add_f32(float* gdst, const void* ssrc, uint32_t bytes) {
+    asm volatile(
+        "cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;"
+        ::"l"(reinterpret_cast<uint64_t>(gdst)), "r"(smem_u32(ssrc)), "r"(bytes)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until every bulk copy this thread committed has finished reading its
+// shared-memory source (the writes to global memory may still be in flight).
+__device__ __forceinline__ void bulk_wait_group_read0() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
 // --------------------------------------------------------------- tcgen05 --
@@ -329,6 +358,54 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
 // Four floats to four e4m3 bytes, element 0 in the lowest byte.
 __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
     return cvt_e4m3x2(a, b) | (cvt_e4m3x2(c, d) << 16);
+}
+
+// Three-input maximum (one instruction on sm_100); NaN operands are ignored
+// as by fmaxf.
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// Maximum of N (a multiple of 8, >= 24) values as a tree of three-input
+// maxima: eight independent chains, then their combination.
+template <int N>
+__device__ __forceinline__ float row_max(const float (&v)[N]) {
+    static_assert(N % 8 == 0 && N >= 24, "row_max: N must be a multiple of 8, at least 24");
+    float m8[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) m8[e] = max3(v[e], v[8 + e], v[16 + e]);
+    int c = 24;
+#pragma unroll
+    for (; c + 16 <= N; c += 16)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m8[e] = max3(m8[e], v[c + e], v[c + 8 + e]);
+    if (c < N) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m8[e] = fmaxf(m8[e], v[c + e]);
+    }
+    return max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+}
+
+// Packed float32x2 arithmetic (one instruction for two lanes of work on
+// sm_100): d = a * b + c and d = a + b, element-wise, rounded to nearest.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    float2 d;
+    asm("{.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
 }
 
 // Register-count hand-off between warpgroups.

@@ -1,7 +1,8 @@
 // Host build of the quantiser's quotient step (csrc/e4m3_quotient.cuh): for
 // random and for constructed double-rounding cases, the e4m3 rounding of the
-// returned float32 value must equal the real quotient x / s rounded once to
-// e4m3 (nearest, ties to even).  The reference rounds the float64 quotient
+// returned float32 value -- of the fast reciprocal path with its fallback, and
+// of the exact path alone -- must equal the real quotient x / s rounded once
+// to e4m3 (nearest, ties to even).  The reference rounds the float64 quotient
 // (which lies on an e4m3 midpoint only when the real one does) by counting
 // e4m3 steps; the value under test is rounded with integer bit arithmetic on
 // its float32 pattern, as the conversion instruction would.  Prints "ok".
@@ -56,8 +57,11 @@ int main() {
     std::mt19937_64 rng(12345);
     std::uniform_real_distribution<float> amax_d(1e-3f, 50.f), u(-1.f, 1.f);
     long fixups = 0, checked = 0;
+    long exact_path = 0;
     auto check = [&](float x, float s) {
-        const float q = fa::e4m3_quotient(x, s);
+        const float inv = 1.f / s;
+        const float q = fa::e4m3_quotient(x, s, inv);
+        if (q != x * inv) ++exact_path;
         const double want = ref_e4m3(static_cast<double>(x) / static_cast<double>(s));
         const double got = bits_e4m3(q);
         ++checked;
@@ -65,8 +69,12 @@ int main() {
             std::printf("x=%a s=%a got %.9g want %.9g\n", x, s, got, want);
             std::exit(1);
         }
-        float q0 = x / s;
-        if (q0 != q) ++fixups;
+        const float q0 = fa::e4m3_quotient_exact(x, s);
+        if (q0 != x / s) ++fixups;
+        if (bits_e4m3(q0) != want) {
+            std::printf("exact path: x=%a s=%a got %.9g want %.9g\n", x, s, bits_e4m3(q0), want);
+            std::exit(1);
+        }
     };
     for (int n = 0; n < 2000000; ++n) {
         const float amax = amax_d(rng);
@@ -96,8 +104,8 @@ int main() {
                                     : (1.0 + (k + 0.5) / 8.0) * std::ldexp(1.0, E);
             check(static_cast<float>(M * 0.25), 0.25f);
         }
-    if (fixups == 0) {
-        std::printf("the constructed cases never exercised the residual step\n");
+    if (fixups == 0 || exact_path == 0) {
+        std::printf("the constructed cases never exercised the exact path or its residual step\n");
         return 1;
     }
     std::printf("ok\n");

@@ -40,11 +40,15 @@ void fail(const char* what, int a, int b, int c, int d) {
     if (failures++ < 10) std::printf("FAIL %s (%d %d %d %d)\n", what, a, b, c, d);
 }
 
-// Visit every CTA's walk and count the (s, h, blk) it yields.
+// Visit every CTA's walk and count the (s, h, blk) it yields.  With `rank`,
+// packed batches are dealt longest first (when they are small enough).
+// Returns the largest per-CTA cost over the mean per-CTA cost, a block's cost
+// taken as the keys it sees under a causal mask (or all of them).
 template <bool kTail>
-void check_cover(const fa::Geometry& g, const std::vector<int>& lens, int rows_per_item, int order,
-                 int G) {
+double check_cover(const fa::Geometry& g, const std::vector<int>& lens, int rows_per_item, int order,
+                   int G, bool rank = false) {
     std::vector<int> bpre(fa::kMaxVarlenSeqs + 1), upre(fa::kMaxVarlenSeqs + 1);
+    std::vector<short> rank_seq(fa::kMaxSortedSeqs, -1);
     std::vector<int> scratch(2);
     fa::Schedule sch;
     sch.g = g;
@@ -55,10 +59,23 @@ void check_cover(const fa::Geometry& g, const std::vector<int>& lens, int rows_p
     blockDim.x = 1;
     threadIdx.x = 0;
     gridDim.x = G;
+    bool ranked = false;
     sch.total_units = fa::build_schedule_prefix(g, rows_per_item, bpre.data(), upre.data(),
-                                                scratch.data());
+                                                scratch.data(), rank ? rank_seq.data() : nullptr,
+                                                &ranked);
+    sch.rank_seq = ranked ? rank_seq.data() : nullptr;
+    if (ranked) {
+        // the ranks are a permutation, longest first
+        std::vector<int> hit(g.B, 0);
+        for (int r = 0; r < g.B; ++r) {
+            const int sr = rank_seq[r];
+            if (sr < 0 || sr >= g.B || hit[sr]++) fail("rank order is not a permutation", r, sr, g.B, 0);
+            else if (r > 0 && lens[rank_seq[r - 1]] < lens[sr]) fail("rank order not longest first", r, sr, 0, 0);
+        }
+    }
     fa::schedule_split_tail(sch);
     std::map<std::tuple<int, int, int>, int> seen;
+    std::vector<double> cost(G, 0.0);
     for (int c = 0; c < G; ++c) {
         blockIdx.x = c;
         fa::ItemIter<kTail> it;
@@ -66,9 +83,11 @@ void check_cover(const fa::Geometry& g, const std::vector<int>& lens, int rows_p
         while (it.next(sch, s, h, blk)) {
             if (++guard > 1000000) {
                 fail("walk does not end", c, G, rows_per_item, order);
-                return;
+                return 0.0;
             }
             ++seen[std::make_tuple(s, h, blk)];
+            const int hi = min(lens[s], (blk + 1) * rows_per_item);
+            cost[c] += g.causal ? hi : lens[s];
         }
     }
     size_t expected = 0;
@@ -85,6 +104,12 @@ void check_cover(const fa::Geometry& g, const std::vector<int>& lens, int rows_p
     }
     if (seen.size() != expected) fail("walk yields blocks outside the batch", (int)seen.size(),
                                       (int)expected, G, order);
+    double mx = 0.0, tot = 0.0;
+    for (double v : cost) {
+        mx = std::max(mx, v);
+        tot += v;
+    }
+    return tot > 0.0 ? mx / (tot / G) : 1.0;
 }
 
 void check_masks(std::mt19937& rng) {
@@ -168,6 +193,41 @@ int main() {
         g.cu_seqlens_k = cu.data();
         for (int G : grids) check_cover<false>(g, lens, 256, 0, G);
         for (int G : grids) check_cover<true>(g, lens, 128, fa::schedule_order(g, 1), G);
+        for (int G : grids) check_cover<false>(g, lens, 256, 0, G, true);
+        for (int G : grids) check_cover<true>(g, lens, 128, fa::schedule_order(g, 1), G, true);
+    }
+    // the packed workload shape (16 sequences of 128..4096 tokens, 32 heads,
+    // causal, 148 CTAs): longest-first snake dealing balances the CTAs at
+    // least as well as dealing in sequence order, across many draws
+    {
+        double worst_plain = 0.0, worst_ranked = 0.0;
+        for (int trial = 0; trial < 50; ++trial) {
+            const int B = 16;
+            std::vector<int> lens(B), cu(B + 1, 0);
+            for (int s = 0; s < B; ++s) {
+                lens[s] = 128 + rng() % 3969;
+                cu[s + 1] = cu[s] + lens[s];
+            }
+            fa::Geometry g{};
+            g.B = B;
+            g.H = 32;
+            g.T = cu[B];
+            g.cu_seqlens = cu.data();
+            g.causal = 1;
+            g.Tk = g.T;
+            g.cu_seqlens_k = cu.data();
+            for (int rows : {128, 256}) {
+                const double plain = check_cover<false>(g, lens, rows, 0, 148);
+                const double ranked = check_cover<false>(g, lens, rows, 0, 148, true);
+                worst_plain = std::max(worst_plain, plain);
+                worst_ranked = std::max(worst_ranked, ranked);
+            }
+        }
+        if (worst_ranked > worst_plain || worst_ranked > 1.12)
+            fail("longest-first dealing does not balance the packed workload",
+                 (int)(1000 * worst_ranked), (int)(1000 * worst_plain), 0, 0);
+        std::fprintf(stderr, "packed workload, worst max/mean CTA cost: in order %.3f, longest first %.3f\n",
+                     worst_plain, worst_ranked);
     }
     check_masks(rng);
     if (failures) {
