@@ -53,8 +53,8 @@ struct FusedCfg {
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int OFF_SCRATCH = OFF_MISC + 16;
     static constexpr int OFF_PREFIX = OFF_SCRATCH + 2 * THREADS * 4;
-    static constexpr int OFF_RANK = OFF_PREFIX + 2 * (kMaxVarlenSeqs + 1) * 4;
-    static constexpr int SMEM_BYTES = OFF_RANK + kMaxSortedSeqs * 2 + 1024;
+    // block prefix, unit prefix, then the rank order (short[kMaxSortedSeqs])
+    static constexpr int SMEM_BYTES = OFF_PREFIX + 2 * (kMaxVarlenSeqs + 1) * 4 + kMaxSortedSeqs * 2 + 1024;
 };
 
 struct FusedParams {
@@ -90,7 +90,7 @@ dkdvq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
     int* scratch = reinterpret_cast<int*>(smem + C::OFF_SCRATCH);
     int* prefix = reinterpret_cast<int*>(smem + C::OFF_PREFIX);
-    float2* vec = reinterpret_cast<float2*>(smem + C::OFF_VEC);
+    float* vec = reinterpret_cast<float*>(smem + C::OFF_VEC);   // per stage: x[128], y[128]
     const int warp = threadIdx.x >> 5;
     const int lane = lane_id();
 
@@ -132,11 +132,8 @@ dkdvq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     sch.order = schedule_order(p.g, 0);     // key blocks: fewer queries see later keys
     sch.bprefix = prefix;
     sch.uprefix = prefix + kMaxVarlenSeqs + 1;
-    short* rank_seq = reinterpret_cast<short*>(smem + C::OFF_RANK);
-    bool ranked = false;
-    sch.total_units = build_schedule_prefix(p.g, 128, prefix, prefix + kMaxVarlenSeqs + 1, scratch,
-                                            rank_seq, &ranked);   // __syncthreads inside
-    sch.rank_seq = ranked ? rank_seq : nullptr;
+    sch.total_units = build_schedule_prefix(p.g, 128, prefix, prefix + kMaxVarlenSeqs + 1,
+                                            scratch);   // __syncthreads inside
     schedule_split_tail(sch);
     tc_fence_before();
     __syncthreads();
@@ -187,7 +184,7 @@ dkdvq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                                 tma_load_3d(st + C::TILE_BYTES + b * C::BOX, &tm_do, stage_full + slot,
                                             b * 64, h, sp.start + i * 128);
                             }
-                            bulk_load(vec + slot * 128,
+                            bulk_load(vec + slot * 256,
                                       p.stats + stats_index(p.g, p.stats_stride, s, h, blocks_before,
                                                             i * 128),
                                       C::VEC_BYTES, stage_full + slot);
@@ -317,7 +314,8 @@ dkdvq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 if (!mbar_wait(s_full, cnt & 1, wc)) { ok = false; break; }
                 if (!mbar_wait(stage_full + slot, (cnt / C::NSTAGE) & 1, wc)) { ok = false; break; }
                 tc_fence_after();
-                const float2* vs = vec + slot * 128 + 64 * g;   // {-L log2e, D}
+                const float* xs = vec + slot * 256 + 64 * g;   // -L log2e
+                const float* ys = xs + 128;                    // -D
                 const int q0 = i * 128 + 64 * g;       // this half's first query
                 const bool need_mask = (k0 + 128 > n) || (q0 + 64 > n) ||
                                        (p.g.causal && k0 + 127 > q0) ||
@@ -331,11 +329,11 @@ dkdvq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                     if (!need_mask) {
 #pragma unroll
                         for (int c = 32 * part; c < 32 * part + 32; ++c)
-                            pf[c] = ex2(fmaf(__uint_as_float(r[c]), sl2, vs[c].x));
+                            pf[c] = ex2(fmaf(__uint_as_float(r[c]), sl2, xs[c]));
                     } else {
 #pragma unroll
                         for (int c = 32 * part; c < 32 * part + 32; ++c) {
-                            const float x = ex2(fmaf(__uint_as_float(r[c]), sl2, vs[c].x));
+                            const float x = ex2(fmaf(__uint_as_float(r[c]), sl2, xs[c]));
                             pf[c] = (q0 + c < n && key_allowed(q0 + c, j, n, p.g.causal, p.g.window)) ? x : 0.f;
                         }
                     }
@@ -359,8 +357,8 @@ dkdvq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
 #pragma unroll
                     for (int c = 0; c < 16; ++c) {
                         const int k = 32 * part + 2 * c;
-                        const float d0 = pf[k] * (__uint_as_float(r[k]) - vs[k].y);
-                        const float d1 = pf[k + 1] * (__uint_as_float(r[k + 1]) - vs[k + 1].y);
+                        const float d0 = pf[k] * (__uint_as_float(r[k]) + ys[k]);
+                        const float d1 = pf[k + 1] * (__uint_as_float(r[k + 1]) + ys[k + 1]);
                         pk[c] = pack_bf16(pf[k] != 0.f ? d0 : 0.f, pf[k + 1] != 0.f ? d1 : 0.f);
                     }
                     tmem_st16(tP + 16 * part, pk);   // dS^T for the dK GEMM

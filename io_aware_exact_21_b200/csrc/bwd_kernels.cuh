@@ -42,16 +42,20 @@ namespace fa {
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Per-row statistics the two gradient kernels read, written by the pre-pass
-// into the workspace: {-LSE_i * log2(e), D_i} for each (sequence, head, row),
-// in a layout padded to 128-row blocks so that a streamed tile's statistics
-// are one aligned 1 KB bulk copy:
-//   fixed length: ((s * H + h) * stride) + i,     stride = N rounded up to 128
-//   packed:       h * stride + 128 * blocks(s) + i, blocks(s) = sum over earlier
+// into the workspace: x_i = -LSE_i * log2(e) and y_i = -D_i for each
+// (sequence, head, row), in a layout padded to 128-row blocks so that a
+// streamed tile's statistics are one aligned 1 KB bulk copy, and split within
+// each block (its 128 x values, then its 128 y values) so that consecutive
+// rows' values sit next to each other for packed float32x2 arithmetic.  Row i
+// of a (sequence, head) whose rows start at row index R (a multiple of 128):
+//   fixed length: R = (s * H + h) * stride,           stride = N rounded up to 128
+//   packed:       R = h * stride + 128 * blocks(s),    blocks(s) = sum over earlier
 //                 sequences of ceil(len / 128), stride >= 128 * blocks(B)
+//   x at float 2 (R + i - i % 128) + i % 128, y 128 floats further.
 // Entries of padding rows are never written; readers mask them.
 struct BwdParams {
     Geometry g;
-    const float2* stats;
+    const float* stats;
     int64_t stats_stride;
     const __nv_bfloat16* qrows;   // Q and dO (the dQ kernel reads its own rows directly)
     const __nv_bfloat16* dorows;
@@ -69,12 +73,15 @@ __device__ __forceinline__ size_t rowstat_index(const Geometry& g, int s, int h,
                         : (static_cast<size_t>(s) * g.H + h) * g.N + i;
 }
 
-// Index of row i of sequence s, head h in the padded statistics array;
-// `blocks_before` = 128-row blocks of the sequences before s (packed only).
+// Float index of x for row i of sequence s, head h in the padded statistics
+// array (y is 128 floats further); `blocks_before` = 128-row blocks of the
+// sequences before s (packed only).  For i a multiple of 128 it is the start
+// of that block's 1 KB.
 __device__ __forceinline__ size_t stats_index(const Geometry& g, int64_t stride, int s, int h,
                                               int blocks_before, int i) {
-    return g.cu_seqlens ? static_cast<size_t>(h) * stride + static_cast<size_t>(blocks_before) * 128 + i
-                        : (static_cast<size_t>(s) * g.H + h) * stride + i;
+    const size_t R = g.cu_seqlens ? static_cast<size_t>(h) * stride + static_cast<size_t>(blocks_before) * 128
+                                  : (static_cast<size_t>(s) * g.H + h) * stride;
+    return 2 * (R + (i & ~127)) + (i & 127);
 }
 
 // ------------------------------------------------------------ pre-pass --
@@ -87,7 +94,7 @@ __device__ __forceinline__ size_t stats_index(const Geometry& g, int64_t stride,
 template <int D>
 __global__ void __launch_bounds__(256)
 stats_kernel(const __nv_bfloat16* __restrict__ dO, const __nv_bfloat16* __restrict__ O,
-             const float* __restrict__ lse, float2* __restrict__ stats, int64_t stride,
+             const float* __restrict__ lse, float* __restrict__ stats, int64_t stride,
              Geometry g, float* __restrict__ dq_acc) {
     constexpr int LPR = D / 8;                 // lanes per row (16-byte vectors)
     constexpr int RPW = 32 / LPR;              // rows per warp per iteration
@@ -98,7 +105,7 @@ stats_kernel(const __nv_bfloat16* __restrict__ dO, const __nv_bfloat16* __restri
     int* scratch = cu + kMaxVarlenSeqs + 1;    // 2 * blockDim
     if (g.cu_seqlens) {
         for (int i = threadIdx.x; i <= g.B; i += blockDim.x) cu[i] = g.cu_seqlens[i];
-        build_schedule_prefix(g, 128, prefix, uprefix, scratch);   // __syncthreads inside
+        build_schedule_prefix(g, 128, prefix, uprefix, scratch, false);   // __syncthreads inside
     }
     const int lane = threadIdx.x & 31;
     const int sub = lane / LPR;
@@ -148,7 +155,9 @@ stats_kernel(const __nv_bfloat16* __restrict__ dO, const __nv_bfloat16* __restri
                 i = static_cast<int>(token - static_cast<int64_t>(s) * g.N);
             }
             const float l = lse[rowstat_index(g, s, h, g.cu_seqlens ? cu[s] : 0, i)];
-            stats[stats_index(g, stride, s, h, blocks_before, i)] = make_float2(-l * 1.4426950408889634f, acc);
+            const size_t xi = stats_index(g, stride, s, h, blocks_before, i);
+            stats[xi] = -l * 1.4426950408889634f;
+            stats[xi + 128] = -acc;
         }
     }
 }
@@ -175,8 +184,8 @@ struct BwdCfg {
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int OFF_SCRATCH = OFF_MISC + 16;
     static constexpr int OFF_PREFIX = OFF_SCRATCH + 2 * THREADS * 4;   // block and unit prefixes
-    static constexpr int OFF_RANK = OFF_PREFIX + 2 * (kMaxVarlenSeqs + 1) * 4;   // short[kMaxSortedSeqs]
-    static constexpr int SMEM_BYTES = OFF_RANK + kMaxSortedSeqs * 2 + 1024;
+    // block prefix, unit prefix, then the rank order (short[kMaxSortedSeqs])
+    static constexpr int SMEM_BYTES = OFF_PREFIX + 2 * (kMaxVarlenSeqs + 1) * 4 + kMaxSortedSeqs * 2 + 1024;
 };
 
 // Query-tile range [ib, ie) (tiles of BS rows) whose rows can see some key of
@@ -340,11 +349,8 @@ __device__ __forceinline__ uint32_t bwd_prologue(uint8_t* smem, const BwdBarrier
     sch.order = schedule_order(p.g, 0);     // key blocks: fewer queries see later keys
     sch.bprefix = prefix;
     sch.uprefix = prefix + kMaxVarlenSeqs + 1;
-    short* rank_seq = reinterpret_cast<short*>(smem + C::OFF_RANK);
-    bool ranked = false;
     sch.total_units = build_schedule_prefix(p.g, C::BM, prefix, prefix + kMaxVarlenSeqs + 1,
-                                            scratch, rank_seq, &ranked);   // __syncthreads inside
-    sch.rank_seq = ranked ? rank_seq : nullptr;
+                                            scratch);   // __syncthreads inside
     schedule_split_tail(sch);
     tc_fence_before();
     __syncthreads();
@@ -373,7 +379,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
     uint8_t* smem = align_smem_1024(smem_raw);
     const BwdBarriers br = carve_barriers<D>(smem);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
-    float2* vec = reinterpret_cast<float2*>(smem + C::OFF_VEC);
+    float* vec = reinterpret_cast<float*>(smem + C::OFF_VEC);   // per stage: x[128], y[128]
     const CUtensorMap* maps[4] = {&tm_k, &tm_v, &tm_q, &tm_do};
     Schedule sch;
     const uint32_t tmem = bwd_prologue<D>(smem, br, abort_flag, p, sch, maps);
@@ -425,7 +431,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                                             b * 64, h, sp.start + i * C::BS);
                             }
                             // the tile's per-query statistics, one aligned 1 KB copy
-                            bulk_load(vec + slot * C::BS,
+                            bulk_load(vec + slot * 2 * C::BS,
                                       p.stats + stats_index(p.g, p.stats_stride, s, h, blocks_before,
                                                             i * C::BS),
                                       C::VEC_BYTES, br.stage_full + slot);
@@ -546,7 +552,8 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                     break;
                 }
                 tc_fence_after();
-                const float2* vs = vec + (cnt % C::NSTAGE) * C::BS + 64 * g;   // {-L log2e, D}
+                const float* xs = vec + (cnt % C::NSTAGE) * 2 * C::BS + 64 * g;   // -L log2e
+                const float* ys = xs + C::BS;                                     // -D
                 const int q0 = i * C::BS + 64 * g;     // this half's first query
                 const bool need_mask = (k0 + C::BM > n) || (q0 + 64 > n) ||
                                        (p.g.causal && k0 + C::BM - 1 > q0) ||
@@ -558,15 +565,21 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
 #pragma unroll
                 for (int part = 0; part < 2; ++part) {
                     if (!need_mask) {
+                        // pairs of queries: the argument in packed float32x2
 #pragma unroll
-                        for (int c = 32 * part; c < 32 * part + 32; ++c)
-                            pf[c] = ex2(fmaf(__uint_as_float(r[c]), sl2, vs[c].x));
+                        for (int c = 32 * part; c < 32 * part + 32; c += 2) {
+                            const float2 a = ffma2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])),
+                                                   make_float2(sl2, sl2),
+                                                   *reinterpret_cast<const float2*>(xs + c));
+                            pf[c] = ex2(a.x);
+                            pf[c + 1] = ex2(a.y);
+                        }
                     } else {
                         // masked pairs, and query rows past the sequence end (their
                         // statistics are padding), get P = 0
 #pragma unroll
                         for (int c = 32 * part; c < 32 * part + 32; ++c) {
-                            const float x = ex2(fmaf(__uint_as_float(r[c]), sl2, vs[c].x));
+                            const float x = ex2(fmaf(__uint_as_float(r[c]), sl2, xs[c]));
                             pf[c] = (q0 + c < n && key_allowed(q0 + c, j, n, p.g.causal, p.g.window)) ? x : 0.f;
                         }
                     }
@@ -585,19 +598,22 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                 for (int part = 0; part < 2; ++part) {
                     uint32_t pk[16];
                     if (!need_mask) {
+                        // dS = P (dP - D), pairs of queries in packed float32x2
 #pragma unroll
                         for (int c = 0; c < 16; ++c) {
                             const int k = 32 * part + 2 * c;
-                            pk[c] = pack_bf16(pf[k] * (__uint_as_float(r[k]) - vs[k].y),
-                                              pf[k + 1] * (__uint_as_float(r[k + 1]) - vs[k + 1].y));
+                            const float2 d = fmul2(make_float2(pf[k], pf[k + 1]),
+                                                   fadd2(make_float2(__uint_as_float(r[k]), __uint_as_float(r[k + 1])),
+                                                         *reinterpret_cast<const float2*>(ys + k)));
+                            pk[c] = pack_bf16(d.x, d.y);
                         }
                     } else {
                         // P = 0 must give dS = 0 even where the padding D is not finite
 #pragma unroll
                         for (int c = 0; c < 16; ++c) {
                             const int k = 32 * part + 2 * c;
-                            const float d0 = pf[k] * (__uint_as_float(r[k]) - vs[k].y);
-                            const float d1 = pf[k + 1] * (__uint_as_float(r[k + 1]) - vs[k + 1].y);
+                            const float d0 = pf[k] * (__uint_as_float(r[k]) + ys[k]);
+                            const float d1 = pf[k + 1] * (__uint_as_float(r[k + 1]) + ys[k + 1]);
                             pk[c] = pack_bf16(pf[k] != 0.f ? d0 : 0.f, pf[k + 1] != 0.f ? d1 : 0.f);
                         }
                     }
@@ -652,8 +668,8 @@ struct DqCfg {
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int OFF_SCRATCH = OFF_MISC + 16;
     static constexpr int OFF_PREFIX = OFF_SCRATCH + 2 * THREADS * 4;
-    static constexpr int OFF_RANK = OFF_PREFIX + 2 * (kMaxVarlenSeqs + 1) * 4;   // short[kMaxSortedSeqs]
-    static constexpr int SMEM_BYTES = OFF_RANK + kMaxSortedSeqs * 2 + 1024;
+    // block prefix, unit prefix, then the rank order (short[kMaxSortedSeqs])
+    static constexpr int SMEM_BYTES = OFF_PREFIX + 2 * (kMaxVarlenSeqs + 1) * 4 + kMaxSortedSeqs * 2 + 1024;
 };
 
 struct DqBarriers {
@@ -729,11 +745,8 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
     sch.order = schedule_order(p.g, 1);     // query blocks: later queries see more keys
     sch.bprefix = prefix;
     sch.uprefix = prefix + kMaxVarlenSeqs + 1;
-    short* rank_seq = reinterpret_cast<short*>(smem + C::OFF_RANK);
-    bool ranked = false;
     sch.total_units = build_schedule_prefix(p.g, C::BM, prefix, prefix + kMaxVarlenSeqs + 1,
-                                            scratch, rank_seq, &ranked);   // __syncthreads inside
-    sch.rank_seq = ranked ? rank_seq : nullptr;
+                                            scratch);   // __syncthreads inside
     schedule_split_tail(sch);
     tc_fence_before();
     __syncthreads();
@@ -887,12 +900,11 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
                     tmem_st32(dst + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
                 arrive_warp(br.fix_ready);
             }
-            float nl = -INFINITY, dq_d = 0.f;
+            float nl = -INFINITY, neg_d = 0.f;     // -L log2e, -D of this row
             if (q < n) {
-                const float2 st = p.stats[stats_index(p.g, p.stats_stride, s, h,
-                                                      sch.blocks_before(s), q)];
-                nl = st.x;
-                dq_d = st.y;
+                const size_t xi = stats_index(p.g, p.stats_stride, s, h, sch.blocks_before(s), q);
+                nl = p.stats[xi];
+                neg_d = p.stats[xi + 128];
             }
             for (int j = jb; j < je; ++j, ++cnt) {
                 if (!mbar_wait(br.s_full, cnt & 1, wc)) { ok = false; break; }
@@ -907,8 +919,14 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
                 if (lane == 0) mbar_arrive(br.mid);     // S read: the next S may overwrite it
                 float pf[64];
                 if (!need_mask) {
+                    // pairs of keys: the argument in packed float32x2
 #pragma unroll
-                    for (int c = 0; c < 64; ++c) pf[c] = ex2(fmaf(__uint_as_float(r[c]), sl2, nl));
+                    for (int c = 0; c < 64; c += 2) {
+                        const float2 a = ffma2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])),
+                                               make_float2(sl2, sl2), make_float2(nl, nl));
+                        pf[c] = ex2(a.x);
+                        pf[c + 1] = ex2(a.y);
+                    }
                 } else {
 #pragma unroll
                     for (int c = 0; c < 64; ++c) {
@@ -926,8 +944,10 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
 #pragma unroll
                     for (int c = 0; c < 16; ++c) {
                         const int k = 32 * part + 2 * c;
-                        pk[c] = pack_bf16(pf[k] * (__uint_as_float(r[k]) - dq_d),
-                                          pf[k + 1] * (__uint_as_float(r[k + 1]) - dq_d));
+                        const float2 d = fmul2(make_float2(pf[k], pf[k + 1]),
+                                               fadd2(make_float2(__uint_as_float(r[k]), __uint_as_float(r[k + 1])),
+                                                     make_float2(neg_d, neg_d)));
+                        pk[c] = pack_bf16(d.x, d.y);
                     }
                     tmem_st16(tP + 16 * part, pk);   // dS packed over the first 32 columns of this half
                     arrive_warp(br.ready + part);
@@ -968,7 +988,7 @@ struct BwdArgs {
     const void *q, *o, *dO;
     const float* lse;
     void *dq, *dk, *dv;
-    float2* stats;           // workspace
+    float* stats;            // workspace
     int64_t stats_stride;
     float scale;
     int num_sms;

@@ -70,6 +70,16 @@ float e4m3_quotient_exact(float x, float s) {
     return q;
 }
 
+// The fast path's test: q1 at least 2^-6 in magnitude and more than 8
+// float32 steps from every e4m3 midpoint.
+__host__ __device__ __forceinline__ bool e4m3_product_safe(float q1) {
+    uint32_t bits;
+    memcpy(&bits, &q1, 4);
+    bits &= 0x7FFFFFFFu;
+    const int dist = static_cast<int>(bits & 0xFFFFFu) - 0x80000;
+    return bits >= 0x3C800000u /* 2^-6 */ && (dist > 8 || dist < -8);
+}
+
 // inv must be RN(1 / s).
 __host__ __device__ __forceinline__ float e4m3_quotient(float x, float s, float inv) {
 #ifdef __CUDA_ARCH__
@@ -77,12 +87,32 @@ __host__ __device__ __forceinline__ float e4m3_quotient(float x, float s, float 
 #else
     const float q1 = x * inv;
 #endif
-    uint32_t bits;
-    memcpy(&bits, &q1, 4);
-    bits &= 0x7FFFFFFFu;
-    const int dist = static_cast<int>(bits & 0xFFFFFu) - 0x80000;
-    const bool safe = bits >= 0x3C800000u /* 2^-6 */ && (dist > 8 || dist < -8);
-    return safe ? q1 : e4m3_quotient_exact(x, s);
+    return e4m3_product_safe(q1) ? q1 : e4m3_quotient_exact(x, s);
+}
+
+// Four at once: the products first, and the exact path only when one of them
+// needs it (one rarely taken branch per four values).
+__host__ __device__ __forceinline__ void e4m3_quotient4(const float (&x)[4], float s, float inv,
+                                                       float (&q)[4]) {
+    bool all_safe = true;
+#ifdef __CUDA_ARCH__
+#pragma unroll
+#endif
+    for (int e = 0; e < 4; ++e) {
+#ifdef __CUDA_ARCH__
+        q[e] = __fmul_rn(x[e], inv);
+#else
+        q[e] = x[e] * inv;
+#endif
+        all_safe = all_safe && e4m3_product_safe(q[e]);
+    }
+    if (!all_safe) {
+#ifdef __CUDA_ARCH__
+#pragma unroll
+#endif
+        for (int e = 0; e < 4; ++e)
+            if (!e4m3_product_safe(q[e])) q[e] = e4m3_quotient_exact(x[e], s);
+    }
 }
 
 }  // namespace fa

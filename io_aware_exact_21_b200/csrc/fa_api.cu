@@ -294,7 +294,8 @@ int launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const fa::Decode
 }
 
 // ------------------------------------------------ allocation-free backward --
-// Built-in scratch for fa_bwd_noalloc: the D values of one backward call.  In
+// Built-in scratch for fa_bwd_noalloc: the per-row statistics (two floats a
+// row, padded to 128-row blocks) of one backward call.  In
 // host code the symbol is only a host-side stand-in; kernels get the device
 // address looked up once per device below.
 static __device__ __align__(256) float2 g_noalloc_scratch[FA_NOALLOC_MAX_ROWS];
@@ -646,7 +647,7 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
     a.dq = dq;
     a.dk = dk;
     a.dv = dv;
-    a.stats = static_cast<float2*>(workspace);
+    a.stats = static_cast<float*>(workspace);
     a.stats_stride = stride;
     a.scale = scale;
     a.num_sms = st->num_sms;
@@ -700,7 +701,7 @@ int fa_bwd_fused(const void* q, const void* k, const void* v, const void* o, con
     a.dq = dq;
     a.dk = dk;
     a.dv = dv;
-    a.stats = static_cast<float2*>(workspace);
+    a.stats = static_cast<float*>(workspace);
     a.stats_stride = stride;
     a.scale = scale;
     a.num_sms = st->num_sms;
@@ -749,7 +750,7 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
     a.dq = dq;
     a.dk = dk;
     a.dv = dv;
-    a.stats = scratch;    // every entry the kernels use is written first by the pre-pass
+    a.stats = reinterpret_cast<float*>(scratch);   // every entry the kernels use is written first by the pre-pass
     a.stats_stride = stride;
     a.scale = scale;
     a.num_sms = st->num_sms;

@@ -133,9 +133,9 @@ quantize_fp8_kernel(const QuantParams p) {
     for (int k = 0; k < kQuantRows; ++k) {
         const int rr = warp + kQuantWarps * k;
         const int r = r0 + rr;
-        const uint32_t code =
-            pack_e4m3x4(e4m3_quotient(y[k][0], sc, inv), e4m3_quotient(y[k][1], sc, inv),
-                        e4m3_quotient(y[k][2], sc, inv), e4m3_quotient(y[k][3], sc, inv));
+        float q4[4];
+        e4m3_quotient4(y[k], sc, inv, q4);
+        const uint32_t code = pack_e4m3x4(q4[0], q4[1], q4[2], q4[3]);
         if (!p.transpose) {
             if (r < p.N)
                 *reinterpret_cast<uint32_t*>(

@@ -127,8 +127,8 @@ struct FwdCfg {
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int OFF_SCRATCH = OFF_MISC + 16;
     static constexpr int OFF_PREFIX = OFF_SCRATCH + 2 * THREADS * 4;   // block and unit prefixes
-    static constexpr int OFF_RANK = OFF_PREFIX + 2 * (kMaxVarlenSeqs + 1) * 4;   // short[kMaxSortedSeqs]
-    static constexpr int SMEM_BYTES = OFF_RANK + kMaxSortedSeqs * 2 + 1024;
+    // block prefix, unit prefix, then the rank order (short[kMaxSortedSeqs])
+    static constexpr int SMEM_BYTES = OFF_PREFIX + 2 * (kMaxVarlenSeqs + 1) * 4 + kMaxSortedSeqs * 2 + 1024;
 };
 
 template <int D, bool kF8 = false, bool kCache = false>
@@ -196,17 +196,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     sch.order = kCache ? 0 : schedule_order(p.g, 1);
     sch.bprefix = prefix;
     sch.uprefix = prefix + kMaxVarlenSeqs + 1;
-    short* rank_seq = reinterpret_cast<short*>(smem + C::OFF_RANK);
-    bool ranked = false;
     if constexpr (kCache) {
         sch.g.H = p.g.H * p.nsplit;             // (head, split) pairs
         sch.total_units = build_schedule_prefix(sch.g, C::ROWS, prefix,
                                                 prefix + kMaxVarlenSeqs + 1, scratch);
     } else {
         sch.total_units = build_schedule_prefix(p.g, C::ROWS, prefix, prefix + kMaxVarlenSeqs + 1,
-                                                scratch, rank_seq, &ranked);  // has __syncthreads
+                                                scratch);  // has __syncthreads
     }
-    sch.rank_seq = ranked ? rank_seq : nullptr;
     schedule_split_tail(sch);
     tc_fence_before();
     __syncthreads();

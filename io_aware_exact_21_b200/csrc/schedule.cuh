@@ -98,9 +98,9 @@ __device__ __forceinline__ bool tile_needs_mask(int r0, int BM, int k0, int BN, 
 // costly units to cheap ones and the costs even out across CTAs (a greedy
 // longest-first assignment in the usual sense).
 //
-// Pairs + snake tail (the backward kernels, for fixed length with a causal or
-// window mask, where a block's cost is monotone in its index; the forward
-// kernel keeps pairs alone): when the units per CTA are few, the
+// Pairs + snake tail (every kernel, for fixed length with a causal or window
+// mask, where a block's cost is monotone in its index): when the units per
+// CTA are few, the
 // last round of units leaves up to a unit's worth of imbalance.  So only the
 // whole heads that fit in all rounds but the last go out as units; the blocks
 // of the remaining heads are sorted heaviest first (block index major, then
@@ -117,9 +117,20 @@ struct Schedule {
     int tail_heads;         //   (sequence, head)s in the tail
     int tail_c0;            //   CTA that takes the tail's first block
     const int* bprefix;     // shared memory: blocks of the sequences before s (packed only)
-    const int* uprefix;     // shared memory: units of the sequences ranked before r (packed only)
-    const short* rank_seq;  // shared memory: the sequence at each rank, or nullptr (rank = index)
+    const int* uprefix;     // shared memory: units of the sequences ranked before r (packed
+                            // only), followed by the sequence of each rank (ranked_seqs)
     int total_units;
+
+    // Packed batches of up to kMaxSortedSeqs sequences are dealt longest first
+    // (build_schedule_prefix ranks them).  Derived from the geometry rather
+    // than stored: a field more stays live in a register across every role's
+    // loop, which measurably slows the kernels.
+    __device__ __forceinline__ bool ranked() const {
+        return g.cu_seqlens != nullptr && g.B <= kMaxSortedSeqs;
+    }
+    __device__ __forceinline__ const short* ranked_seqs() const {
+        return reinterpret_cast<const short*>(uprefix + kMaxVarlenSeqs + 1);
+    }
 
     __device__ __forceinline__ int blocks_of(int len) const {
         return (len + rows_per_item - 1) / rows_per_item;
@@ -169,7 +180,7 @@ struct Schedule {
                 int mid = (lo + hi + 1) >> 1;
                 if (uprefix[mid] * g.H <= w) lo = mid; else hi = mid - 1;
             }
-            s = rank_seq ? rank_seq[lo] : lo;
+            s = ranked() ? ranked_seqs()[lo] : lo;
             nu = uprefix[lo + 1] - uprefix[lo];
             nb = bprefix[s + 1] - bprefix[s];
             local = w - uprefix[lo] * g.H;
@@ -181,15 +192,13 @@ struct Schedule {
 
 // Walks the blocks one CTA processes: its units in order, both blocks of each
 // (pairs), then, with kTail and a non-zero order, its blocks of the snake
-// tail round by round.  Without kTail the walk is pairs alone (no tail state
-// is kept: the forward kernel's roles have no registers to spare).
+// tail round by round.  Without kTail the walk is pairs alone.
 template <bool kTail>
 struct ItemIter {
     int w;        // pairs: next unit
     int half;
-    int pround;   // pairs: round of the next unit
     int round;    // snake tail: next round
-    __device__ __forceinline__ ItemIter() : w(blockIdx.x), half(0), pround(0), round(0) {}
+    __device__ __forceinline__ ItemIter() : w(blockIdx.x), half(0), round(0) {}
     __device__ __forceinline__ bool next(const Schedule& sch, int& s, int& h, int& blk) {
         const int limit = (kTail && sch.order != 0) ? sch.bulk_units : sch.total_units;
         while (w < limit) {
@@ -203,10 +212,14 @@ struct ItemIter {
             half = 0;
             // the next round's unit: forwards in even rounds, backwards in odd
             // ones when the units run longest first, else w + gridDim.x
-            ++pround;
-            const int G = gridDim.x;
-            w = pround * G + ((sch.rank_seq && (pround & 1)) ? G - 1 - static_cast<int>(blockIdx.x)
-                                                             : static_cast<int>(blockIdx.x));
+            if (sch.ranked()) {
+                const int G = gridDim.x;
+                const int r = w / G + 1;
+                w = r * G + ((r & 1) ? G - 1 - static_cast<int>(blockIdx.x)
+                                     : static_cast<int>(blockIdx.x));
+            } else {
+                w += gridDim.x;
+            }
             if (nb - 1 - p != p) {
                 blk = nb - 1 - p;
                 return true;
@@ -254,22 +267,23 @@ __device__ __forceinline__ int schedule_order(const Geometry& g, int cost_grows_
 
 // Build the per-sequence block prefix (in sequence order) and the unit prefix
 // (in rank order) in shared memory (packed batches only) and return the number
-// of work units.  With `rank_seq` non-null and at most kMaxSortedSeqs
-// sequences, the ranks are by length, longest first (ties by index), and
-// rank_seq[r] receives the sequence of rank r; the caller then sets the
-// schedule's rank_seq to it, else to nullptr (rank = index).  Returns the rank
-// order's use through *ranked.  All threads of the CTA call it.
+// of work units.  `uprefix` must have room for kMaxVarlenSeqs + 1 ints and,
+// right after them, kMaxSortedSeqs shorts: with at most kMaxSortedSeqs
+// sequences (Schedule::ranked) the ranks are by length, longest first (ties
+// by index), and the sequence of each rank is stored there
+// (Schedule::ranked_seqs); otherwise the rank is the index.  With
+// `with_rank` false only the block prefix is needed (the unit prefix is then
+// in sequence order).  All threads of the CTA call it.
 __device__ __forceinline__ int build_schedule_prefix(const Geometry& g, int rows_per_item,
                                                      int* bprefix, int* uprefix,
                                                      int* scratch /* 2 * blockDim */,
-                                                     short* rank_seq = nullptr,
-                                                     bool* ranked = nullptr) {
-    if (ranked) *ranked = false;
+                                                     bool with_rank = true) {
     if (!g.cu_seqlens) {
         const int nb = (g.N + rows_per_item - 1) / rows_per_item;
         return g.B * g.H * ((nb + 1) >> 1);
     }
-    const bool sort = rank_seq != nullptr && g.B <= kMaxSortedSeqs;
+    const bool sort = with_rank && g.B <= kMaxSortedSeqs;
+    short* rank_seq = reinterpret_cast<short*>(uprefix + kMaxVarlenSeqs + 1);
     const int tid = threadIdx.x, nt = blockDim.x;
     const int per = (g.B + nt - 1) / nt;
     const int s0 = min(g.B, tid * per), s1 = min(g.B, s0 + per);
@@ -320,7 +334,6 @@ __device__ __forceinline__ int build_schedule_prefix(const Geometry& g, int rows
         uprefix[x + 1] += ou;
     }
     __syncthreads();
-    if (ranked) *ranked = sort;
     return uprefix[g.B] * g.H;
 }
 

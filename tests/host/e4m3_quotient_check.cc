@@ -62,6 +62,14 @@ int main() {
         const float inv = 1.f / s;
         const float q = fa::e4m3_quotient(x, s, inv);
         if (q != x * inv) ++exact_path;
+        // the four-at-once form agrees element by element
+        float xs4[4] = {x, x * 0.5f, -x, x * 3.0f}, q4[4];
+        fa::e4m3_quotient4(xs4, s, inv, q4);
+        for (int e = 0; e < 4; ++e)
+            if (bits_e4m3(q4[e]) != ref_e4m3(static_cast<double>(xs4[e]) / static_cast<double>(s))) {
+                std::printf("four-at-once: x=%a s=%a\n", xs4[e], s);
+                std::exit(1);
+            }
         const double want = ref_e4m3(static_cast<double>(x) / static_cast<double>(s));
         const double got = bits_e4m3(q);
         ++checked;

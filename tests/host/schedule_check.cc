@@ -40,15 +40,16 @@ void fail(const char* what, int a, int b, int c, int d) {
     if (failures++ < 10) std::printf("FAIL %s (%d %d %d %d)\n", what, a, b, c, d);
 }
 
-// Visit every CTA's walk and count the (s, h, blk) it yields.  With `rank`,
-// packed batches are dealt longest first (when they are small enough).
-// Returns the largest per-CTA cost over the mean per-CTA cost, a block's cost
-// taken as the keys it sees under a causal mask (or all of them).
+// Visit every CTA's walk and count the (s, h, blk) it yields.  Packed batches
+// of up to kMaxSortedSeqs sequences are dealt longest first (the schedule
+// derives that from the geometry).  Returns the largest per-CTA cost over the
+// mean per-CTA cost, a block's cost taken as the keys it sees under a causal
+// mask (or all of them).
 template <bool kTail>
 double check_cover(const fa::Geometry& g, const std::vector<int>& lens, int rows_per_item, int order,
-                   int G, bool rank = false) {
-    std::vector<int> bpre(fa::kMaxVarlenSeqs + 1), upre(fa::kMaxVarlenSeqs + 1);
-    std::vector<short> rank_seq(fa::kMaxSortedSeqs, -1);
+                   int G) {
+    // the unit prefix is followed by the rank order (kMaxSortedSeqs shorts)
+    std::vector<int> bpre(fa::kMaxVarlenSeqs + 1), upre(fa::kMaxVarlenSeqs + 1 + fa::kMaxSortedSeqs);
     std::vector<int> scratch(2);
     fa::Schedule sch;
     sch.g = g;
@@ -59,13 +60,11 @@ double check_cover(const fa::Geometry& g, const std::vector<int>& lens, int rows
     blockDim.x = 1;
     threadIdx.x = 0;
     gridDim.x = G;
-    bool ranked = false;
     sch.total_units = fa::build_schedule_prefix(g, rows_per_item, bpre.data(), upre.data(),
-                                                scratch.data(), rank ? rank_seq.data() : nullptr,
-                                                &ranked);
-    sch.rank_seq = ranked ? rank_seq.data() : nullptr;
-    if (ranked) {
+                                                scratch.data());
+    if (sch.ranked()) {
         // the ranks are a permutation, longest first
+        const short* rank_seq = sch.ranked_seqs();
         std::vector<int> hit(g.B, 0);
         for (int r = 0; r < g.B; ++r) {
             const int sr = rank_seq[r];
@@ -193,8 +192,6 @@ int main() {
         g.cu_seqlens_k = cu.data();
         for (int G : grids) check_cover<false>(g, lens, 256, 0, G);
         for (int G : grids) check_cover<true>(g, lens, 128, fa::schedule_order(g, 1), G);
-        for (int G : grids) check_cover<false>(g, lens, 256, 0, G, true);
-        for (int G : grids) check_cover<true>(g, lens, 128, fa::schedule_order(g, 1), G, true);
     }
     // the packed workload shape (16 sequences of 128..4096 tokens, 32 heads,
     // causal, 148 CTAs): longest-first snake dealing balances the CTAs at
@@ -217,9 +214,24 @@ int main() {
             g.Tk = g.T;
             g.cu_seqlens_k = cu.data();
             for (int rows : {128, 256}) {
-                const double plain = check_cover<false>(g, lens, rows, 0, 148);
-                const double ranked = check_cover<false>(g, lens, rows, 0, 148, true);
-                worst_plain = std::max(worst_plain, plain);
+                const double ranked = check_cover<false>(g, lens, rows, 0, 148);
+                // the same units dealt round robin in sequence order
+                std::vector<double> cost(148, 0.0);
+                int w = 0;
+                for (int sq = 0; sq < B; ++sq) {
+                    const int nb = (lens[sq] + rows - 1) / rows;
+                    for (int h = 0; h < g.H; ++h)
+                        for (int p = 0; p < (nb + 1) / 2; ++p, ++w) {
+                            cost[w % 148] += min(lens[sq], (p + 1) * rows);
+                            if (nb - 1 - p != p) cost[w % 148] += min(lens[sq], (nb - p) * rows);
+                        }
+                }
+                double mx = 0.0, tot = 0.0;
+                for (double v : cost) {
+                    mx = std::max(mx, v);
+                    tot += v;
+                }
+                worst_plain = std::max(worst_plain, mx / (tot / 148));
                 worst_ranked = std::max(worst_ranked, ranked);
             }
         }
