@@ -1,23 +1,25 @@
 // e4m3_quotient.cuh -- the float32 value whose e4m3 conversion (round to
-// nearest, ties to even) is the real quotient x / s rounded once to e4m3.
+// nearest, ties to even, saturating at +-448) is the real quotient x / s
+// rounded once to e4m3.
 //
-// Fast path: the product q1 = x * inv with inv = RN(1 / s) is within two
-// float32 steps of x / s (two roundings of relative size 2^-24 each), so when
-// q1 lies more than 8 steps from every e4m3 rounding boundary, x / s lies on
-// the same side and e4m3(q1) is the answer.  e4m3 midpoints in the normal
-// range (|q| >= 2^-6) have four significant bits with the fourth one set, so
-// the distance in float32 steps is the low 20 mantissa bits' distance from
-// 0x80000.  Values below 2^-6 (the subnormal range, rare for block-scaled
-// data) and values near a midpoint take the exact path.
-//
-// Exact path: the float32 quotient q = RN(x / s) rounds to the same e4m3
-// value as x / s unless q itself lies exactly halfway between two e4m3 values
-// while x / s does not (double rounding).  Only then the residual
-// r = x - q s, which one fused multiply-add computes exactly for a correctly
-// rounded quotient (the exact-remainder property of IEEE division), says on
-// which side of that midpoint x / s lies, and q moves one float32 step
-// towards it.  Below 2^-6 the midpoints are the odd multiples of 2^-10.
-// Requires s > 0.
+// The product q1 = x * inv with inv = RN(1 / s) is within two float32 steps
+// of x / s, so it names the e4m3 interval [V, V'] that x / s lies in or
+// borders.  Which way x / s rounds is decided by its side of that interval's
+// midpoint M: the sign of M s - |x|, which one fused multiply-add gives
+// exactly (the exact value is rounded once, and rounding keeps its sign and
+// whether it is zero).  The returned magnitude is M moved one float32 step
+// towards that side, or M itself on an exact tie, so its conversion gives V,
+// V' or the even one of the two.  When x / s lies just across V or V' (in a
+// neighbouring interval), it is close to that end and far from the
+// neighbour's midpoint, and the same rule picks that end, which is correct.
+//   normal range, |q1| >= 2^-6: M has q1's exponent and top three mantissa
+//     bits followed by a one (e4m3 keeps three mantissa bits);
+//   below 2^-6 (e4m3 subnormals, steps of 2^-9): M is the odd multiple of
+//     2^-10 inside q1's step.
+// Every step is exact arithmetic or one rounding, so no branch depends on how
+// close q1 happens to fall to a midpoint.  Requires s > 0; exact while
+// M s - |x| stays inside the float32 range (s >= 2^-100 suffices), which any
+// block scale of bf16 data above 448 * 2^-100 in magnitude satisfies.
 //
 // Self-contained (no CUDA headers) so that the host test can build it.
 #pragma once
@@ -28,91 +30,64 @@
 
 namespace fa {
 
-// Out of line: the kernel reaches it rarely, and one copy keeps the unrolled
-// quantiser loop small.
-#ifdef __CUDA_ARCH__
-__device__ __noinline__
-#else
-inline
-#endif
-float e4m3_quotient_exact(float x, float s) {
-#ifdef __CUDA_ARCH__
-    float q = __fdiv_rn(x, s);
-#else
-    float q = x / s;
-#endif
-    const float a = fabsf(q);
-    bool mid;
-    if (a >= 0.015625f) {
-        uint32_t bits;
-        memcpy(&bits, &a, 4);
-        mid = (bits & 0x7FFFFu) == 0u && (bits & 0x80000u) != 0u;
-    } else {
-        const float t = a * 1024.f;          // exact: a power-of-two scaling, t < 16
-        mid = t == floorf(t) && (static_cast<int>(t) & 1) == 1;
-    }
-    if (mid) {
-#ifdef __CUDA_ARCH__
-        const float r = __fmaf_rn(-q, s, x);
-#else
-        const float r = fmaf(-q, s, x);
-#endif
-        if (r != 0.f) {
-            // one float32 step towards x / s: up when r > 0 (s > 0)
-            uint32_t qb;
-            memcpy(&qb, &q, 4);
-            const bool up = r > 0.f;
-            const bool neg = (qb >> 31) != 0u;
-            qb = (up != neg) ? qb + 1u : qb - 1u;   // the magnitude grows iff moving away from 0
-            memcpy(&q, &qb, 4);
-        }
-    }
-    return q;
+__host__ __device__ __forceinline__ uint32_t e4m3q_bits(float f) {
+    uint32_t b;
+    memcpy(&b, &f, 4);
+    return b;
 }
 
-// The fast path's test: q1 at least 2^-6 in magnitude and more than 8
-// float32 steps from every e4m3 midpoint.
-__host__ __device__ __forceinline__ bool e4m3_product_safe(float q1) {
-    uint32_t bits;
-    memcpy(&bits, &q1, 4);
-    bits &= 0x7FFFFFFFu;
-    const int dist = static_cast<int>(bits & 0xFFFFFu) - 0x80000;
-    return bits >= 0x3C800000u /* 2^-6 */ && (dist > 8 || dist < -8);
+__host__ __device__ __forceinline__ float e4m3q_float(uint32_t b) {
+    float f;
+    memcpy(&f, &b, 4);
+    return f;
+}
+
+// The e4m3 midpoint M (as float32 bits) of the interval of |q1| = ab.
+__host__ __device__ __forceinline__ uint32_t e4m3q_mid_normal(uint32_t ab) {   // |q1| >= 2^-6
+    return (ab & 0xFFF00000u) | 0x80000u;
+}
+__host__ __device__ __forceinline__ uint32_t e4m3q_mid_small(uint32_t ab) {    // |q1| < 2^-6
+    // t * 2^-9 <= |q1| < (t + 1) * 2^-9, t in 0 .. 7; M = (t + 1/2) 2^-9
+    const float t = floorf(e4m3q_float(ab) * 512.f);   // exact scaling by 2^9
+    return e4m3q_bits((t + 0.5f) * 0.001953125f);      // exact: a 5-bit value times 2^-9
+}
+__host__ __device__ __forceinline__ uint32_t e4m3q_mid(uint32_t ab) {
+    return ab >= 0x3C800000u ? e4m3q_mid_normal(ab) : e4m3q_mid_small(ab);
+}
+
+// M moved one float32 step towards x / s (r > 0: x / s below M, r < 0:
+// above, r == 0: exactly M), with the sign of x.
+__host__ __device__ __forceinline__ float e4m3q_finish(float x, float s, uint32_t sign, uint32_t mb) {
+#ifdef __CUDA_ARCH__
+    const float r = __fmaf_rn(e4m3q_float(mb), s, -fabsf(x));
+#else
+    const float r = fmaf(e4m3q_float(mb), s, -fabsf(x));
+#endif
+    mb = mb + (r < 0.f ? 1u : 0u) - (r > 0.f ? 1u : 0u);
+    return e4m3q_float(mb | sign);
+}
+
+__host__ __device__ __forceinline__ float e4m3q_product(float x, float inv) {
+#ifdef __CUDA_ARCH__
+    return __fmul_rn(x, inv);
+#else
+    return x * inv;
+#endif
 }
 
 // inv must be RN(1 / s).
 __host__ __device__ __forceinline__ float e4m3_quotient(float x, float s, float inv) {
-#ifdef __CUDA_ARCH__
-    const float q1 = __fmul_rn(x, inv);
-#else
-    const float q1 = x * inv;
-#endif
-    return e4m3_product_safe(q1) ? q1 : e4m3_quotient_exact(x, s);
+    const uint32_t qb = e4m3q_bits(e4m3q_product(x, inv));
+    return e4m3q_finish(x, s, qb & 0x80000000u, e4m3q_mid(qb & 0x7FFFFFFFu));
 }
 
-// Four at once: the products first, and the exact path only when one of them
-// needs it (one rarely taken branch per four values).
+// Four values with one scale (the quantiser's unit of work).
 __host__ __device__ __forceinline__ void e4m3_quotient4(const float (&x)[4], float s, float inv,
                                                        float (&q)[4]) {
-    bool all_safe = true;
 #ifdef __CUDA_ARCH__
 #pragma unroll
 #endif
-    for (int e = 0; e < 4; ++e) {
-#ifdef __CUDA_ARCH__
-        q[e] = __fmul_rn(x[e], inv);
-#else
-        q[e] = x[e] * inv;
-#endif
-        all_safe = all_safe && e4m3_product_safe(q[e]);
-    }
-    if (!all_safe) {
-#ifdef __CUDA_ARCH__
-#pragma unroll
-#endif
-        for (int e = 0; e < 4; ++e)
-            if (!e4m3_product_safe(q[e])) q[e] = e4m3_quotient_exact(x[e], s);
-    }
+    for (int e = 0; e < 4; ++e) q[e] = e4m3_quotient(x[e], s, inv);
 }
 
 }  // namespace fa

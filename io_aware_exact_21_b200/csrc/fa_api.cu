@@ -118,6 +118,9 @@ int device_setup(DeviceState** out) {
             allow_smem(fa::fwd_kernel<128, true>, fa::FwdCfg<128, true>::SMEM_BYTES) != cudaSuccess ||
             allow_smem(fa::fwd_kernel<64, false, true>, fa::FwdCfg<64>::SMEM_BYTES) != cudaSuccess ||
             allow_smem(fa::fwd_kernel<128, false, true>, fa::FwdCfg<128>::SMEM_BYTES) != cudaSuccess ||
+            allow_smem(fa::quantize_fp8_kernel<true, false>, fa::QuantCfg::SMEM_BYTES) != cudaSuccess ||
+            allow_smem(fa::quantize_fp8_kernel<false, false>, fa::QuantCfg::SMEM_BYTES) != cudaSuccess ||
+            allow_smem(fa::quantize_fp8_kernel<false, true>, fa::QuantCfg::SMEM_BYTES) != cudaSuccess ||
             fa::bwd_set_smem_limits() != cudaSuccess || fa::fused_set_smem_limit() != cudaSuccess)
             return FA_ERR_CUDA;
         st.ready = true;
@@ -561,9 +564,20 @@ int fa_quantize_fp8(const void* x, void* out, float* scales, int B, int N, int H
     p.nb = static_cast<int>(nb);
     p.Np = static_cast<int>(fp8_vt_pitch(N));
     p.transpose = transpose ? 1 : 0;
+    p.error_word = st->error_word;
+    p.timeout_ns = g_fault_timeout_ns ? g_fault_timeout_ns : kDefaultTimeoutNs;
+    CUtensorMap mx;
+    if (make_map(&mx, x, rows, H, d, 128)) return FA_ERR_CUDA;
+    // persistent: two CTAs per SM walk the blocks
+    const int64_t nblocks = static_cast<int64_t>(B) * H * nb;
+    const int grid = static_cast<int>(std::min<int64_t>(nblocks, 2 * static_cast<int64_t>(st->num_sms)));
     const int slot = prof_start(6, stream);
-    fa::quantize_fp8_kernel<<<static_cast<int>(static_cast<int64_t>(B) * H * nb), 32 * fa::kQuantWarps, 0,
-                              stream>>>(p);
+    if (transpose)
+        fa::quantize_fp8_kernel<false, true><<<grid, fa::QuantCfg::THREADS, fa::QuantCfg::SMEM_BYTES, stream>>>(mx, p);
+    else if (signs)
+        fa::quantize_fp8_kernel<true, false><<<grid, fa::QuantCfg::THREADS, fa::QuantCfg::SMEM_BYTES, stream>>>(mx, p);
+    else
+        fa::quantize_fp8_kernel<false, false><<<grid, fa::QuantCfg::THREADS, fa::QuantCfg::SMEM_BYTES, stream>>>(mx, p);
     prof_stop(6, slot, stream);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
