@@ -331,10 +331,12 @@ dkdvq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                         for (int c = 32 * part; c < 32 * part + 32; ++c)
                             pf[c] = ex2(fmaf(__uint_as_float(r[c]), sl2, xs[c]));
                     } else {
+                        int c_lo, c_hi;      // this key's allowed queries of the half
+                        tile_query_bounds(j, q0, n, p.g.causal, p.g.window, 64, c_lo, c_hi);
 #pragma unroll
                         for (int c = 32 * part; c < 32 * part + 32; ++c) {
                             const float x = ex2(fmaf(__uint_as_float(r[c]), sl2, xs[c]));
-                            pf[c] = (q0 + c < n && key_allowed(q0 + c, j, n, p.g.causal, p.g.window)) ? x : 0.f;
+                            pf[c] = (c >= c_lo && c < c_hi) ? x : 0.f;
                         }
                     }
                     uint32_t pk[16];

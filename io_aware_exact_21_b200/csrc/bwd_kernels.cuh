@@ -576,11 +576,14 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                         }
                     } else {
                         // masked pairs, and query rows past the sequence end (their
-                        // statistics are padding), get P = 0
+                        // statistics are padding), get P = 0: this key's allowed
+                        // queries of the half are columns [c_lo, c_hi)
+                        int c_lo, c_hi;
+                        tile_query_bounds(j, q0, n, p.g.causal, p.g.window, 64, c_lo, c_hi);
 #pragma unroll
                         for (int c = 32 * part; c < 32 * part + 32; ++c) {
                             const float x = ex2(fmaf(__uint_as_float(r[c]), sl2, xs[c]));
-                            pf[c] = (q0 + c < n && key_allowed(q0 + c, j, n, p.g.causal, p.g.window)) ? x : 0.f;
+                            pf[c] = (c >= c_lo && c < c_hi) ? x : 0.f;
                         }
                     }
                     uint32_t pk[16];
@@ -928,10 +931,13 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
                         pf[c + 1] = ex2(a.y);
                     }
                 } else {
+                    // this row's allowed keys of the tile are columns [c_lo, c_hi)
+                    int c_lo, c_hi;
+                    tile_key_bounds(q, kb, n, p.g.causal, p.g.window, 64, c_lo, c_hi);
 #pragma unroll
                     for (int c = 0; c < 64; ++c) {
                         const float x = ex2(fmaf(__uint_as_float(r[c]), sl2, nl));
-                        pf[c] = key_allowed(q, kb + c, n, p.g.causal, p.g.window) ? x : 0.f;
+                        pf[c] = (c >= c_lo && c < c_hi) ? x : 0.f;
                     }
                 }
                 if (!mbar_wait(br.dp_full, cnt & 1, wc)) { ok = false; break; }

@@ -494,9 +494,11 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 const bool masked = tile_needs_mask_pos(r0 + off, min(r0 + C::BM, n) + off, k0, C::BN,
                                                         nk, p.g.causal, p.g.window);
                 if (masked) {
+                    // this row's allowed keys of the tile are columns [c_lo, c_hi)
+                    int c_lo, c_hi;
+                    tile_key_bounds(i + off, k0, nk, p.g.causal, p.g.window, C::BN, c_lo, c_hi);
 #pragma unroll
-                    for (int c = 0; c < C::BN; ++c)
-                        if (!key_allowed(i + off, k0 + c, nk, p.g.causal, p.g.window)) sv[c] = -INFINITY;
+                    for (int c = 0; c < C::BN; ++c) sv[c] = (c >= c_lo && c < c_hi) ? sv[c] : -INFINITY;
                 }
                 // row maximum as a tree of three-input maxima (the max is exact
                 // in any order), so the compares are not one dependent chain

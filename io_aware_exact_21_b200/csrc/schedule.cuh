@@ -43,6 +43,31 @@ __device__ __forceinline__ bool key_allowed(int i, int j, int n, int causal, int
     return j < n && (!causal || j <= i) && (window <= 0 || j > i - window);
 }
 
+// The same test for one row against a tile, as a column range: key k0 + c is
+// allowed for row position ip iff c_lo <= c < c_hi (0 <= c_lo <= c_hi <= BN),
+// so a masked tile costs two compares per element.
+__device__ __forceinline__ void tile_key_bounds(int ip, int k0, int nk, int causal, int window, int BN,
+                                                int& c_lo, int& c_hi) {
+    int hi = nk - k0;                                    // k0 + c < nk
+    if (causal) hi = min(hi, ip - k0 + 1);               // k0 + c <= ip
+    const int lo = window > 0 ? max(0, ip - window + 1 - k0) : 0;   // k0 + c > ip - window
+    c_lo = min(lo, BN);
+    c_hi = max(c_lo, min(hi, BN));
+}
+
+// And for one key against a tile of queries (self-attention, n rows): query
+// q0 + c may attend key j iff c_lo <= c < c_hi (0 <= c_lo <= c_hi <= BM);
+// queries past n get none.
+__device__ __forceinline__ void tile_query_bounds(int j, int q0, int n, int causal, int window, int BM,
+                                                  int& c_lo, int& c_hi) {
+    int hi = n - q0;                                     // q0 + c < n
+    if (j >= n) hi = 0;                                  // the key itself exists
+    if (window > 0) hi = min(hi, j + window - q0);       // j > q0 + c - window
+    const int lo = causal ? max(0, j - q0) : 0;          // j <= q0 + c
+    c_lo = min(lo, BM);
+    c_hi = max(c_lo, min(hi, BM));
+}
+
 // Key-tile range [jb, je) that queries at key positions [p_lo, p_hi) need in
 // a key sequence of length nk, for key tiles of BN keys; tiles outside it are
 // fully masked and never loaded.  An empty range becomes one (fully masked)

@@ -7,7 +7,10 @@
 //   2. the key-tile range of a block holds every key any of its rows may see,
 //      and the tiles outside it hold none;
 //   3. a tile classified as needing no mask has every (row, key) pair of the
-//      block allowed.
+//      block allowed;
+//   4. the column ranges the kernels mask with (tile_key_bounds for a row
+//      against a key tile, tile_query_bounds for a key against a query tile)
+//      hold exactly the pairs key_allowed allows.
 // The CUDA built-ins the header reads (blockIdx, gridDim, threadIdx,
 // blockDim, __syncthreads) are host variables here; the packed-batch prefix
 // is built by one emulated thread.  Prints "ok" and exits 0, or names the
@@ -144,6 +147,39 @@ void check_masks(std::mt19937& rng) {
     }
 }
 
+void check_bounds(std::mt19937& rng) {
+    for (int trial = 0; trial < 3000; ++trial) {
+        const int n = 1 + rng() % 700;
+        const int causal = rng() % 3 != 0;
+        const int window = rng() % 2 ? 1 + rng() % 400 : 0;
+        const int BN = rng() % 2 ? 128 : 64;
+        const int nk = n + (rng() % 2 ? 0 : static_cast<int>(rng() % 300));   // cached keys before the queries
+        const int off = nk - n;
+        // a row against key tiles (query positions shifted by off, keys of nk)
+        const int i = rng() % n;
+        for (int k0 = 0; k0 < nk + BN; k0 += BN) {
+            int lo, hi;
+            fa::tile_key_bounds(i + off, k0, nk, causal, window, BN, lo, hi);
+            if (lo < 0 || hi < lo || hi > BN) fail("key bounds out of range", lo, hi, BN, k0);
+            for (int c = 0; c < BN; ++c)
+                if ((c >= lo && c < hi) != fa::key_allowed(i + off, k0 + c, nk, causal, window))
+                    fail("tile_key_bounds disagrees with key_allowed", i, k0, c, window);
+        }
+        // a key against query tiles (self-attention, n rows, queries past n
+        // allowed nothing)
+        const int j = rng() % (n + 3);
+        for (int q0 = 0; q0 < n + BN; q0 += 64) {
+            int lo, hi;
+            fa::tile_query_bounds(j, q0, n, causal, window, BN, lo, hi);
+            if (lo < 0 || hi < lo || hi > BN) fail("query bounds out of range", lo, hi, BN, q0);
+            for (int c = 0; c < BN; ++c) {
+                const bool want = q0 + c < n && fa::key_allowed(q0 + c, j, n, causal, window);
+                if ((c >= lo && c < hi) != want) fail("tile_query_bounds disagrees with key_allowed", j, q0, c, window);
+            }
+        }
+    }
+}
+
 }  // namespace
 
 int main() {
@@ -242,6 +278,7 @@ int main() {
                      worst_plain, worst_ranked);
     }
     check_masks(rng);
+    check_bounds(rng);
     if (failures) {
         std::printf("%d violations\n", failures);
         return 1;
