@@ -632,14 +632,13 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             const size_t off = (static_cast<size_t>(sp.start) + j) * H * D + static_cast<size_t>(h) * D;
             if (g == 0) {
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c)
-                    store_row_chunk(tmem + lane_base + C::COL_ACC1 + c * 32, 1.f, p.out1 + off + c * 32,
-                                    valid);
+                for (int c = 0; c < D / 64; ++c)
+                    store_line_bf16(tmem + lane_base + C::COL_ACC1 + c * 64, 1.f, p.out1 + off + c * 64, valid);
             } else {
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c)
-                    store_row_chunk(tmem + lane_base + C::COL_ACC0 + c * 32, p.scale,
-                                    p.out0 + off + c * 32, valid);
+                for (int c = 0; c < D / 64; ++c)
+                    store_line_bf16(tmem + lane_base + C::COL_ACC0 + c * 64, p.scale, p.out0 + off + c * 64,
+                                    valid);
             }
             tc_fence_before();
             __syncwarp();
@@ -965,10 +964,15 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
             tc_fence_after();
             const bool valid = q < n;
             const size_t off = (static_cast<size_t>(sp.start) + q) * H * D + static_cast<size_t>(h) * D;
+            if constexpr (D == 128) {
+                // this group's 64 columns: one 128-byte line of the row
+                store_line_bf16(tmem + lane_base + C::COL_DQ + g * 64, p.scale, p.out0 + off + g * 64, valid);
+            } else {
 #pragma unroll
-            for (int c = 0; c < D / 64; ++c) {
-                const int col = g * (D / 2) + c * 32;
-                store_row_chunk(tmem + lane_base + C::COL_DQ + col, p.scale, p.out0 + off + col, valid);
+                for (int c = 0; c < D / 64; ++c) {
+                    const int col = g * (D / 2) + c * 32;
+                    store_row_chunk(tmem + lane_base + C::COL_DQ + col, p.scale, p.out0 + off + col, valid);
+                }
             }
             tc_fence_before();
             __syncwarp();

@@ -606,23 +606,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             }
             __nv_bfloat16* orow = p.o + (static_cast<size_t>(sp.start) + i) * H * D +
                                   static_cast<size_t>(h) * D;
+            // 64 columns (one 128-byte line of the row) at a time, whole lines
+            // per store instruction
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tO + c * 32, r);
-                tmem_wait_ld();
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    pk[e] = pack_bf16(__uint_as_float(r[2 * e]) * inv_l,
-                                      __uint_as_float(r[2 * e + 1]) * inv_l);
-                if (valid) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-                }
-            }
+            for (int c = 0; c < D / 64; ++c) store_line_bf16(tO + c * 64, inv_l, orow + c * 64, valid);
             if (valid) {
                 const float lse = l > 0.f ? (m_ref + __log2f(l)) * kLn2 : -INFINITY;
                 const size_t idx = p.g.cu_seqlens

@@ -347,6 +347,59 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Warp-cooperative store of one 128-byte line per lane: 64 bf16 values of the
+// lane's row, read from 64 TMEM columns at `taddr` and multiplied by `mul`,
+// to `dst` (16-byte aligned; not written when `valid` is false).  Written
+// lane by lane, every store instruction would touch 32 lines; instead the 8
+// 16-byte chunks of each lane are transposed within groups of 8 lanes (three
+// exchange stages of shuffles), after which instruction k has lanes
+// 8q .. 8q + 7 write the 8 chunks of lane 8q + k's line: 4 whole lines per
+// instruction.  The whole warp must call it.
+__device__ __forceinline__ void store_line_bf16(uint32_t taddr, float mul, void* dst, bool valid) {
+    uint32_t r0[32], r1[32];
+    tmem_ld32(taddr, r0);
+    tmem_ld32(taddr + 32, r1);
+    tmem_wait_ld();
+    uint4 ch[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        ch[j] = make_uint4(pack_bf16(__uint_as_float(r0[8 * j]) * mul, __uint_as_float(r0[8 * j + 1]) * mul),
+                           pack_bf16(__uint_as_float(r0[8 * j + 2]) * mul, __uint_as_float(r0[8 * j + 3]) * mul),
+                           pack_bf16(__uint_as_float(r0[8 * j + 4]) * mul, __uint_as_float(r0[8 * j + 5]) * mul),
+                           pack_bf16(__uint_as_float(r0[8 * j + 6]) * mul, __uint_as_float(r0[8 * j + 7]) * mul));
+        ch[j + 4] = make_uint4(pack_bf16(__uint_as_float(r1[8 * j]) * mul, __uint_as_float(r1[8 * j + 1]) * mul),
+                               pack_bf16(__uint_as_float(r1[8 * j + 2]) * mul, __uint_as_float(r1[8 * j + 3]) * mul),
+                               pack_bf16(__uint_as_float(r1[8 * j + 4]) * mul, __uint_as_float(r1[8 * j + 5]) * mul),
+                               pack_bf16(__uint_as_float(r1[8 * j + 6]) * mul, __uint_as_float(r1[8 * j + 7]) * mul));
+    }
+    const int lane = lane_id();
+    const int l8 = lane & 7;
+    // transpose: lane l8 of a group ends up holding, at index k, chunk l8 of
+    // group lane k's line (the off-diagonal halves swap at each stage)
+#pragma unroll
+    for (int b = 1; b < 8; b <<= 1) {
+        const bool up = (l8 & b) != 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            if (i & b) continue;
+            const uint4 send = up ? ch[i] : ch[i | b];
+            uint4 recv;
+            recv.x = __shfl_xor_sync(0xffffffffu, send.x, b);
+            recv.y = __shfl_xor_sync(0xffffffffu, send.y, b);
+            recv.z = __shfl_xor_sync(0xffffffffu, send.z, b);
+            recv.w = __shfl_xor_sync(0xffffffffu, send.w, b);
+            if (up) ch[i] = recv;
+            else ch[i | b] = recv;
+        }
+    }
+    const unsigned long long mine = valid ? reinterpret_cast<unsigned long long>(dst) : 0ull;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const unsigned long long line = __shfl_sync(0xffffffffu, mine, (lane & ~7) | k);
+        if (line) *reinterpret_cast<uint4*>(line + 16 * l8) = ch[k];
+    }
+}
+
 // Two floats to two e4m3 bytes (round to nearest even, saturating at
 // +-448): `lo` in the low byte.
 __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
