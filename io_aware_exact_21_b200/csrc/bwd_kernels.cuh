@@ -463,8 +463,10 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                 const int k0 = blk * C::BM;
                 int ib, ie;
                 query_tile_range(k0, min(n, k0 + C::BM), n, p.g.causal, p.g.window, C::BS, ib, ie);
+                // the item's first S^T and dP^T do not touch the accumulators, so
+                // they run while the element-wise warps still store the previous
+                // item's dK and dV; the accumulators are awaited before the first dV
                 if (!mbar_wait(br.fix_full, item_it & 1, wc)) { ok = false; break; }
-                if (!mbar_wait(br.acc_empty, (item_it & 1) ^ 1, wc)) { ok = false; break; }
                 if (!mbar_wait(br.stage_full + cnt % C::NSTAGE, (cnt / C::NSTAGE) & 1, wc)) {
                     ok = false;
                     break;
@@ -476,7 +478,10 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                     umma_commit(br.s_full);
                     issue_scores_ss<D>(tmem + C::COL_DP, fb_addr, x + C::TILE_BYTES);  // V dO^T
                     umma_commit(br.dp_full);
+                    if (ib + 1 == ie) umma_commit(br.fix_empty);   // K and V read for the last time
                 }
+                if (!mbar_wait(br.acc_empty, (item_it & 1) ^ 1, wc)) { ok = false; break; }
+                tc_fence_after();
                 for (int i = ib; i < ie; ++i, ++cnt) {
                     const bool last = (i + 1 == ie);
                     const uint32_t slot = cnt % C::NSTAGE;
@@ -510,9 +515,11 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                     if (!last) {
                         issue_scores_ss<D>(tmem + C::COL_DP, fb_addr, xn + C::TILE_BYTES);  // next V dO^T
                         umma_commit(br.dp_full);
+                        // K and V read for the last time: the producer may load the
+                        // next item's while this one finishes
+                        if (i + 2 == ie) umma_commit(br.fix_empty);
                     } else {
                         umma_commit(br.acc_final);
-                        umma_commit(br.fix_empty);
                     }
                 }
             }
@@ -806,8 +813,10 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
                 const int q0 = blk * C::BM;
                 int jb, je;
                 key_tile_range(q0, min(n, q0 + C::BM), n, p.g.causal, p.g.window, C::BS, jb, je);
+                // the block's first S and dP do not touch the dQ accumulator, so
+                // they run during the previous block's epilogue; the
+                // accumulator is awaited before the first dQ GEMM
                 if (!mbar_wait(br.fix_ready, item_it & 1, wc)) { ok = false; break; }
-                if (!mbar_wait(br.acc_empty, (item_it & 1) ^ 1, wc)) { ok = false; break; }
                 if (!mbar_wait(br.stage_full + cnt % C::NSTAGE, (cnt / C::NSTAGE) & 1, wc)) {
                     ok = false;
                     break;
@@ -820,6 +829,8 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
                     issue_scores_ts<D>(tmem + C::COL_DP, tmem + C::COL_DO, x + C::TILE_BYTES);  // dO V^T
                     umma_commit(br.dp_full);
                 }
+                if (!mbar_wait(br.acc_empty, (item_it & 1) ^ 1, wc)) { ok = false; break; }
+                tc_fence_after();
                 for (int j = jb; j < je; ++j, ++cnt) {
                     const bool last = (j + 1 == je);
                     const uint32_t slot = cnt % C::NSTAGE;
@@ -870,38 +881,43 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
         const uint32_t tP = tmem + lane_base + C::COL_DP + 64 * g;
         uint32_t cnt = 0, item_it = 0;
         bool ok = true;
+        // this thread's row of Q (warpgroup 0) or dO (warpgroup 1) of block
+        // (s, h, blk) into TMEM as packed bf16 pairs; rows past the sequence
+        // end are zero.  Called before the first block, and for every later
+        // block once the previous block's last S and dP have completed (the
+        // only GEMMs that read these columns), ahead of that block's epilogue.
+        auto load_rows = [&](int s_, int h_, int blk_) {
+            const SeqSpan sp_ = sch.span(s_);
+            const int qr = blk_ * C::BM + row;
+            const __nv_bfloat16* src = (g == 0 ? p.qrows : p.dorows) +
+                                       ((static_cast<size_t>(sp_.start) + qr) * H + h_) * D;
+            uint32_t r[D / 2];
+#pragma unroll
+            for (int v = 0; v < D / 8; ++v) {
+                uint4 x4 = make_uint4(0, 0, 0, 0);
+                if (qr < sp_.len) x4 = __ldg(reinterpret_cast<const uint4*>(src) + v);
+                r[4 * v] = x4.x;
+                r[4 * v + 1] = x4.y;
+                r[4 * v + 2] = x4.z;
+                r[4 * v + 3] = x4.w;
+            }
+            const uint32_t dst = tmem + lane_base + (g == 0 ? C::COL_Q : C::COL_DO);
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c)
+                tmem_st32(dst + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+            arrive_warp(br.fix_ready);
+        };
         ItemIter<true> it;
         int s, h, blk;
-        for (; ok && it.next(sch, s, h, blk); ++item_it) {
+        bool have = it.next(sch, s, h, blk);
+        if (have) load_rows(s, h, blk);
+        for (; ok && have; ++item_it) {
             const SeqSpan sp = sch.span(s);
             const int n = sp.len;
             const int q0 = blk * C::BM;
             const int q = q0 + row;               // this thread's query row
             int jb, je;
             key_tile_range(q0, min(n, q0 + C::BM), n, p.g.causal, p.g.window, C::BS, jb, je);
-            {
-                // this row of Q (warpgroup 0) or dO (warpgroup 1) into TMEM as
-                // packed bf16 pairs; rows past the sequence end are zero.  The
-                // previous block's GEMMs have all completed (its epilogue waited
-                // for the last one), so the columns are free.
-                const __nv_bfloat16* src = (g == 0 ? p.qrows : p.dorows) +
-                                           ((static_cast<size_t>(sp.start) + q) * H + h) * D;
-                uint32_t r[D / 2];
-#pragma unroll
-                for (int v = 0; v < D / 8; ++v) {
-                    uint4 x4 = make_uint4(0, 0, 0, 0);
-                    if (q < n) x4 = __ldg(reinterpret_cast<const uint4*>(src) + v);
-                    r[4 * v] = x4.x;
-                    r[4 * v + 1] = x4.y;
-                    r[4 * v + 2] = x4.z;
-                    r[4 * v + 3] = x4.w;
-                }
-                const uint32_t dst = tmem + lane_base + (g == 0 ? C::COL_Q : C::COL_DO);
-#pragma unroll
-                for (int c = 0; c < D / 64; ++c)
-                    tmem_st32(dst + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
-                arrive_warp(br.fix_ready);
-            }
             float nl = -INFINITY, neg_d = 0.f;     // -L log2e, -D of this row
             if (q < n) {
                 const size_t xi = stats_index(p.g, p.stats_stride, s, h, sch.blocks_before(s), q);
@@ -959,6 +975,11 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
                 }
             }
             if (!ok) break;
+            // the next block's rows first, so that its first S and dP run
+            // during this block's epilogue
+            int s_next, h_next, blk_next;
+            const bool have_next = it.next(sch, s_next, h_next, blk_next);
+            if (have_next) load_rows(s_next, h_next, blk_next);
             // ------------------------------------------------ epilogue --
             if (!mbar_wait(br.acc_final, item_it & 1, wc)) { ok = false; break; }
             tc_fence_after();
@@ -977,6 +998,10 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(br.acc_empty);
+            s = s_next;
+            h = h_next;
+            blk = blk_next;
+            have = have_next;
         }
     }
     tc_fence_before();
