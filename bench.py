@@ -62,16 +62,18 @@ NOMINAL_BF16_DENSE_TFLOPS = 2250.0
 # the kernel sources a capture was taken on: each entry carries a hash of their
 # comment-free text and is reported as null once that changes.
 TRAFFIC = {
-    "fwd": {"bytes_per_launch": 2 * (207.10e6 + 48.93e6), "workload": "train",
-            "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh"), "sha": "db7381e1f845ff58"},
-    "dkdv": {"bytes_per_launch": 2 * (271.87e6 + 107.11e6), "workload": "train",
-             "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "eac9bf149dae49e0"},
-    "dq": {"bytes_per_launch": 2 * (271.07e6 + 53.35e6), "workload": "train",
-           "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "eac9bf149dae49e0"},
-    "decode": {"bytes_per_launch": 792.82e6 + 5.62e6, "workload": "decode",
-               "sources": ("decode_kernel.cuh", "sm100.cuh"), "sha": "5424c1188ad151db"},
-    "fwd_fp8": {"bytes_per_launch": 2 * (101.02e6 + 32.14e6), "workload": "fp8",
-                "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh"), "sha": "db7381e1f845ff58"},
+    "fwd": {"bytes_per_launch": 2 * (208.53e6 + 49.55e6), "workload": "train",
+            "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh"), "sha": "f96a3e0f94d3bdba"},
+    "dot": {"bytes_per_launch": 2 * (135.30e6 + 4.94e6), "workload": "train",
+            "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "1a04cdea55ac7705"},
+    "dkdv": {"bytes_per_launch": 2 * (275.31e6 + 109.41e6), "workload": "train",
+             "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "1a04cdea55ac7705"},
+    "dq": {"bytes_per_launch": 2 * (271.99e6 + 53.04e6), "workload": "train",
+           "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "1a04cdea55ac7705"},
+    "decode": {"bytes_per_launch": 792.89e6 + 4.95e6, "workload": "decode",
+               "sources": ("decode_kernel.cuh", "sm100.cuh"), "sha": "34b0f87f0cc6cfec"},
+    "fwd_fp8": {"bytes_per_launch": 2 * (100.99e6 + 35.70e6), "workload": "fp8",
+                "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh"), "sha": "f96a3e0f94d3bdba"},
 }
 
 
