@@ -289,12 +289,11 @@ int fa_bwd_fused(const void* q, const void* k, const void* v, const void* o, con
  *   FA_ERR_SCRATCH_LIMIT and launch nothing; use fa_bwd for them.
  * - It calls no cudaMalloc / cudaFree and no allocating library routine.
  * - The first call on a device looks up the array's device address (a
- *   one-time set-up with that device current); make that first call before
- *   any stream capture.
- * - All calls share the one array per device and leave their D values in it;
- *   every call rewrites the part it uses before reading it.  Calls whose
- *   kernels overlap on the GPU (different streams, or different host threads)
- *   race on the array: serialise them.
+ *   one-time set-up with that device current).
+ * - All calls share the one array per device and leave their per-row
+ *   statistics in it; every call rewrites the part it uses before reading
+ *   it.  Calls whose kernels overlap on the GPU (different streams, or
+ *   different host threads) race on the array: serialise them.
  */
 #define FA_NOALLOC_MAX_ROWS (1 << 20)
 int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
