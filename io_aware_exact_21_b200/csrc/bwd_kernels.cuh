@@ -92,7 +92,7 @@ __device__ __forceinline__ size_t stats_index(const Geometry& g, int64_t stride,
 // With dq_acc non-null (the fused backward) it also zeroes that fp32 [rows, d]
 // accumulator, row by row.
 template <int D>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 8)
 stats_kernel(const __nv_bfloat16* __restrict__ dO, const __nv_bfloat16* __restrict__ O,
              const float* __restrict__ lse, float* __restrict__ stats, int64_t stride,
              Geometry g, float* __restrict__ dq_acc) {
@@ -115,6 +115,38 @@ stats_kernel(const __nv_bfloat16* __restrict__ dO, const __nv_bfloat16* __restri
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
     for (int64_t base = warp_global * RPW; base < rows; base += nwarps * RPW) {
         const int64_t r = base + sub;
+        // the row's place (and its LSE load) first, so that the LSE read is in
+        // flight together with the dO and O rows
+        bool out = false;
+        float l = 0.f;
+        size_t xi = 0;
+        if (r < rows && part == 0) {
+            const int64_t token = r / g.H;
+            const int h = static_cast<int>(r - token * g.H);
+            int s = 0, i = 0, blocks_before = 0;
+            bool inside = true;
+            if (g.cu_seqlens) {
+                inside = token < cu[g.B];              // else a row outside every sequence
+                if (inside) {
+                    int lo = 0, hi = g.B - 1;          // last s with cu[s] <= token
+                    while (lo < hi) {
+                        const int mid = (lo + hi + 1) >> 1;
+                        if (cu[mid] <= token) lo = mid; else hi = mid - 1;
+                    }
+                    s = lo;
+                    i = static_cast<int>(token - cu[s]);
+                    blocks_before = prefix[s];
+                }
+            } else {
+                s = static_cast<int>(token / g.N);
+                i = static_cast<int>(token - static_cast<int64_t>(s) * g.N);
+            }
+            if (inside) {
+                out = true;
+                l = lse[rowstat_index(g, s, h, g.cu_seqlens ? cu[s] : 0, i)];
+                xi = stats_index(g, stride, s, h, blocks_before, i);
+            }
+        }
         float acc = 0.f;
         if (r < rows && dq_acc) {
             float4* z = reinterpret_cast<float4*>(dq_acc + r * D + part * 8);
@@ -136,26 +168,7 @@ stats_kernel(const __nv_bfloat16* __restrict__ dO, const __nv_bfloat16* __restri
         }
 #pragma unroll
         for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (r < rows && part == 0) {
-            const int64_t token = r / g.H;
-            const int h = static_cast<int>(r - token * g.H);
-            int s, i, blocks_before = 0;
-            if (g.cu_seqlens) {
-                if (token >= cu[g.B]) continue;        // a row outside every sequence
-                int lo = 0, hi = g.B - 1;              // last s with cu[s] <= token
-                while (lo < hi) {
-                    const int mid = (lo + hi + 1) >> 1;
-                    if (cu[mid] <= token) lo = mid; else hi = mid - 1;
-                }
-                s = lo;
-                i = static_cast<int>(token - cu[s]);
-                blocks_before = prefix[s];
-            } else {
-                s = static_cast<int>(token / g.N);
-                i = static_cast<int>(token - static_cast<int64_t>(s) * g.N);
-            }
-            const float l = lse[rowstat_index(g, s, h, g.cu_seqlens ? cu[s] : 0, i)];
-            const size_t xi = stats_index(g, stride, s, h, blocks_before, i);
+        if (out) {
             stats[xi] = -l * 1.4426950408889634f;
             stats[xi + 128] = -acc;
         }
