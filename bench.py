@@ -62,14 +62,14 @@ NOMINAL_BF16_DENSE_TFLOPS = 2250.0
 # the kernel sources a capture was taken on: each entry carries a hash of their
 # comment-free text and is reported as null once that changes.
 TRAFFIC = {
-    "fwd": {"bytes_per_launch": 2 * (208.53e6 + 49.55e6), "workload": "train",
+    "fwd": {"bytes_per_launch": 2 * (208.66e6 + 52.33e6), "workload": "train",
             "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh"), "sha": "f96a3e0f94d3bdba"},
-    "dot": {"bytes_per_launch": 2 * (135.30e6 + 4.94e6), "workload": "train",
-            "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "1a04cdea55ac7705"},
-    "dkdv": {"bytes_per_launch": 2 * (275.31e6 + 109.41e6), "workload": "train",
-             "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "1a04cdea55ac7705"},
-    "dq": {"bytes_per_launch": 2 * (271.99e6 + 53.04e6), "workload": "train",
-           "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "1a04cdea55ac7705"},
+    "dot": {"bytes_per_launch": 2 * (135.29e6 + 4.49e6), "workload": "train",
+            "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "893c4b285a6b3d87"},
+    "dkdv": {"bytes_per_launch": 2 * (275.24e6 + 109.35e6), "workload": "train",
+             "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "893c4b285a6b3d87"},
+    "dq": {"bytes_per_launch": 2 * (272.24e6 + 55.72e6), "workload": "train",
+           "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "893c4b285a6b3d87"},
     "decode": {"bytes_per_launch": 792.89e6 + 4.95e6, "workload": "decode",
                "sources": ("decode_kernel.cuh", "sm100.cuh"), "sha": "34b0f87f0cc6cfec"},
     "fwd_fp8": {"bytes_per_launch": 2 * (100.99e6 + 35.70e6), "workload": "fp8",
