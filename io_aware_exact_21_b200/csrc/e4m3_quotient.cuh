@@ -81,6 +81,19 @@ __host__ __device__ __forceinline__ float e4m3_quotient(float x, float s, float 
     return e4m3q_finish(x, s, qb & 0x80000000u, e4m3q_mid(qb & 0x7FFFFFFFu));
 }
 
+// True when the rounded product q1 = RN(x * inv) alone decides the e4m3
+// value: q1 lies in the normal e4m3 range (|q1| >= 2^-6) and more than 8
+// float32 steps from the e4m3 midpoint of its interval.  x / s is within two
+// float32 steps of q1 (two roundings of relative size 2^-24 each), so it then
+// lies on the same side of every midpoint and e4m3(q1) = e4m3(x / s).
+// (Normal-range midpoints have the low 20 mantissa bits 0x80000, and never
+// sit at a binade boundary.)  A cheap test for data whose products rarely
+// fall near a midpoint, so that the exact step runs only when one does.
+__host__ __device__ __forceinline__ bool e4m3_product_decides(float q1) {
+    const uint32_t b = e4m3q_bits(q1) & 0x7FFFFFFFu;
+    return b >= 0x3C800000u && ((b & 0xFFFFFu) - 0x7FFF8u) > 16u;
+}
+
 // Four values with one scale (the quantiser's unit of work).
 __host__ __device__ __forceinline__ void e4m3_quotient4(const float (&x)[4], float s, float inv,
                                                        float (&q)[4]) {

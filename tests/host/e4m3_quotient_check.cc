@@ -7,6 +7,8 @@
 // quotient (which lies on an e4m3 midpoint only when the real one does) by
 // counting e4m3 steps; the value under test is rounded with integer bit
 // arithmetic on its float32 pattern, as the conversion instruction would.
+// The fast test e4m3_product_decides must never accept a product whose
+// rounding differs from the exact one.
 // Prints "ok".
 #include <cmath>
 #include <cstdint>
@@ -58,7 +60,8 @@ static double bits_e4m3(float q) {
 int main() {
     std::mt19937_64 rng(12345);
     std::uniform_real_distribution<float> amax_d(1e-3f, 50.f), u(-1.f, 1.f);
-    long fixups = 0, checked = 0;
+    long fixups = 0, checked = 0, decided = 0, random_checked = 0;
+    bool random_phase = true;
     auto check = [&](float x, float s) {
         const float inv = 1.f / s;
         const float q = fa::e4m3_quotient(x, s, inv);
@@ -79,6 +82,12 @@ int main() {
         }
         // cases where rounding the product x * inv alone would have been wrong
         if (bits_e4m3(x * inv) != want) ++fixups;
+        // the fast test never claims such a case
+        if (fa::e4m3_product_decides(x * inv) && bits_e4m3(x * inv) != want) {
+            std::printf("product test: x=%a s=%a\n", x, s);
+            std::exit(1);
+        }
+        if (random_phase && fa::e4m3_product_decides(x * inv)) ++decided;
     };
     auto bf16 = [](float f) {       // round to nearest bf16, ties to even
         uint32_t b;
@@ -111,6 +120,8 @@ int main() {
         const float s = amax / 448.f;
         check(u(rng) * amax, s);
     }
+    random_checked = checked;
+    random_phase = false;
     // constructed cases: x = fl(M * s) for an e4m3 midpoint M, so that the
     // float32 quotient often lands exactly on M while x / s does not
     std::uniform_int_distribution<int> mant(0, 7), expo(-9, 8);
@@ -136,6 +147,11 @@ int main() {
         }
     if (fixups == 0) {
         std::printf("no case needed more than the rounded product x * inv\n");
+        return 1;
+    }
+    // on random values the fast test should decide nearly every case
+    if (decided < random_checked * 99 / 100) {
+        std::printf("the product test decided only %ld of %ld random cases\n", decided, random_checked);
         return 1;
     }
     std::printf("ok\n");
