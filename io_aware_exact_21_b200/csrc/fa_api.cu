@@ -68,6 +68,18 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn g_encode = nullptr;
 
+// The warp-specialised kernels (forward, dK/dV, dQ, fused backward) hand
+// registers between their warpgroups with setmaxnreg; the shares add up to
+// 168 per thread over their 384 threads, which must not exceed what a kernel
+// was launched with, or the increase would wait forever.  A build whose
+// kernels came out with fewer registers is refused at set-up.
+template <typename K>
+bool regs_pool_ok(K kernel) {
+    cudaFuncAttributes a;
+    return cudaFuncGetAttributes(&a, reinterpret_cast<const void*>(kernel)) == cudaSuccess &&
+           a.numRegs >= 168;
+}
+
 template <typename K>
 cudaError_t allow_smem(K kernel, int bytes) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -122,6 +134,12 @@ int device_setup(DeviceState** out) {
             allow_smem(fa::quantize_fp8_kernel<false, false>, fa::QuantCfg::SMEM_BYTES) != cudaSuccess ||
             allow_smem(fa::quantize_fp8_kernel<false, true>, fa::QuantCfg::SMEM_BYTES) != cudaSuccess ||
             fa::bwd_set_smem_limits() != cudaSuccess || fa::fused_set_smem_limit() != cudaSuccess)
+            return FA_ERR_CUDA;
+        if (!regs_pool_ok(fa::fwd_kernel<64>) || !regs_pool_ok(fa::fwd_kernel<128>) ||
+            !regs_pool_ok(fa::fwd_kernel<128, true>) || !regs_pool_ok(fa::fwd_kernel<64, false, true>) ||
+            !regs_pool_ok(fa::fwd_kernel<128, false, true>) || !regs_pool_ok(fa::dkdv_kernel<64>) ||
+            !regs_pool_ok(fa::dkdv_kernel<128>) || !regs_pool_ok(fa::dq_kernel<64>) ||
+            !regs_pool_ok(fa::dq_kernel<128>) || !regs_pool_ok(fa::dkdvq_kernel))
             return FA_ERR_CUDA;
         st.ready = true;
     }

@@ -212,8 +212,11 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     const WaitCtl wc{abort_flag, p.error_word, p.timeout_ns};
     const int H = p.g.H;
 
+    // register split: 120 per thread for the producer / MMA warpgroup, 192 for
+    // the two softmax warpgroups: 120 * 128 + 192 * 256 = 64512, the launch's
+    // 168 * 384 (at 104 / 200 the producer and MMA code spilled)
     if (warp < 4) {
-        regs_dealloc<104>();
+        regs_dealloc<120>();
         if (warp == 0 && lane == 0) {
             // ------------------------------------------------ TMA producer --
             uint32_t cnt = 0, item_it = 0;
@@ -417,7 +420,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         __syncwarp();
     } else {
         // --------------------------------------------- softmax warpgroups --
-        regs_alloc<200>();
+        regs_alloc<192>();
         const int t = (warp >> 2) - 1;               // query tile 0 or 1
         const int wq = warp & 3;                     // TMEM lane quarter
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
