@@ -74,11 +74,11 @@ def test_quantiser_bit_exact(B, N, H, rotate):
     assert torch.count_nonzero(full[..., N:]) == 0            # padding keys are zero
 
 
-def oracle_fp8(x, signs, causal, window):
+def oracle_fp8(x, signs, causal, window, scale=1 / math.sqrt(128)):
     qc, sq = orc.quantize_fp8(x["q"], signs)
     kc, sk = orc.quantize_fp8(x["k"], signs)
     vc, sv = orc.quantize_fp8(x["v"])
-    O, L, t = orc.fwd_fp8(qc, kc, vc, sq, sk, sv, 1 / math.sqrt(128), causal, window, terms=True)
+    O, L, t = orc.fwd_fp8(qc, kc, vc, sq, sk, sv, scale, causal, window, terms=True)
     return O, L, t, sv
 
 
@@ -117,6 +117,20 @@ def test_fwd_fp8_matches_its_oracle(B, N, H, causal, window, rotate):
     torch.cuda.synchronize()
     assert fa.fa_get_device_error() == 0
     check_close(o, lse, oracle_fp8(x, signs, causal, window))
+
+
+@pytest.mark.parametrize("scale", [0.05, 0.15])
+@pytest.mark.parametrize("causal", [False, True])
+def test_fwd_fp8_scale(scale, causal):
+    """The softmax scale as an argument (the other cases run at 1/sqrt(128))."""
+    B, N, H = 2, 300, 2
+    x = fixed_inputs(B, N, H, 128, seed=760)
+    signs = fp8_signs(12)
+    qz = gpu_quantize(x, signs)
+    o, lse = fa.forward_fp8(qz, B, N, H, causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_error() == 0
+    check_close(o, lse, oracle_fp8(x, signs, causal, 0, scale))
 
 
 def test_fwd_fp8_error_against_exact_attention():
