@@ -47,7 +47,7 @@ def test_bwd_small_elementwise(B, H, N, d, causal, window):
     check((dq, dk, dv), ref)
 
 
-@pytest.mark.parametrize("lens", [[1, 127, 128, 129, 200], [5, 300, 64]])
+@pytest.mark.parametrize("lens", [[1, 127, 128, 129, 200], [5, 300, 64], [0, 129, 0, 300, 0]])
 @pytest.mark.parametrize("causal,window", [(False, 0), (True, 0), (True, 33)])
 def test_bwd_varlen_elementwise(lens, causal, window):
     x = varlen_inputs(len(lens), 0, 0, 2, 128, seed=21, with_dout=True, lengths=lens)

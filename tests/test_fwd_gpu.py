@@ -43,7 +43,8 @@ def test_fwd_small_elementwise(B, H, N, d, causal, window):
     assert_close_lse(lse, L)
 
 
-@pytest.mark.parametrize("lens", [[1, 127, 128, 129, 700], [300], [5, 1, 1000, 64, 257, 3]])
+@pytest.mark.parametrize("lens", [[1, 127, 128, 129, 700], [300], [5, 1, 1000, 64, 257, 3],
+                                  [0, 129, 0, 300, 0]])
 @pytest.mark.parametrize("causal,window", [(False, 0), (True, 0), (True, 64), (True, 1)])
 def test_fwd_varlen_elementwise(lens, causal, window):
     x = varlen_inputs(len(lens), 0, 0, 3, 128, seed=7, lengths=lens)
