@@ -123,14 +123,14 @@ __device__ __forceinline__ bool tile_needs_mask(int r0, int BM, int k0, int BN, 
 // costly units to cheap ones and the costs even out across CTAs (a greedy
 // longest-first assignment in the usual sense).
 //
-// Pairs + snake tail (every kernel, for fixed length with a causal or window
-// mask, where a block's cost is monotone in its index): when the units per
-// CTA are few, the
-// last round of units leaves up to a unit's worth of imbalance.  So only the
-// whole heads that fit in all rounds but the last go out as units; the blocks
-// of the remaining heads are sorted heaviest first (block index major, then
-// head) and dealt one by one in rounds of gridDim.x CTAs, forwards in even
-// rounds and backwards in odd ones, starting at the CTA after the last unit.
+// Pairs + snake tail (every kernel but the cached-KV forward, for fixed length
+// with a causal or window mask, where a block's cost is monotone in its
+// index): when the units per CTA are few, the last round of units leaves up
+// to a unit's worth of imbalance.  So only the whole heads that fit in all
+// rounds but the last go out as units; the blocks of the remaining heads are
+// sorted heaviest first (block index major, then head) and dealt one by one
+// in rounds of gridDim.x CTAs, forwards in even rounds and backwards in odd
+// ones, starting at the CTA after the last unit.
 // `order` is +1 when cost grows with the block index (query blocks), -1 when
 // it shrinks (key blocks), 0 for pairs alone.
 struct Schedule {
