@@ -144,12 +144,12 @@ int fa_fwd_kv(const void* q, const void* k, const void* v, void* o, float* lse,
  *           tensor-core forward kernel, split along the keys the same way.
  * k_cache, v_cache : [B, Nk, H, d] bf16; sequence b uses rows 0 .. nk_b - 1
  *           of its slice, nk_b = seqlens_k[b] (device int32 [B], clamped to
- *           [0, Nk]) or Nk when seqlens_k is NULL.  Rows past nk_b never
- *           reach a result; with Nq <= 16 they are never read and may hold
- *           anything, with Nq > 16 the rows past nk_b that share a 128-row tile
- *           with used ones are read and multiplied by zero, so they must hold
- *           finite values (a zero-initialised cache does).  k_cache and v_cache
- *           may be NULL when B * Nk = 0.
+ *           [0, Nk]) or Nk when seqlens_k is NULL.  Rows past nk_b are
+ *           never read and may hold anything, NaN included (with Nq > 16 a
+ *           key tile that would reach past nk_b is read as the 128 rows that
+ *           end at nk_b, zeros before row 0, and its rows already covered by
+ *           the tile before are masked out).  k_cache and v_cache may be NULL
+ *           when B * Nk = 0.
  * lse     : [B, H, Nq] fp32, natural log.
  * Masks   : as fa_fwd_kv with the queries at the last Nq positions of the
  *           nk_b keys: query i is at position nk_b - Nq + i.

@@ -163,6 +163,26 @@ int make_map(CUtensorMap* map, const void* ptr, int64_t rows, int H, int d, int 
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
+// Tensor map over a padded cache [B, rows, H, d] bf16 tensor, coordinates
+// (channel, head, row, sequence); boxes of 64 channels x 1 head x box_rows
+// rows x 1 sequence (the same shared-memory layout as make_map's boxes),
+// 128-byte swizzle, zero fill outside -- so a box that starts at a negative
+// row never reads the sequence before it.
+int make_map_cache(CUtensorMap* map, const void* ptr, int B, int rows, int H, int d, int box_rows) {
+    const cuuint64_t row_bytes = static_cast<cuuint64_t>(H) * static_cast<cuuint64_t>(d) * 2;
+    cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                          static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(B)};
+    cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2, row_bytes,
+                             row_bytes * static_cast<cuuint64_t>(rows)};
+    cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(box_rows), 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
 bool misaligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
 
 // FP8 operands: e4m3 codes [rows, H, 128] (3-D, boxes of 128 channels x 1 head x
@@ -461,14 +481,15 @@ int fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, void
     if (Nq > fa::kDecMaxQ) {
         // a prefill chunk: the tensor-core forward, split along the keys when ns > 1
         if (rows_q > (int64_t{1} << 31) - 1) return FA_ERR_BAD_SHAPE;
-        // with no cache rows at all the maps are pointed at q: every key is
-        // masked and nothing of q is used as a key
+        // with no cache rows at all the maps are pointed at q: every key tile is
+        // then read at rows [-128, 0), outside the map, so nothing of q is read
         const void* kk = rows_k > 0 ? k_cache : q;
         const void* vv = rows_k > 0 ? v_cache : q;
-        const int64_t map_rows_k = rows_k > 0 ? rows_k : rows_q;
+        const int map_rows_k = rows_k > 0 ? Nk : Nq;
+        if (static_cast<int64_t>(map_rows_k) * H * d * 2 >= (int64_t{1} << 40)) return FA_ERR_BAD_SHAPE;
         CUtensorMap mq, mk, mv;
-        if (make_map(&mq, q, rows_q, H, d, 128) || make_map(&mk, kk, map_rows_k, H, d, 128) ||
-            make_map(&mv, vv, map_rows_k, H, d, 128))
+        if (make_map(&mq, q, rows_q, H, d, 128) || make_map_cache(&mk, kk, B, map_rows_k, H, d, 128) ||
+            make_map_cache(&mv, vv, B, map_rows_k, H, d, 128))
             return FA_ERR_CUDA;
         fa::FwdParams p;
         p.g.B = B;

@@ -52,7 +52,12 @@
 // each item then writes O / l as fp32 and the base-2 log-sum-exp of its range
 // to the split buffers ([nsplit, rows, H, D] and [nsplit, H, rows]), which
 // combine_kernel merges.  A split with no tiles writes -inf and is skipped by
-// the merge.
+// the merge.  Cache rows past a sequence's used length are never read: K and V
+// come through 4-D maps [B, Nk, H, d] (coordinates channel, head, row,
+// sequence), and a key tile that would reach past the used length nk is read
+// right-aligned instead, as keys [nk - 128, nk) -- rows before 0 are outside
+// the map and arrive as zeros -- with the keys below the tile's own start
+// (those of the tile before it) masked out in the softmax.
 #pragma once
 
 #include "schedule.cuh"
@@ -106,6 +111,24 @@ __device__ __forceinline__ bool split_tile_range(int nsplit, int split, int& jb,
     return true;
 }
 
+// 4-D tiled load, box coordinates (c0 innermost), into this CTA's shared
+// memory (the padded cache's maps: channel, head, row, sequence).
+__device__ __forceinline__ void tma_load_4d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1, int c2, int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];"
+        ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)),
+          "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+
+// First key of cache tile j as read (128 keys): j * 128, or nk - 128 for the
+// tile that would reach past the used length nk (negative when nk < 128).
+__device__ __forceinline__ int cache_tile_key0(int j, int nk) {
+    return (j + 1) * 128 > nk ? nk - 128 : j * 128;
+}
+
 template <int D, bool kF8 = false>
 struct FwdCfg {
     static constexpr int BM = 128;              // rows per query tile
@@ -138,6 +161,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     using C = FwdCfg<D, kF8>;
     static_assert(!kF8 || D == 128, "the FP8 variant is built for d = 128");
     static_assert(!(kF8 && kCache), "no FP8 cache variant");
+    static_assert(!kCache || C::BN == 128, "cache_tile_key0 assumes 128-key tiles");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align_smem_1024(smem_raw);
     uint8_t* sQ = smem + C::OFF_Q;
@@ -268,6 +292,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                             if (kF8 && kv == 1) {
                                 // V^T tile: d rows of this (sequence, head), 128 keys
                                 tma_load_2d(dst, &tm_v, slot_full + slot, j * C::BN, (s * H + h) * D);
+                            } else if constexpr (kCache) {
+                                const CUtensorMap* tm = kv == 0 ? &tm_k : &tm_v;
+                                const int k0 = cache_tile_key0(j, kp.len);
+                                for (int b = 0; b < C::NBOX; ++b)
+                                    tma_load_4d(dst + b * C::BOX_BYTES, tm, slot_full + slot,
+                                                b * 128 / C::ESIZE, h, k0, s);
                             } else {
                                 const CUtensorMap* tm = kv == 0 ? &tm_k : &tm_v;
                                 for (int b = 0; b < C::NBOX; ++b)
@@ -499,7 +529,16 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 if (masked) {
                     // this row's allowed keys of the tile are columns [c_lo, c_hi)
                     int c_lo, c_hi;
-                    tile_key_bounds(i + off, k0, nk, p.g.causal, p.g.window, C::BN, c_lo, c_hi);
+                    if constexpr (kCache) {
+                        // the tile holds keys from k0r on; those below k0 belong to
+                        // the tile before it
+                        const int k0r = cache_tile_key0(j, nk);
+                        tile_key_bounds(i + off, k0r, nk, p.g.causal, p.g.window, C::BN, c_lo, c_hi);
+                        c_lo = max(c_lo, min(k0 - k0r, C::BN));
+                        c_hi = max(c_hi, c_lo);
+                    } else {
+                        tile_key_bounds(i + off, k0, nk, p.g.causal, p.g.window, C::BN, c_lo, c_hi);
+                    }
 #pragma unroll
                     for (int c = 0; c < C::BN; ++c) sv[c] = (c >= c_lo && c < c_hi) ? sv[c] : -INFINITY;
                 }

@@ -117,19 +117,6 @@ def test_decode_workload_parity():
 
 # ------------------------------------------- prefill chunks (Nq > 16) ---
 
-def fill_unused_rows(x, value):
-    """A finite value in the cache rows past each sequence's length (the
-    forward kernel multiplies those in a shared tile by zero)."""
-    lens = x["seqlens_k"]
-    if lens is None:
-        return x
-    k, v = x["k"].clone(), x["v"].clone()
-    for b, n in enumerate(lens.tolist()):
-        k[b, n:] = value
-        v[b, n:] = value
-    return dict(x, k=k, v=v)
-
-
 PREFILL = [(2, 17, 300, 2, 128), (1, 200, 1000, 2, 64), (2, 300, 300, 1, 128),
            (1, 257, 4096, 2, 128), (3, 129, 2000, 1, 128)]
 
@@ -141,7 +128,7 @@ def test_prefill_chunk_elementwise(B, Nq, Nk, H, d, causal, window, num_splits):
     # cache lengths drawn from [0, Nk]: includes empty caches and caches
     # shorter than the chunk (its first queries then see no key when causal)
     x = kvcache_inputs(B, Nq, Nk, H, d, seed=Nk + 7 * Nq, lens=(0, Nk))
-    o, lse = run_decode(fill_unused_rows(x, 3.0e4), causal, window, num_splits)
+    o, lse = run_decode(poison_unused_rows(x), causal, window, num_splits)
     O, L = oracle_decode(x, causal, window)
     assert_close_bf16(o, O, "O")
     assert_lse_with_empty_rows(lse, L)
@@ -175,7 +162,23 @@ def test_prefill_chunk_few_blocks_split():
     x = kvcache_inputs(1, 512, 8192, 2, 128, seed=9, lens=[8000])
     ns = fa.fa_fwd_kvcache_num_splits(1, 2, 512, 8192, 128)
     assert ns > 1
-    o, lse = run_decode(fill_unused_rows(x, 0.0), True, 0, 0)
+    o, lse = run_decode(poison_unused_rows(x), True, 0, 0)
     O, L = oracle_decode(x, True, 0)
+    assert_close_bf16(o, O, "O")
+    assert_lse_with_empty_rows(lse, L)
+
+
+@pytest.mark.parametrize("Nq", [17, 40, 200])
+@pytest.mark.parametrize("causal,window", [(False, 0), (True, 0), (True, 50)])
+@pytest.mark.parametrize("num_splits", [1, 3])
+def test_prefill_chunk_cache_ends(Nq, causal, window, num_splits):
+    # used lengths at and around multiples of the 128-key tile, and below one
+    # tile; every row past them NaN, in every sequence, so a tile that read a
+    # row past its sequence's length (its own padding or the next sequence's
+    # first rows) would put NaN into the result
+    lens = [0, 1, 17, 127, 128, 129, 255, 256, 300, 383]
+    x = kvcache_inputs(len(lens), Nq, 384, 1, 128, seed=31 + Nq, lens=lens)
+    o, lse = run_decode(poison_unused_rows(x), causal, window, num_splits)
+    O, L = oracle_decode(x, causal, window)
     assert_close_bf16(o, O, "O")
     assert_lse_with_empty_rows(lse, L)
