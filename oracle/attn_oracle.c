@@ -357,6 +357,123 @@ int oracle_bwd(const double *q, const double *k, const double *v, const double *
     return 0;
 }
 
+/*
+ * The same gradients as oracle_bwd, for listed rows only (self-attention):
+ * qrows[3*r .. 3*r+2] = (sequence, head, query row) gets dq_rows[r*d ..] =
+ * dQ_i, and krows[3*r .. 3*r+2] = (sequence, head, key row) gets
+ * dk_rows[r*d ..] = dK_j and dv_rows[r*d ..] = dV_j, with the formulas of
+ * oracle_bwd.  dQ_i needs only row i's own LSE_i and D_i.  dK_j and dV_j
+ * need LSE_i and D_i of every query row i that may attend key j; for each
+ * (sequence, head) of the key list they are computed (three-pass forward)
+ * for the query rows from the smallest listed key (causal: no earlier row
+ * sees it) to the largest listed key + W - 1 (window W; else the sequence
+ * end), which is every row that can contribute.  So a long causal sequence
+ * with keys listed near its end costs little.
+ */
+int oracle_bwd_rows(const double *q, const double *k, const double *v, const double *dout,
+                    int T, int H, int d, int nseq, const int *starts, const int *lens,
+                    double scale, int causal, int window,
+                    int nq, const int *qrows, double *dq_rows,
+                    int nk, const int *krows, double *dk_rows, double *dv_rows)
+{
+    int rc = check_args(T, H, d, nseq, starts, lens, causal, window);
+    if (rc) return rc;
+    const size_t rs = (size_t)H * d;
+    for (int r = 0; r < nq; ++r) {
+        int s = qrows[3 * r], h = qrows[3 * r + 1], i = qrows[3 * r + 2];
+        if (s < 0 || s >= nseq || h < 0 || h >= H || i < 0 || i >= lens[s]) return -3;
+    }
+    for (int r = 0; r < nk; ++r) {
+        int s = krows[3 * r], h = krows[3 * r + 1], j = krows[3 * r + 2];
+        if (s < 0 || s >= nseq || h < 0 || h >= H || j < 0 || j >= lens[s]) return -3;
+    }
+
+    /* dQ_i = scale * sum_j P_ij (dP_ij - D_i) k_j, from row i's own statistics */
+    int fail = 0;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < nq; ++r) {
+        const int s = qrows[3 * r], h = qrows[3 * r + 1], i = qrows[3 * r + 2];
+        const int start = starts[s], n = lens[s];
+        double *o_i = (double *)malloc(sizeof(double) * (size_t)d);
+        if (!o_i) { fail = 1; continue; }
+        const double lse_i = three_pass_row(q, k, v, H, d, start, n, h, i, scale, causal, window, o_i);
+        const double *qi = q + (size_t)(start + i) * rs + (size_t)h * d;
+        const double *doi = dout + (size_t)(start + i) * rs + (size_t)h * d;
+        const double D_i = dot(doi, o_i, d);
+        double *dqi = dq_rows + (size_t)r * d;
+        for (int c = 0; c < d; ++c) dqi[c] = 0.0;
+        if (lse_i != -INFINITY)
+            for (int j = 0; j < n; ++j) {
+                if (!key_allowed(i, j, causal, window)) continue;
+                const double *kj = k + (size_t)(start + j) * rs + (size_t)h * d;
+                const double *vj = v + (size_t)(start + j) * rs + (size_t)h * d;
+                const double P = exp(scale * dot(qi, kj, d) - lse_i);
+                const double dS = P * (dot(doi, vj, d) - D_i);
+                for (int c = 0; c < d; ++c) dqi[c] += scale * dS * kj[c];
+            }
+        free(o_i);
+    }
+    if (fail) return -3;
+
+    /* dV_j = sum_i P_ij dO_i ;  dK_j = scale * sum_i P_ij (dP_ij - D_i) q_i,
+       one (sequence, head) of the key list at a time */
+    char *done = (char *)calloc(nk > 0 ? (size_t)nk : 1, 1);
+    if (!done) return -3;
+    for (int r0 = 0; r0 < nk; ++r0) {
+        if (done[r0]) continue;
+        const int s = krows[3 * r0], h = krows[3 * r0 + 1];
+        const int start = starts[s], n = lens[s];
+        int jmin = n, jmax = -1;
+        for (int r = r0; r < nk; ++r)
+            if (krows[3 * r] == s && krows[3 * r + 1] == h) {
+                if (krows[3 * r + 2] < jmin) jmin = krows[3 * r + 2];
+                if (krows[3 * r + 2] > jmax) jmax = krows[3 * r + 2];
+            }
+        const int i_lo = causal ? jmin : 0;
+        const int i_hi = window > 0 ? (jmax + window < n ? jmax + window : n) : n;
+        const int m = i_hi - i_lo;
+        double *lse_h = (double *)malloc(sizeof(double) * (size_t)(m > 0 ? m : 1));
+        double *D_h = (double *)malloc(sizeof(double) * (size_t)(m > 0 ? m : 1));
+        if (!lse_h || !D_h) { free(lse_h); free(D_h); free(done); return -3; }
+        #pragma omp parallel for schedule(dynamic, 8)
+        for (int x = 0; x < m; ++x) {
+            double *o_i = (double *)malloc(sizeof(double) * (size_t)d);
+            if (!o_i) { lse_h[x] = NAN; D_h[x] = NAN; continue; }
+            const int i = i_lo + x;
+            lse_h[x] = three_pass_row(q, k, v, H, d, start, n, h, i, scale, causal, window, o_i);
+            D_h[x] = dot(dout + (size_t)(start + i) * rs + (size_t)h * d, o_i, d);
+            free(o_i);
+        }
+        #pragma omp parallel for schedule(dynamic, 1)
+        for (int r = r0; r < nk; ++r) {
+            if (krows[3 * r] != s || krows[3 * r + 1] != h) continue;
+            const int j = krows[3 * r + 2];
+            const double *kj = k + (size_t)(start + j) * rs + (size_t)h * d;
+            const double *vj = v + (size_t)(start + j) * rs + (size_t)h * d;
+            double *dkj = dk_rows + (size_t)r * d;
+            double *dvj = dv_rows + (size_t)r * d;
+            for (int c = 0; c < d; ++c) { dkj[c] = 0.0; dvj[c] = 0.0; }
+            for (int i = i_lo; i < i_hi; ++i) {
+                const double lse_i = lse_h[i - i_lo];
+                if (!key_allowed(i, j, causal, window) || lse_i == -INFINITY) continue;
+                const double *qi = q + (size_t)(start + i) * rs + (size_t)h * d;
+                const double *doi = dout + (size_t)(start + i) * rs + (size_t)h * d;
+                const double P = exp(scale * dot(qi, kj, d) - lse_i);
+                const double dS = P * (dot(doi, vj, d) - D_h[i - i_lo]);
+                for (int c = 0; c < d; ++c) {
+                    dvj[c] += P * doi[c];
+                    dkj[c] += scale * dS * qi[c];
+                }
+            }
+        }
+        for (int r = r0; r < nk; ++r)
+            if (krows[3 * r] == s && krows[3 * r + 1] == h) done[r] = 1;
+        free(lse_h); free(D_h);
+    }
+    free(done);
+    return 0;
+}
+
 /* Number of OpenMP threads the oracle runs with (1 without OpenMP). */
 int oracle_num_threads(void)
 {

@@ -68,7 +68,11 @@ def _load():
         lib.oracle_bwd.argtypes = ([dp, dp, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                     ctypes.c_int, ip, ip, ctypes.c_double, ctypes.c_int,
                                     ctypes.c_int, ctypes.c_int, ip, dp, dp, dp, dp, dp, dp])
-        for f in (lib.oracle_fwd, lib.oracle_fwd_rows, lib.oracle_fwd_online, lib.oracle_bwd):
+        lib.oracle_bwd_rows.argtypes = ([dp, dp, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_int, ip, ip, ctypes.c_double, ctypes.c_int,
+                                         ctypes.c_int, ctypes.c_int, ip, dp, ctypes.c_int, ip, dp, dp])
+        for f in (lib.oracle_fwd, lib.oracle_fwd_rows, lib.oracle_fwd_online, lib.oracle_bwd,
+                  lib.oracle_bwd_rows):
             f.restype = ctypes.c_int
         lib.oracle_num_threads.restype = ctypes.c_int
         fp = ctypes.POINTER(ctypes.c_float)
@@ -209,6 +213,26 @@ def bwd(q, k, v, dout, scale, causal=False, window=0, cu_seqlens=None, heads=Non
     res["lse"] = pk.rowstat(L)
     res["D"] = pk.rowstat(Dd)
     return res
+
+
+def bwd_rows(q, k, v, dout, scale, qrows, krows, causal=False, window=0, cu_seqlens=None):
+    """Float64 gradients for listed rows: ``qrows`` and ``krows`` are int
+    arrays [R, 3] of (sequence, head, row-within-sequence).  Returns (dQ of
+    the query rows [Rq, d], dK and dV of the key rows [Rk, d]), equal to the
+    corresponding rows of ``bwd`` (same formulas, computed from the rows'
+    own statistics, so a long sequence costs only the rows asked for)."""
+    pk = _Packed(q, cu_seqlens)
+    Q, K, V, dO = pk.tok(q), pk.tok(k), pk.tok(v), pk.tok(dout)
+    QR = np.ascontiguousarray(np.asarray(qrows, dtype=np.int32).reshape(-1, 3))
+    KR = np.ascontiguousarray(np.asarray(krows, dtype=np.int32).reshape(-1, 3))
+    dq = np.zeros((len(QR), pk.d), dtype=np.float64)
+    dk = np.zeros((len(KR), pk.d), dtype=np.float64)
+    dv = np.zeros((len(KR), pk.d), dtype=np.float64)
+    _check(_load().oracle_bwd_rows(_dp(Q), _dp(K), _dp(V), _dp(dO), pk.T, pk.H, pk.d, pk.B,
+                                   _ip(pk.starts), _ip(pk.lens), float(scale),
+                                   int(bool(causal)), int(window), len(QR), _ip(QR), _dp(dq),
+                                   len(KR), _ip(KR), _dp(dk), _dp(dv)))
+    return dq, dk, dv
 
 
 def fwd_kv(q, k, v, scale, causal=False, window=0, cu_seqlens_q=None, cu_seqlens_k=None):

@@ -60,9 +60,27 @@ def test_one_sequence_of_65536_tokens(causal):
     og, lg = gather_rows(o, lse, rows)
     assert_close_bf16(og, Or, "O rows")
     assert_close_lse(lg, Lr)
-    # backward at this length: sum_j dV_j = sum_i dO_i (each row of P sums to
-    # one) and sum_j dK_j = 0 (each row of dS sums to zero), both up to the
-    # bf16 rounding of the 65536 summed rows
+    # backward, element by element: dQ of the same sampled rows (each from its
+    # own row's statistics); with the causal mask also dK and dV of key rows
+    # in the last 1024 positions (only the queries after a key attend it, so
+    # the oracle needs the statistics of those rows alone)
+    qrows = rows
+    krows = np.zeros((0, 3), dtype=np.int32)
+    if causal:
+        rng = np.random.default_rng(7)
+        tail = {N - 1, N - 2, N - 128, N - 129, N - 256}
+        tail |= {int(j) for j in rng.integers(N - 1024, N, 16)}
+        krows = np.array([[0, 0, j] for j in sorted(tail)], dtype=np.int32)
+    dq_r, dk_r, dv_r = orc.bwd_rows(x["q"], x["k"], x["v"], x["dout"], scale, qrows, krows,
+                                    causal=causal)
+    g = {n: to64(t)[0, :, 0] for n, t in (("dq", dq), ("dk", dk), ("dv", dv))}
+    assert_close_bf16(np.stack([g["dq"][i] for _, _, i in qrows]), dq_r, "dq rows")
+    if len(krows):
+        assert_close_bf16(np.stack([g["dk"][j] for _, _, j in krows]), dk_r, "dk rows")
+        assert_close_bf16(np.stack([g["dv"][j] for _, _, j in krows]), dv_r, "dv rows")
+    # and over all rows: sum_j dV_j = sum_i dO_i (each row of P sums to one)
+    # and sum_j dK_j = 0 (each row of dS sums to zero), both up to the bf16
+    # rounding of the 65536 summed rows
     dv64, dk64 = to64(dv)[0, :, 0], to64(dk)[0, :, 0]
     do64 = x["dout"].double().numpy()[0, :, 0]
     err_v = np.abs(dv64.sum(0) - do64.sum(0)).max()

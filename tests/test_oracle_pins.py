@@ -292,6 +292,60 @@ def test_rows_and_head_subsets_match_full():
     assert np.isnan(part["dq"][0, :, 1]).all()
 
 
+@pytest.mark.parametrize("causal,window", [(False, 0), (True, 0), (True, 3), (True, 20)])
+def test_backward_rows_match_full_and_autograd(causal, window):
+    """bwd_rows (gradients of listed rows from the rows' own statistics) gives
+    bit for bit the rows of the full bwd, and matches torch float64 autograd
+    directly; key lists that start late in the sequence (where only later
+    queries are computed) included."""
+    B, N, H, d = 2, 41, 2, 8
+    q, k, v, do = (_rand((B, N, H, d), s) for s in (61, 62, 63, 64))
+    scale = 0.3
+    qrows = np.array([[0, 0, 0], [1, 1, 40], [0, 1, 17], [1, 0, 5], [1, 0, 6]])
+    krows = np.array([[0, 0, 0], [1, 1, 40], [1, 1, 30], [0, 1, 17], [1, 0, 39], [0, 0, 25]])
+    dq, dk, dv = orc.bwd_rows(q, k, v, do, scale, qrows, krows, causal=causal, window=window)
+    full = orc.bwd(q, k, v, do, scale, causal=causal, window=window)
+    for r, (s_, h, i) in enumerate(qrows):
+        np.testing.assert_array_equal(dq[r], full["dq"][s_, i, h])
+    for r, (s_, h, j) in enumerate(krows):
+        np.testing.assert_array_equal(dk[r], full["dk"][s_, j, h])
+        np.testing.assert_array_equal(dv[r], full["dv"][s_, j, h])
+    qt, kt, vt = (torch.from_numpy(x).clone().requires_grad_(True) for x in (q, k, v))
+    S = torch.einsum("bihc,bjhc->bhij", qt, kt) * scale
+    i = torch.arange(N)[:, None]
+    j = torch.arange(N)[None, :]
+    allowed = torch.ones(N, N, dtype=torch.bool)
+    if causal:
+        allowed &= j <= i
+    if window > 0:
+        allowed &= j > i - window
+    P = torch.softmax(S.masked_fill(~allowed, float("-inf")), dim=-1)
+    (torch.einsum("bhij,bjhc->bihc", P, vt) * torch.from_numpy(do)).sum().backward()
+    for r, (s_, h, i_) in enumerate(qrows):
+        np.testing.assert_allclose(dq[r], qt.grad[s_, i_, h].numpy(), rtol=0, atol=1e-12)
+    for r, (s_, h, j_) in enumerate(krows):
+        np.testing.assert_allclose(dk[r], kt.grad[s_, j_, h].numpy(), rtol=0, atol=1e-12)
+        np.testing.assert_allclose(dv[r], vt.grad[s_, j_, h].numpy(), rtol=0, atol=1e-12)
+
+
+def test_backward_rows_packed():
+    """bwd_rows on a packed batch equals the full packed bwd at those rows."""
+    lens = [5, 0, 37, 12]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T, H, d = int(cu[-1]), 2, 8
+    q, k, v, do = (_rand((T, H, d), s) for s in (65, 66, 67, 68))
+    qrows = np.array([[0, 1, 4], [2, 0, 36], [3, 1, 0], [2, 1, 3]])
+    krows = np.array([[2, 0, 36], [2, 0, 2], [0, 0, 0], [3, 1, 11]])
+    dq, dk, dv = orc.bwd_rows(q, k, v, do, 0.4, qrows, krows, causal=True, window=9,
+                              cu_seqlens=cu)
+    full = orc.bwd(q, k, v, do, 0.4, causal=True, window=9, cu_seqlens=cu)
+    for r, (s_, h, i) in enumerate(qrows):
+        np.testing.assert_array_equal(dq[r], full["dq"][cu[s_] + i, h])
+    for r, (s_, h, j) in enumerate(krows):
+        np.testing.assert_array_equal(dk[r], full["dk"][cu[s_] + j, h])
+        np.testing.assert_array_equal(dv[r], full["dv"][cu[s_] + j, h])
+
+
 def test_window_without_causal_is_rejected():
     q = _rand((1, 4, 1, 2), 46)
     with pytest.raises(ValueError):
