@@ -172,3 +172,39 @@ def test_bwd_bench_configuration_sampled_head():
             assert_close_bf16(t[s, :, h], ref[name][s, :, h], "%s[%d,:,%d]" % (name, s, h))
     for t in (dq, dk, dv):
         assert torch.isfinite(t).all()
+
+
+@pytest.mark.parametrize("name", ["prefill_b4", "prefill_b4_causal", "train_causal"])
+def test_bwd_sampled_rows_every_head(name):
+    """Full-size backward, every (sequence, head): dQ of ten rows each (tile
+    edges, the middle, the last rows and two seeded random rows) against the
+    oracle's row-wise gradients; under the causal mask also dK and dV of
+    eight key rows in the last 256 positions of four heads (the first, the
+    last, and two the backward's snake tail deals), for which the oracle
+    needs only the queries after them."""
+    wl = WORKLOADS[name]
+    x = fixed_inputs(wl.B, wl.N, wl.H, wl.d, seed=wl.seed, with_dout=True)
+    o, lse, dq, dk, dv = run(x, wl.causal, 0)
+    N = wl.N
+    rng = np.random.default_rng(wl.seed + 100)
+    qrows = []
+    for s in range(wl.B):
+        for h in range(wl.H):
+            picks = {0, 1, 127, 128, 129, N // 2, N - 2, N - 1}
+            picks |= {int(i) for i in rng.integers(0, N, 2)}
+            qrows += [(s, h, i) for i in sorted(picks)]
+    krows = []
+    if wl.causal:
+        for s, h in ((0, 0), (2, 7), (3, 12), (wl.B - 1, wl.H - 1)):
+            picks = {N - 1, N - 2, N - 128, N - 129, N - 256}
+            picks |= {int(j) for j in rng.integers(N - 256, N, 3)}
+            krows += [(s, h, j) for j in sorted(picks)]
+    qrows = np.array(qrows, dtype=np.int32)
+    krows = np.array(krows, dtype=np.int32).reshape(-1, 3)
+    dq_r, dk_r, dv_r = orc.bwd_rows(x["q"], x["k"], x["v"], x["dout"], wl.scale, qrows, krows,
+                                    causal=wl.causal)
+    g = {n: to64(t) for n, t in (("dq", dq), ("dk", dk), ("dv", dv))}
+    assert_close_bf16(np.stack([g["dq"][s, i, h] for s, h, i in qrows]), dq_r, "dq rows")
+    if len(krows):
+        assert_close_bf16(np.stack([g["dk"][s, j, h] for s, h, j in krows]), dk_r, "dk rows")
+        assert_close_bf16(np.stack([g["dv"][s, j, h] for s, h, j in krows]), dv_r, "dv rows")
