@@ -469,9 +469,9 @@ inline cudaError_t bwd_fused_launch(const BwdArgs& a, const BwdMaps& m, float* d
     {
         const int slot = hk.start(1, stream);
         const int64_t rows = static_cast<int64_t>(a.g.T) * a.g.H;
-        const int rows_per_block = 8 * (32 / (D / 8));
+        const int rows_per_block = 8 * 32;
         int64_t blocks = (rows + rows_per_block - 1) / rows_per_block;
-        const int64_t cap = static_cast<int64_t>(a.num_sms) * 8;
+        const int64_t cap = static_cast<int64_t>(a.num_sms) * kStatsCtasPerSm;
         if (blocks > cap) blocks = cap;
         if (blocks < 1) blocks = 1;
         stats_kernel<D><<<static_cast<int>(blocks), 256, a.g.cu_seqlens ? kStatsSmem : 0, stream>>>(

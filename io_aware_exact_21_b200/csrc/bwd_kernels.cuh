@@ -85,14 +85,19 @@ __device__ __forceinline__ size_t stats_index(const Geometry& g, int64_t stride,
 }
 
 // ------------------------------------------------------------ pre-pass --
-// stats[row] = {-LSE * log2(e), D = rowsum(dO * O)}: one row per group of d/8
-// lanes reading 16-byte vectors, the dot product reduced with warp shuffles.
-// Packed batches: each CTA first builds the per-sequence block prefix and a
-// copy of cu_seqlens in shared memory to place each token.
+// stats[row] = {-LSE * log2(e), D = rowsum(dO * O)}: each warp takes 32 rows
+// in the LSE array's order (so their LSE reads and statistics writes are
+// whole lines); a row's dO and O are read by a group of d/8 lanes in 16-byte
+// vectors and the dot product is reduced with warp shuffles.  Packed
+// batches: each CTA first builds the per-sequence block prefix and a copy of
+// cu_seqlens in shared memory to place each token.
 // With dq_acc non-null (the fused backward) it also zeroes that fp32 [rows, d]
 // accumulator, row by row.
+constexpr int kStatsUnroll = 4;        // load steps a warp has in flight
+constexpr int kStatsCtasPerSm = 4;     // 256-thread CTAs resident per SM (64 registers)
+
 template <int D>
-__global__ void __launch_bounds__(256, 8)
+__global__ void __launch_bounds__(256, kStatsCtasPerSm)
 stats_kernel(const __nv_bfloat16* __restrict__ dO, const __nv_bfloat16* __restrict__ O,
              const float* __restrict__ lse, float* __restrict__ stats, int64_t stride,
              Geometry g, float* __restrict__ dq_acc) {
@@ -113,64 +118,104 @@ stats_kernel(const __nv_bfloat16* __restrict__ dO, const __nv_bfloat16* __restri
     const int64_t rows = static_cast<int64_t>(g.T) * g.H;
     const int64_t warp_global = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-    for (int64_t base = warp_global * RPW; base < rows; base += nwarps * RPW) {
-        const int64_t r = base + sub;
-        // the row's place (and its LSE load) first, so that the LSE read is in
-        // flight together with the dO and O rows
+    const bool narrow = rows <= 0x7fffffff;    // row numbers fit 32-bit division
+    // Rows are walked in the LSE array's own order -- r = (s * H + h) * N + i
+    // for fixed length, h * T + token for packed batches -- 32 per warp, so
+    // the warp reads its 32 LSE values and writes its 32 statistics pairs as
+    // whole lines (consecutive rows of one (sequence, head)); each row's dO
+    // and O are read by d / 8 lanes in 16-byte vectors, RPW rows per load
+    // step, kStatsUnroll steps' loads in flight.
+    for (int64_t base = warp_global * 32; base < rows; base += nwarps * 32) {
+        // this lane's row: its place, its LSE, and its token row in dO / O
+        const int64_t r = base + lane;
         bool out = false;
         float l = 0.f;
         size_t xi = 0;
-        if (r < rows && part == 0) {
-            const int64_t token = r / g.H;
-            const int h = static_cast<int>(r - token * g.H);
-            int s = 0, i = 0, blocks_before = 0;
-            bool inside = true;
+        long long src = -1;                     // (token * H + h), or -1: no row
+        if (r < rows) {
             if (g.cu_seqlens) {
-                inside = token < cu[g.B];              // else a row outside every sequence
-                if (inside) {
+                int h, token;
+                if (narrow) {
+                    const uint32_t h32 = static_cast<uint32_t>(r) / static_cast<uint32_t>(g.T);
+                    h = static_cast<int>(h32);
+                    token = static_cast<int>(static_cast<uint32_t>(r) - h32 * static_cast<uint32_t>(g.T));
+                } else {
+                    h = static_cast<int>(r / g.T);
+                    token = static_cast<int>(r - static_cast<int64_t>(h) * g.T);
+                }
+                src = static_cast<long long>(token) * g.H + h;
+                if (token < cu[g.B]) {                 // else a row outside every sequence
                     int lo = 0, hi = g.B - 1;          // last s with cu[s] <= token
                     while (lo < hi) {
                         const int mid = (lo + hi + 1) >> 1;
                         if (cu[mid] <= token) lo = mid; else hi = mid - 1;
                     }
-                    s = lo;
-                    i = static_cast<int>(token - cu[s]);
-                    blocks_before = prefix[s];
+                    out = true;
+                    xi = stats_index(g, stride, lo, h, prefix[lo], token - cu[lo]);
                 }
             } else {
-                s = static_cast<int>(token / g.N);
-                i = static_cast<int>(token - static_cast<int64_t>(s) * g.N);
-            }
-            if (inside) {
+                int64_t sh;
+                int i;
+                if (narrow) {
+                    const uint32_t sh32 = static_cast<uint32_t>(r) / static_cast<uint32_t>(g.N);
+                    sh = sh32;
+                    i = static_cast<int>(static_cast<uint32_t>(r) - sh32 * static_cast<uint32_t>(g.N));
+                } else {
+                    sh = r / g.N;
+                    i = static_cast<int>(r - sh * g.N);
+                }
+                const int s_ = static_cast<int>(sh / g.H);
+                const int h = static_cast<int>(sh - static_cast<int64_t>(s_) * g.H);
+                src = (static_cast<long long>(s_) * g.N + i) * g.H + h;
                 out = true;
-                l = lse[rowstat_index(g, s, h, g.cu_seqlens ? cu[s] : 0, i)];
-                xi = stats_index(g, stride, s, h, blocks_before, i);
+                xi = stats_index(g, stride, s_, h, 0, i);
+            }
+            l = lse[r];
+        }
+        float dsum = 0.f;                       // D of this lane's row, once gathered
+#pragma unroll 1
+        for (int k0 = 0; k0 < 32 / RPW; k0 += kStatsUnroll) {
+            uint4 a[kStatsUnroll], b[kStatsUnroll];
+#pragma unroll
+            for (int u = 0; u < kStatsUnroll; ++u) {
+                const long long rs = __shfl_sync(0xffffffffu, src, (k0 + u) * RPW + sub);
+                a[u] = make_uint4(0u, 0u, 0u, 0u);
+                b[u] = make_uint4(0u, 0u, 0u, 0u);
+                if (rs >= 0) {
+                    a[u] = *reinterpret_cast<const uint4*>(dO + rs * D + part * 8);
+                    b[u] = *reinterpret_cast<const uint4*>(O + rs * D + part * 8);
+                    if (dq_acc) {
+                        float4* z = reinterpret_cast<float4*>(dq_acc + rs * D + part * 8);
+                        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kStatsUnroll; ++u) {
+                float acc = 0.f;
+                const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a[u]);
+                const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b[u]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 fa2 = __bfloat1622float2(pa[e]);
+                    const float2 fb2 = __bfloat1622float2(pb[e]);
+                    acc = fmaf(fa2.x, fb2.x, acc);
+                    acc = fmaf(fa2.y, fb2.y, acc);
+                }
+#pragma unroll
+                for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+                // every lane of group q now holds row (k0 + u) * RPW + q's D
+#pragma unroll
+                for (int q = 0; q < RPW; ++q) {
+                    const float t = __shfl_sync(0xffffffffu, acc, q * LPR);
+                    if (lane == (k0 + u) * RPW + q) dsum = t;
+                }
             }
         }
-        float acc = 0.f;
-        if (r < rows && dq_acc) {
-            float4* z = reinterpret_cast<float4*>(dq_acc + r * D + part * 8);
-            z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-            z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        if (r < rows) {
-            const uint4 a = *reinterpret_cast<const uint4*>(dO + r * D + part * 8);
-            const uint4 b = *reinterpret_cast<const uint4*>(O + r * D + part * 8);
-            const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
-            const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 fa2 = __bfloat1622float2(pa[e]);
-                const float2 fb2 = __bfloat1622float2(pb[e]);
-                acc = fmaf(fa2.x, fb2.x, acc);
-                acc = fmaf(fa2.y, fb2.y, acc);
-            }
-        }
-#pragma unroll
-        for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
         if (out) {
             stats[xi] = -l * 1.4426950408889634f;
-            stats[xi + 128] = -acc;
+            stats[xi + 128] = -dsum;
         }
     }
 }
@@ -1094,9 +1139,9 @@ cudaError_t bwd_launch_d(const BwdArgs& a, const BwdMaps& m, cudaStream_t stream
     {
         const int slot = hk.start(1, stream);
         const int64_t rows = static_cast<int64_t>(a.g.T) * a.g.H;
-        const int rows_per_block = 8 * (32 / (D / 8));
+        const int rows_per_block = 8 * 32;
         int64_t blocks = (rows + rows_per_block - 1) / rows_per_block;
-        const int64_t cap = static_cast<int64_t>(a.num_sms) * 8;
+        const int64_t cap = static_cast<int64_t>(a.num_sms) * kStatsCtasPerSm;
         if (blocks > cap) blocks = cap;
         if (blocks < 1) blocks = 1;
         stats_kernel<D><<<static_cast<int>(blocks), 256, a.g.cu_seqlens ? kStatsSmem : 0, stream>>>(
