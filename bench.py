@@ -64,12 +64,12 @@ NOMINAL_BF16_DENSE_TFLOPS = 2250.0
 TRAFFIC = {
     "fwd": {"bytes_per_launch": 2 * (205.31e6 + 48.29e6), "workload": "train",
             "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh"), "sha": "77c91208f87d79bb"},
-    "dot": {"bytes_per_launch": 2 * (135.29e6 + 4.49e6), "workload": "train",
-            "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "893c4b285a6b3d87"},
-    "dkdv": {"bytes_per_launch": 2 * (275.24e6 + 109.35e6), "workload": "train",
-             "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "893c4b285a6b3d87"},
-    "dq": {"bytes_per_launch": 2 * (272.24e6 + 55.72e6), "workload": "train",
-           "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "893c4b285a6b3d87"},
+    "dot": {"bytes_per_launch": 2 * (135.30e6 + 6.61e6), "workload": "train",
+            "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "cf9cd40aafda1460"},
+    "dkdv": {"bytes_per_launch": 2 * (276.34e6 + 109.81e6), "workload": "train",
+             "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "cf9cd40aafda1460"},
+    "dq": {"bytes_per_launch": 2 * (272.79e6 + 53.31e6), "workload": "train",
+           "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "cf9cd40aafda1460"},
     "decode": {"bytes_per_launch": 792.89e6 + 4.95e6, "workload": "decode",
                "sources": ("decode_kernel.cuh", "sm100.cuh"), "sha": "34b0f87f0cc6cfec"},
     "fwd_fp8": {"bytes_per_launch": 2 * (100.90e6 + 34.20e6), "workload": "fp8",
