@@ -19,7 +19,9 @@
  *       i.e. element (token t, head h, channel c) at ((t * H) + h) * d + c.
  *       Fixed length: tokens = B * N, sequence b at rows b*N .. b*N+N-1
  *       (the usual [B, N, H, d] tensor).  Packed variable length: tokens = T,
- *       sequence b at rows cu_seqlens[b] .. cu_seqlens[b+1]-1.
+ *       sequence b at rows cu_seqlens[b] .. cu_seqlens[b+1]-1; rows past
+ *       cu_seqlens[B] (a buffer larger than its batch) belong to no sequence,
+ *       may hold anything (NaN included), and reach no result.
  *   lse : fp32 natural-log log-sum-exp of the scaled scores of each row,
  *       LSE_i = ln sum_j exp(scale * q_i . k_j) over allowed keys.
  *       Fixed length: [B, H, N].  Packed: [H, T].

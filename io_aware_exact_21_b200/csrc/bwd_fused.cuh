@@ -42,6 +42,7 @@ struct FusedCfg {
     static constexpr int NSTAGE = B::NSTAGE;
     static constexpr int TILE_BYTES = B::TILE_BYTES;    // 32 KB
     static constexpr int BOX = B::BOX;
+    static constexpr int NBOX = B::NBOX;
     static constexpr int THREADS = B::THREADS;
     static constexpr uint32_t COL_ACC0 = B::COL_ACC0, COL_ACC1 = B::COL_ACC1, COL_S = B::COL_S,
                               COL_DP = B::COL_DP;
@@ -308,11 +309,29 @@ dkdvq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             const int j = k0 + row;               // this thread's key
             int ib, ie;
             query_tile_range(k0, min(n, k0 + 128), n, p.g.causal, p.g.window, 128, ib, ie);
+            // packed batches: the first row of the item's last query tile past the
+            // batch's last sequence (128: none)
+            const int dead_r0 = first_dead_row(p.g.cu_seqlens, p.g.B, sp.start + (ie - 1) * 128);
+            // and of the item's own key block, whose K tile is the dQ GEMM's B operand
+            const int dead_k0 = first_dead_row(p.g.cu_seqlens, p.g.B, sp.start + k0);
             for (int i = ib; i < ie; ++i, ++cnt) {
                 const uint32_t slot = cnt % C::NSTAGE;
                 uint8_t* stage = smem + C::OFF_ST + slot * 2 * C::TILE_BYTES;
                 if (!mbar_wait(s_full, cnt & 1, wc)) { ok = false; break; }
                 if (!mbar_wait(stage_full + slot, (cnt / C::NSTAGE) & 1, wc)) { ok = false; break; }
+                if (i == ib && dead_k0 < 128) {
+                    // K rows past the batch end meet dS = 0 in the dQ GEMM: zero them
+                    // after the item's first K Q^T (no other reader is in flight)
+                    zero_tile_rows(smem + C::OFF_FA, C::NBOX, dead_k0, ew, 256);
+                }
+                if (i + 1 == ie && dead_r0 < 128) {
+                    // Q and dO rows past the batch end meet dS = 0 and P = 0 in the
+                    // dK and dV GEMMs: zero them once both score GEMMs have read
+                    // them, before either accumulation is released
+                    if (!mbar_wait(dp_full, cnt & 1, wc)) { ok = false; break; }
+                    zero_tile_rows(stage, C::NBOX, dead_r0, ew, 256);
+                    zero_tile_rows(stage + C::TILE_BYTES, C::NBOX, dead_r0, ew, 256);
+                }
                 tc_fence_after();
                 const float* xs = vec + slot * 256 + 64 * g;   // -L log2e
                 const float* ys = xs + 128;                    // -D

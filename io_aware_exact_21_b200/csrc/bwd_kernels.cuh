@@ -35,6 +35,7 @@
 #pragma once
 
 #include "schedule.cuh"
+#include "dead_rows.cuh"
 #include "sm100.cuh"
 
 namespace fa {
@@ -238,7 +239,7 @@ struct BwdCfg {
     static constexpr int OFF_VEC = OFF_ST + NSTAGE * 2 * TILE_BYTES;  // stage stats: float2[BS]
     static constexpr int VEC_BYTES = BS * 8;
     static constexpr int OFF_BAR = OFF_VEC + NSTAGE * VEC_BYTES;
-    static constexpr int NBAR = 2 + 2 * NSTAGE + 6 + 2 + 1;
+    static constexpr int NBAR = 2 + 2 * NSTAGE + 6 + 2 + 1 + NSTAGE;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int OFF_SCRATCH = OFF_MISC + 16;
     static constexpr int OFF_PREFIX = OFF_SCRATCH + 2 * THREADS * 4;   // block and unit prefixes
@@ -267,7 +268,7 @@ __device__ __forceinline__ void query_tile_range(int k_lo, int k_hi, int n, int 
 // once per step, so its parity is the step count's.
 struct BwdBarriers {
     uint64_t *fix_full, *fix_empty, *stage_full, *stage_empty, *s_full, *dp_full, *mid, *ready,
-        *acc_final, *acc_empty, *drain;
+        *acc_final, *acc_empty, *drain, *land;
 };
 
 template <int D>
@@ -286,6 +287,7 @@ __device__ __forceinline__ BwdBarriers carve_barriers(uint8_t* smem) {
     r.acc_final = r.ready + 2;
     r.acc_empty = r.acc_final + 1;
     r.drain = r.acc_empty + 1;
+    r.land = r.drain + 1;           // [NSTAGE]: stages with rows past a packed batch
     return r;
 }
 
@@ -307,6 +309,7 @@ __device__ __forceinline__ void init_barriers(const BwdBarriers& br, volatile in
     mbar_init(br.acc_final, 1);
     mbar_init(br.acc_empty, 8);
     mbar_init(br.drain, 1);
+    for (int s = 0; s < C::NSTAGE; ++s) mbar_init(br.land + s, 1);
     *abort_flag = 0;
     fence_barrier_init();
 }
@@ -451,6 +454,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
         if (warp == 0) {
             // ---------------------------------- producer (whole warp) --
             uint32_t cnt = 0, item_it = 0, fix_issued = 0;
+            LandTrack lt;
             bool ok = true;
             ItemIter<true> it;
             int s, h, blk;
@@ -475,24 +479,31 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 const int blocks_before = sch.blocks_before(s);
+                // packed batches: the first row of the item's last query tile past
+                // the batch's last sequence (128: none); that stage lands on
+                // land[slot] for the fixer warp
+                const int dead_r0 =
+                    ie > ib ? first_dead_row(p.g.cu_seqlens, p.g.B, sp.start + (ie - 1) * C::BS) : 128;
                 for (int i = ib; i < ie && ok; ++i, ++cnt) {
                     const int slot = cnt % C::NSTAGE;
                     if (lane == 0) {
                         ok = mbar_wait(br.stage_empty + slot, ((cnt / C::NSTAGE) & 1) ^ 1, wc);
                         if (ok) {
-                            mbar_arrive_expect_tx(br.stage_full + slot, 2 * C::TILE_BYTES + C::VEC_BYTES);
+                            const bool to_land = i + 1 == ie && dead_r0 < 128;
+                            uint64_t* full = to_land ? br.land + slot : br.stage_full + slot;
+                            lt.note(slot, to_land);
+                            mbar_arrive_expect_tx(full, 2 * C::TILE_BYTES + C::VEC_BYTES);
                             uint8_t* st = smem + C::OFF_ST + slot * 2 * C::TILE_BYTES;
                             for (int b = 0; b < C::NBOX; ++b) {
-                                tma_load_3d(st + b * C::BOX, &tm_q, br.stage_full + slot, b * 64, h,
+                                tma_load_3d(st + b * C::BOX, &tm_q, full, b * 64, h, sp.start + i * C::BS);
+                                tma_load_3d(st + C::TILE_BYTES + b * C::BOX, &tm_do, full, b * 64, h,
                                             sp.start + i * C::BS);
-                                tma_load_3d(st + C::TILE_BYTES + b * C::BOX, &tm_do, br.stage_full + slot,
-                                            b * 64, h, sp.start + i * C::BS);
                             }
                             // the tile's per-query statistics, one aligned 1 KB copy
                             bulk_load(vec + slot * 2 * C::BS,
                                       p.stats + stats_index(p.g, p.stats_stride, s, h, blocks_before,
                                                             i * C::BS),
-                                      C::VEC_BYTES, br.stage_full + slot);
+                                      C::VEC_BYTES, full);
                         }
                     }
                     ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -500,9 +511,45 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                 }
             }
             if (!ok && lane == 0) {
-                for (uint32_t x = cnt > C::NSTAGE ? cnt - C::NSTAGE : 0; x < cnt; ++x)
-                    drain_wait(br.stage_full + x % C::NSTAGE, (x / C::NSTAGE) & 1, p.error_word);
+                for (uint32_t x = cnt > C::NSTAGE ? cnt - C::NSTAGE : 0; x < cnt; ++x) {
+                    const int sl = x % C::NSTAGE;
+                    if (lt.landed(sl))
+                        drain_wait(br.land + sl, lt.land_parity(sl), p.error_word);
+                    else
+                        drain_wait(br.stage_full + sl, (x / C::NSTAGE) & 1, p.error_word);
+                }
                 if (fix_issued) drain_wait(br.fix_full, (fix_issued - 1) & 1, p.error_word);
+            }
+        } else if (warp == 2) {
+            // ------------------------------------------------------- fixer --
+            // packed batches: zeroes the Q and dO rows past the batch's last
+            // sequence in each stage the producer sent to land[slot] (they meet
+            // dS = 0 and P = 0 in the dK and dV GEMMs), then releases the stage
+            // on stage_full[slot]
+            if (p.g.cu_seqlens) {
+                uint32_t cnt = 0, land_par = 0;
+                ItemIter<true> it;
+                int s, h, blk;
+                while (it.next(sch, s, h, blk)) {
+                    const SeqSpan sp = sch.span(s);
+                    const int n = sp.len;
+                    const int k0 = blk * C::BM;
+                    int ib, ie;
+                    query_tile_range(k0, min(n, k0 + C::BM), n, p.g.causal, p.g.window, C::BS, ib, ie);
+                    const int dead_r0 =
+                        ie > ib ? first_dead_row(p.g.cu_seqlens, p.g.B, sp.start + (ie - 1) * C::BS) : 128;
+                    if (dead_r0 < 128) {
+                        const int slot = (cnt + (ie - 1 - ib)) % C::NSTAGE;
+                        if (!mbar_wait(br.land + slot, (land_par >> slot) & 1u, wc)) break;
+                        land_par ^= 1u << slot;
+                        uint8_t* st = smem + C::OFF_ST + slot * 2 * C::TILE_BYTES;
+                        zero_tile_rows(st, C::NBOX, dead_r0, lane, 32);
+                        zero_tile_rows(st + C::TILE_BYTES, C::NBOX, dead_r0, lane, 32);
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(br.stage_full + slot);
+                    }
+                    cnt += ie - ib;
+                }
             }
         } else if (warp == 1 && lane == 0) {
             // ---------------------------------------------------- MMA --
@@ -731,7 +778,7 @@ struct DqCfg {
     static constexpr uint32_t COL_DQ = 0, COL_Q = 128, COL_DO = 192, COL_S = 256, COL_DP = 384;
     static constexpr int OFF_ST = 0;                                  // stages: K then V
     static constexpr int OFF_BAR = NSTAGE * 2 * TILE_BYTES;
-    static constexpr int NBAR = 2 * NSTAGE + 1 + 2 + 1 + 2 + 2 + 1;
+    static constexpr int NBAR = 2 * NSTAGE + 1 + 2 + 1 + 2 + 2 + 1 + NSTAGE;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int OFF_SCRATCH = OFF_MISC + 16;
     static constexpr int OFF_PREFIX = OFF_SCRATCH + 2 * THREADS * 4;
@@ -741,7 +788,7 @@ struct DqCfg {
 
 struct DqBarriers {
     uint64_t *stage_full, *stage_empty, *fix_ready, *s_full, *dp_full, *mid, *ready, *acc_final,
-        *acc_empty, *drain;
+        *acc_empty, *drain, *land;
 };
 
 // D[128 x 128] = A[tmem 128 x d, packed bf16] * B[smem 128 x d, K-major]^T.
@@ -774,6 +821,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
     br.acc_final = br.ready + 2;
     br.acc_empty = br.acc_final + 1;
     br.drain = br.acc_empty + 1;
+    br.land = br.drain + 1;         // [NSTAGE]: stages with rows past a packed batch
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
     int* scratch = reinterpret_cast<int*>(smem + C::OFF_SCRATCH);
@@ -795,6 +843,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
         mbar_init(br.acc_final, 1);
         mbar_init(br.acc_empty, 8);
         mbar_init(br.drain, 1);
+        for (int i = 0; i < C::NSTAGE; ++i) mbar_init(br.land + i, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -827,6 +876,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
         if (warp == 0 && lane == 0) {
             // -------------------------------------------------- producer --
             uint32_t cnt = 0;
+            LandTrack lt;
             bool ok = true;
             ItemIter<true> it;
             int s, h, blk;
@@ -836,25 +886,66 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
                 const int q0 = blk * C::BM;
                 int jb, je;
                 key_tile_range(q0, min(n, q0 + C::BM), n, p.g.causal, p.g.window, C::BS, jb, je);
+                // packed batches: the first row of the item's last key tile past the
+                // batch's last sequence (128: none); that stage lands on land[slot]
+                // for the fixer warp
+                const int dead_r0 = first_dead_row(p.g.cu_seqlens, p.g.B, sp.start + (je - 1) * C::BS);
                 for (int j = jb; j < je; ++j, ++cnt) {
                     const int slot = cnt % C::NSTAGE;
                     if (!mbar_wait(br.stage_empty + slot, ((cnt / C::NSTAGE) & 1) ^ 1, wc)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(br.stage_full + slot, 2 * C::TILE_BYTES);
+                    const bool to_land = j + 1 == je && dead_r0 < 128;
+                    uint64_t* full = to_land ? br.land + slot : br.stage_full + slot;
+                    lt.note(slot, to_land);
+                    mbar_arrive_expect_tx(full, 2 * C::TILE_BYTES);
                     uint8_t* st = smem + C::OFF_ST + slot * 2 * C::TILE_BYTES;
                     for (int b = 0; b < C::NBOX; ++b) {
-                        tma_load_3d(st + b * C::BOX, &tm_k, br.stage_full + slot, b * 64, h,
+                        tma_load_3d(st + b * C::BOX, &tm_k, full, b * 64, h, sp.start + j * C::BS);
+                        tma_load_3d(st + C::TILE_BYTES + b * C::BOX, &tm_v, full, b * 64, h,
                                     sp.start + j * C::BS);
-                        tma_load_3d(st + C::TILE_BYTES + b * C::BOX, &tm_v, br.stage_full + slot,
-                                    b * 64, h, sp.start + j * C::BS);
                     }
                 }
             }
             if (!ok) {
-                for (uint32_t x = cnt > C::NSTAGE ? cnt - C::NSTAGE : 0; x < cnt; ++x)
-                    drain_wait(br.stage_full + x % C::NSTAGE, (x / C::NSTAGE) & 1, p.error_word);
+                for (uint32_t x = cnt > C::NSTAGE ? cnt - C::NSTAGE : 0; x < cnt; ++x) {
+                    const int sl = x % C::NSTAGE;
+                    if (lt.landed(sl))
+                        drain_wait(br.land + sl, lt.land_parity(sl), p.error_word);
+                    else
+                        drain_wait(br.stage_full + sl, (x / C::NSTAGE) & 1, p.error_word);
+                }
+            }
+        } else if (warp == 2) {
+            // ------------------------------------------------------- fixer --
+            // packed batches: zeroes the K and V rows past the batch's last
+            // sequence in each stage the producer sent to land[slot] (they meet
+            // P = 0 in dP's use and dS = 0 in the dQ GEMM), then releases the
+            // stage on stage_full[slot]
+            if (p.g.cu_seqlens) {
+                uint32_t cnt = 0, land_par = 0;
+                ItemIter<true> it;
+                int s, h, blk;
+                while (it.next(sch, s, h, blk)) {
+                    const SeqSpan sp = sch.span(s);
+                    const int n = sp.len;
+                    const int q0 = blk * C::BM;
+                    int jb, je;
+                    key_tile_range(q0, min(n, q0 + C::BM), n, p.g.causal, p.g.window, C::BS, jb, je);
+                    const int dead_r0 = first_dead_row(p.g.cu_seqlens, p.g.B, sp.start + (je - 1) * C::BS);
+                    if (dead_r0 < 128) {
+                        const int slot = (cnt + (je - 1 - jb)) % C::NSTAGE;
+                        if (!mbar_wait(br.land + slot, (land_par >> slot) & 1u, wc)) break;
+                        land_par ^= 1u << slot;
+                        uint8_t* st = smem + C::OFF_ST + slot * 2 * C::TILE_BYTES;
+                        zero_tile_rows(st, C::NBOX, dead_r0, lane, 32);
+                        zero_tile_rows(st + C::TILE_BYTES, C::NBOX, dead_r0, lane, 32);
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(br.stage_full + slot);
+                    }
+                    cnt += je - jb;
+                }
             }
         } else if (warp == 1 && lane == 0) {
             // ---------------------------------------------------- MMA --

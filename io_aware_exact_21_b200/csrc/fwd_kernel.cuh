@@ -60,6 +60,7 @@
 // (those of the tile before it) masked out in the softmax.
 #pragma once
 
+#include "dead_rows.cuh"
 #include "schedule.cuh"
 #include "sm100.cuh"
 
@@ -146,7 +147,7 @@ struct FwdCfg {
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_KV = OFF_Q + 2 * TILE_BYTES;
     static constexpr int OFF_BAR = OFF_KV + NSLOT * TILE_BYTES;
-    static constexpr int NBAR = 2 + 2 * NSLOT + 8 + 1;
+    static constexpr int NBAR = 2 + 2 * NSLOT + 8 + 1 + NSLOT;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int OFF_SCRATCH = OFF_MISC + 16;
     static constexpr int OFF_PREFIX = OFF_SCRATCH + 2 * THREADS * 4;   // block and unit prefixes
@@ -175,6 +176,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     uint64_t* p_full = s_full + 2;                  // [2 tiles x 2 halves]
     uint64_t* o_final = p_full + 4;                 // [2]
     uint64_t* drain = o_final + 2;
+    uint64_t* land = drain + 1;                    // [NSLOT]: tiles with rows past the batch
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
     int* scratch = reinterpret_cast<int*>(smem + C::OFF_SCRATCH);
@@ -199,6 +201,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             mbar_init(o_final + t, 1);
         }
         mbar_init(drain, 1);
+        for (int s = 0; s < C::NSLOT; ++s) mbar_init(land + s, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -245,6 +248,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             // ------------------------------------------------ TMA producer --
             uint32_t cnt = 0, item_it = 0;
             uint32_t q_issued = 0;
+            LandTrack lt;
             bool ok = true;
             bool skipped = false;
             uint32_t skipped_at = 0xffffffffu;
@@ -269,6 +273,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                         continue;
                     }
                 }
+                // packed batches: the first row of the item's last key tile past
+                // the batch's last sequence (128: none); that tile's V lands on
+                // land[slot] for the fixer warp
+                int dead_r0 = 128;
+                if constexpr (!kF8 && !kCache)
+                    dead_r0 = first_dead_row(p.g.cu_seqlens_k, p.g.B, kp.start + (je - 1) * C::BN);
                 if (!mbar_wait(q_empty, (item_it & 1) ^ 1, wc)) { ok = false; break; }
                 mbar_arrive_expect_tx(q_full, 2 * C::TILE_BYTES);
                 for (int t = 0; t < 2; ++t)
@@ -287,22 +297,25 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                             skipped = true;   // test hook: this slot never fills
                             skipped_at = cnt;
                         } else {
-                            mbar_arrive_expect_tx(slot_full + slot, C::TILE_BYTES);
+                            const bool to_land = kv == 1 && j + 1 == je && dead_r0 < 128;
+                            uint64_t* full = to_land ? land + slot : slot_full + slot;
+                            lt.note(slot, to_land);
+                            mbar_arrive_expect_tx(full, C::TILE_BYTES);
                             uint8_t* dst = sKV + slot * C::TILE_BYTES;
                             if (kF8 && kv == 1) {
                                 // V^T tile: d rows of this (sequence, head), 128 keys
-                                tma_load_2d(dst, &tm_v, slot_full + slot, j * C::BN, (s * H + h) * D);
+                                tma_load_2d(dst, &tm_v, full, j * C::BN, (s * H + h) * D);
                             } else if constexpr (kCache) {
                                 const CUtensorMap* tm = kv == 0 ? &tm_k : &tm_v;
                                 const int k0 = cache_tile_key0(j, kp.len);
                                 for (int b = 0; b < C::NBOX; ++b)
-                                    tma_load_4d(dst + b * C::BOX_BYTES, tm, slot_full + slot,
-                                                b * 128 / C::ESIZE, h, k0, s);
+                                    tma_load_4d(dst + b * C::BOX_BYTES, tm, full, b * 128 / C::ESIZE, h,
+                                                k0, s);
                             } else {
                                 const CUtensorMap* tm = kv == 0 ? &tm_k : &tm_v;
                                 for (int b = 0; b < C::NBOX; ++b)
-                                    tma_load_3d(dst + b * C::BOX_BYTES, tm, slot_full + slot,
-                                                b * 128 / C::ESIZE, h, kp.start + j * C::BN);
+                                    tma_load_3d(dst + b * C::BOX_BYTES, tm, full, b * 128 / C::ESIZE, h,
+                                                kp.start + j * C::BN);
                             }
                         }
                         ++cnt;
@@ -315,9 +328,47 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 volatile int no_abort = 0;
                 dw.abort_flag = &no_abort;
                 // The latest phase of every slot is one of the last NSLOT loads.
-                for (uint32_t x = cnt > C::NSLOT ? cnt - C::NSLOT : 0; x < cnt; ++x)
-                    if (x != skipped_at) mbar_wait(slot_full + x % C::NSLOT, (x / C::NSLOT) & 1, dw);
+                for (uint32_t x = cnt > C::NSLOT ? cnt - C::NSLOT : 0; x < cnt; ++x) {
+                    if (x == skipped_at) continue;
+                    const int sl = x % C::NSLOT;
+                    if (lt.landed(sl))
+                        mbar_wait(land + sl, lt.land_parity(sl), dw);
+                    else
+                        mbar_wait(slot_full + sl, (x / C::NSLOT) & 1, dw);
+                }
                 if (q_issued) mbar_wait(q_full, (q_issued - 1) & 1, dw);
+            }
+        } else if (warp == 2) {
+            // ------------------------------------------------------- fixer --
+            // packed batches: zeroes the V rows past the batch's last sequence in
+            // each tile the producer sent to land[slot], then releases the tile
+            // on slot_full[slot] (walks the items and ring slots as the MMA
+            // issuer does)
+            if constexpr (!kF8 && !kCache) {
+                if (p.g.cu_seqlens_k) {
+                    uint32_t cnt = 0, land_par = 0;
+                    ItemIter<true> it;
+                    int s, h, blk;
+                    while (it.next(sch, s, h, blk)) {
+                        const SeqSpan sp = sch.span(s);
+                        const SeqSpan kp = sch.kspan(s);
+                        const int off = kp.len - sp.len;
+                        const int r_lo = blk * C::ROWS;
+                        const int r_hi = min(sp.len, r_lo + C::ROWS);
+                        int jb, je;
+                        key_tile_range(r_lo + off, r_hi + off, kp.len, p.g.causal, p.g.window, C::BN, jb, je);
+                        const int dead_r0 = first_dead_row(p.g.cu_seqlens_k, p.g.B, kp.start + (je - 1) * C::BN);
+                        if (dead_r0 < 128) {
+                            const int slot = (cnt + 2 * (je - 1 - jb) + 1) % C::NSLOT;
+                            if (!mbar_wait(land + slot, (land_par >> slot) & 1u, wc)) break;
+                            land_par ^= 1u << slot;
+                            zero_tile_rows(sKV + slot * C::TILE_BYTES, C::NBOX, dead_r0, lane, 32);
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(slot_full + slot);
+                        }
+                        cnt += 2 * (je - jb);
+                    }
+                }
             }
         } else if (warp == 1 && lane == 0) {
             // --------------------------------------------------- MMA issuer --

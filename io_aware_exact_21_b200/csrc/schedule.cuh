@@ -33,6 +33,21 @@ struct Geometry {
     const int* cu_seqlens_k;
 };
 
+// Rows of a packed batch's buffers past cu_seqlens[B] hold no sequence (a
+// buffer may be larger than the batch) and may hold anything, NaN included.
+// A 128-row tile that reaches past that end is loaded whole by TMA; where its
+// rows would meet the tensor core in a product whose other factor is a masked
+// zero (P = 0 times a V row, dS = 0 times a K, Q or dO row), 0 * NaN would
+// still be NaN, so the kernels zero those rows in shared memory first
+// (zero_tile_rows in dead_rows.cuh).  first_dead_row gives the first such
+// row of a tile that starts at global row `row0`, or 128 when it has none
+// (fixed-length batches never have any: their buffers end with the batch).
+__device__ __forceinline__ int first_dead_row(const int* cu, int B, int row0) {
+    if (!cu) return 128;
+    const int end = cu[B];
+    return row0 + 128 <= end ? 128 : max(0, end - row0);
+}
+
 struct SeqSpan {
     int start;
     int len;

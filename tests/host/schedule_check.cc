@@ -10,7 +10,8 @@
 //      block allowed;
 //   4. the column ranges the kernels mask with (tile_key_bounds for a row
 //      against a key tile, tile_query_bounds for a key against a query tile)
-//      hold exactly the pairs key_allowed allows.
+//      hold exactly the pairs key_allowed allows;
+//   5. first_dead_row finds the first tile row past a packed batch's end.
 // The CUDA built-ins the header reads (blockIdx, gridDim, threadIdx,
 // blockDim, __syncthreads) are host variables here; the packed-batch prefix
 // is built by one emulated thread.  Prints "ok" and exits 0, or names the
@@ -182,6 +183,27 @@ void check_bounds(std::mt19937& rng) {
 
 }  // namespace
 
+// first_dead_row against a row-by-row count: the first row of a 128-row tile
+// at global row row0 that lies at or past cu[B] (128 if none); no rows are
+// dead without a packed batch.
+void check_dead_rows(std::mt19937& rng) {
+    for (int trial = 0; trial < 2000; ++trial) {
+        const int B = 1 + static_cast<int>(rng() % 6);
+        std::vector<int> cu(B + 1, 0);
+        for (int s = 0; s < B; ++s) cu[s + 1] = cu[s] + static_cast<int>(rng() % 400);
+        const int row0 = static_cast<int>(rng() % (cu[B] + 1));
+        int want = 128;
+        for (int r = 0; r < 128; ++r)
+            if (row0 + r >= cu[B]) {
+                want = r;
+                break;
+            }
+        const int got = fa::first_dead_row(cu.data(), B, row0);
+        if (got != want) fail("first_dead_row", row0, cu[B], got, want);
+        if (fa::first_dead_row(nullptr, B, row0) != 128) fail("first_dead_row without cu", row0, 0, 0, 0);
+    }
+}
+
 int main() {
     std::mt19937 rng(12345);
     // fixed length: pairs, and pairs + snake tail in both cost directions
@@ -279,6 +301,7 @@ int main() {
     }
     check_masks(rng);
     check_bounds(rng);
+    check_dead_rows(rng);
     if (failures) {
         std::printf("%d violations\n", failures);
         return 1;
