@@ -62,18 +62,18 @@ NOMINAL_BF16_DENSE_TFLOPS = 2250.0
 # the kernel sources a capture was taken on: each entry carries a hash of their
 # comment-free text and is reported as null once that changes.
 TRAFFIC = {
-    "fwd": {"bytes_per_launch": 2 * (205.31e6 + 48.29e6), "workload": "train",
-            "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh"), "sha": "77c91208f87d79bb"},
-    "dot": {"bytes_per_launch": 2 * (135.30e6 + 6.61e6), "workload": "train",
-            "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "cf9cd40aafda1460"},
-    "dkdv": {"bytes_per_launch": 2 * (276.34e6 + 109.81e6), "workload": "train",
-             "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "cf9cd40aafda1460"},
-    "dq": {"bytes_per_launch": 2 * (272.79e6 + 53.31e6), "workload": "train",
-           "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh"), "sha": "cf9cd40aafda1460"},
+    "fwd": {"bytes_per_launch": 2 * (209.10e6 + 48.42e6), "workload": "train",
+            "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh", "dead_rows.cuh"), "sha": "c8393da6db9c645b"},
+    "dot": {"bytes_per_launch": 2 * (135.29e6 + 0.13e6), "workload": "train",
+            "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh", "dead_rows.cuh"), "sha": "b3c85d65544e5312"},
+    "dkdv": {"bytes_per_launch": 2 * (274.73e6 + 105.34e6), "workload": "train",
+             "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh", "dead_rows.cuh"), "sha": "b3c85d65544e5312"},
+    "dq": {"bytes_per_launch": 2 * (271.98e6 + 49.58e6), "workload": "train",
+           "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh", "dead_rows.cuh"), "sha": "b3c85d65544e5312"},
     "decode": {"bytes_per_launch": 792.89e6 + 4.95e6, "workload": "decode",
                "sources": ("decode_kernel.cuh", "sm100.cuh"), "sha": "34b0f87f0cc6cfec"},
-    "fwd_fp8": {"bytes_per_launch": 2 * (100.90e6 + 34.20e6), "workload": "fp8",
-                "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh"), "sha": "77c91208f87d79bb"},
+    "fwd_fp8": {"bytes_per_launch": 2 * (101.06e6 + 34.34e6), "workload": "fp8",
+                "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh", "dead_rows.cuh"), "sha": "c8393da6db9c645b"},
 }
 
 
