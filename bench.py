@@ -58,7 +58,8 @@ NOMINAL_BF16_DENSE_TFLOPS = 2250.0
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
 # ncu captures.  Training step and FP8 forward: the B=2 H=16 N=8192 d=128
 # non-causal case, scaled by 2 to the B=4 workload (each kernel's traffic grows
-# with the number of heads it processes).  Decode: the decode workload itself.  Valid only for
+# with the number of heads it processes).  Decode and cached-KV prefill: those
+# workloads themselves (the prefill figure is for the unsplit launch).  Valid only for
 # the kernel sources a capture was taken on: each entry carries a hash of their
 # comment-free text and is reported as null once that changes.
 TRAFFIC = {
@@ -72,6 +73,9 @@ TRAFFIC = {
            "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh", "dead_rows.cuh"), "sha": "b3c85d65544e5312"},
     "decode": {"bytes_per_launch": 792.89e6 + 4.95e6, "workload": "decode",
                "sources": ("decode_kernel.cuh", "sm100.cuh"), "sha": "34b0f87f0cc6cfec"},
+    "fwd_kv": {"bytes_per_launch": 304.79e6 + 23.17e6, "workload": "prefill_kv",
+               "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh", "dead_rows.cuh"),
+               "sha": "40a92148d57c1fbc"},
     "fwd_fp8": {"bytes_per_launch": 2 * (101.06e6 + 34.34e6), "workload": "fp8",
                 "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh", "dead_rows.cuh"), "sha": "c8393da6db9c645b"},
 }
@@ -713,7 +717,7 @@ def run_prefill_kv(args, rank, world, device):
         "roofline": {"kernel": "fwd", "bound": "tensor", "achieved": round(achieved, 2),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "peak_source": "%s bf16_tflops (burst: the kernel is timed alone)" % peak_src,
-                     "traffic": None,
+                     "traffic": traffic_for("fwd_kv", "prefill_kv") if ns == 1 else None,
                      "traffic_unit": "bytes per launch (ncu dram read + write)"},
         "e2e": {"value": round(job_throughput(f, world, e2e_steps, e2e_elapsed), 2), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,

@@ -224,9 +224,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     sch.bprefix = prefix;
     sch.uprefix = prefix + kMaxVarlenSeqs + 1;
     if constexpr (kCache) {
-        sch.g.H = p.g.H * p.nsplit;             // (head, split) pairs
-        sch.total_units = build_schedule_prefix(sch.g, C::ROWS, prefix,
-                                                prefix + kMaxVarlenSeqs + 1, scratch);
+        // (head, split) pairs; one block per unit (ItemIter's kSingles walk)
+        sch.g.H = p.g.H * p.nsplit;
+        sch.total_units = sch.g.B * sch.g.H * sch.blocks_of(sch.g.N);
     } else {
         sch.total_units = build_schedule_prefix(p.g, C::ROWS, prefix, prefix + kMaxVarlenSeqs + 1,
                                                 scratch);  // has __syncthreads
@@ -252,7 +252,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             bool ok = true;
             bool skipped = false;
             uint32_t skipped_at = 0xffffffffu;
-            ItemIter<true> it;
+            ItemIter<true, kCache> it;
             int s, h, blk;
             for (; ok && it.next(sch, s, h, blk); ++item_it) {
                 [[maybe_unused]] int split = 0;
@@ -347,7 +347,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             if constexpr (!kF8 && !kCache) {
                 if (p.g.cu_seqlens_k) {
                     uint32_t cnt = 0, land_par = 0;
-                    ItemIter<true> it;
+                    ItemIter<true, kCache> it;
                     int s, h, blk;
                     while (it.next(sch, s, h, blk)) {
                         const SeqSpan sp = sch.span(s);
@@ -417,7 +417,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     }
                 }
             };
-            ItemIter<true> it;
+            ItemIter<true, kCache> it;
             int s, h, blk;
             for (; ok && it.next(sch, s, h, blk); ++item_it) {
                 [[maybe_unused]] int split = 0;
@@ -511,7 +511,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         const float sl2 = p.scale_log2;
         uint32_t step = 0, item_it = 0;
         bool ok = true;
-        ItemIter<true> it;
+        ItemIter<true, kCache> it;
         int s, h, blk;
         for (; ok && it.next(sch, s, h, blk); ++item_it) {
             [[maybe_unused]] int split = 0;

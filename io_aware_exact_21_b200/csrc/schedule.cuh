@@ -233,13 +233,36 @@ struct Schedule {
 // Walks the blocks one CTA processes: its units in order, both blocks of each
 // (pairs), then, with kTail and a non-zero order, its blocks of the snake
 // tail round by round.  Without kTail the walk is pairs alone.
-template <bool kTail>
+//
+// kSingles (fixed length only): every block is a unit of its own, in
+// sequence-major, head, block order, dealt in rounds of gridDim.x CTAs,
+// forwards in even rounds and backwards in odd ones.  For blocks of similar
+// cost (a chunk of queries after a long cached prefix) this balances as well
+// as pairs do, and the CTAs that run at the same time then share the K/V of
+// about gridDim.x / (blocks per head) heads -- half as many as with pairs,
+// whose two blocks of a head run one after the other on one CTA -- so the
+// heads in flight fit in L2.  total_units is then B * H * blocks.
+template <bool kTail, bool kSingles = false>
 struct ItemIter {
     int w;        // pairs: next unit
     int half;
-    int round;    // snake tail: next round
+    int round;    // snake tail (and singles): next round
     __device__ __forceinline__ ItemIter() : w(blockIdx.x), half(0), round(0) {}
     __device__ __forceinline__ bool next(const Schedule& sch, int& s, int& h, int& blk) {
+        if constexpr (kSingles) {
+            const int G = gridDim.x;
+            const int x = static_cast<int>(blockIdx.x);
+            const int u = round * G + ((round & 1) ? G - 1 - x : x);
+            if (u >= sch.total_units) return false;
+            ++round;
+            const int nb = sch.blocks_of(sch.g.N);
+            const int per_seq = sch.g.H * nb;
+            s = u / per_seq;
+            const int local = u - s * per_seq;
+            h = local / nb;
+            blk = local - h * nb;
+            return true;
+        }
         const int limit = (kTail && sch.order != 0) ? sch.bulk_units : sch.total_units;
         while (w < limit) {
             int p, nb;

@@ -11,7 +11,8 @@
 //   4. the column ranges the kernels mask with (tile_key_bounds for a row
 //      against a key tile, tile_query_bounds for a key against a query tile)
 //      hold exactly the pairs key_allowed allows;
-//   5. first_dead_row finds the first tile row past a packed batch's end.
+//   5. first_dead_row finds the first tile row past a packed batch's end;
+//   6. the singles walk visits every block exactly once.
 // The CUDA built-ins the header reads (blockIdx, gridDim, threadIdx,
 // blockDim, __syncthreads) are host variables here; the packed-batch prefix
 // is built by one emulated thread.  Prints "ok" and exits 0, or names the
@@ -183,6 +184,47 @@ void check_bounds(std::mt19937& rng) {
 
 }  // namespace
 
+// The singles walk (fixed length; every block its own unit, dealt in snake
+// rounds): every (sequence, head, block) exactly once, for several grids.
+void check_singles() {
+    for (int B : {1, 3, 4})
+        for (int H : {1, 5, 16})
+            for (int N : {1, 255, 256, 257, 2048, 3000})
+                for (int G : {1, 7, 148, 1000}) {
+                    fa::Geometry g{};
+                    g.B = B;
+                    g.H = H;
+                    g.N = N;
+                    g.T = B * N;
+                    fa::Schedule sch{};
+                    sch.g = g;
+                    sch.rows_per_item = 256;
+                    const int nb = (N + 255) / 256;
+                    sch.total_units = B * H * nb;
+                    gridDim.x = G;
+                    std::map<std::tuple<int, int, int>, int> seen;
+                    for (int c = 0; c < G; ++c) {
+                        blockIdx.x = c;
+                        fa::ItemIter<true, true> it;
+                        int s, h, blk, guard = 0;
+                        while (it.next(sch, s, h, blk)) {
+                            if (++guard > 100000) {
+                                fail("singles walk does not end", c, G, N, 0);
+                                break;
+                            }
+                            if (s < 0 || s >= B || h < 0 || h >= H || blk < 0 || blk >= nb)
+                                fail("singles walk leaves the batch", s, h, blk, G);
+                            ++seen[std::make_tuple(s, h, blk)];
+                        }
+                    }
+                    if (static_cast<int>(seen.size()) != B * H * nb)
+                        fail("singles walk misses blocks", (int)seen.size(), B * H * nb, G, N);
+                    for (auto& kv : seen)
+                        if (kv.second != 1) fail("singles block visited != once", std::get<0>(kv.first),
+                                                 std::get<1>(kv.first), std::get<2>(kv.first), kv.second);
+                }
+}
+
 // first_dead_row against a row-by-row count: the first row of a 128-row tile
 // at global row row0 that lies at or past cu[B] (128 if none); no rows are
 // dead without a packed batch.
@@ -302,6 +344,7 @@ int main() {
     check_masks(rng);
     check_bounds(rng);
     check_dead_rows(rng);
+    check_singles();
     if (failures) {
         std::printf("%d violations\n", failures);
         return 1;
