@@ -253,6 +253,16 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+// The padded-cache instantiation: 4-D K/V maps (make_map_cache), one block
+// per work unit, optional split along the keys (p.nsplit).
+template <int D>
+int launch_fwd_cache(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                     const fa::FwdParams& p, int grid, cudaStream_t stream) {
+    fa::fwd_kernel<D, false, true><<<grid, fa::FwdCfg<D>::THREADS, fa::FwdCfg<D>::SMEM_BYTES,
+                                      stream>>>(mq, mk, mv, p);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 // ------------------------------------------------------ decode / split-KV --
 // Split count for a decode call: each split gets at least 4 key tiles (256
 // keys); among the counts up to that limit, the smallest whose CTAs fill the
@@ -399,6 +409,39 @@ int fa_fwd_kv(const void* q, const void* k, const void* v, void* o, float* lse, 
     DeviceState* st = nullptr;
     if ((rc = device_setup(&st)) != FA_OK) return rc;
 
+    // Fixed length with at least twice as many keys as queries (a chunk of
+    // queries after a cached prefix): the padded-cache instantiation, which
+    // deals every query block as its own work unit, so that the CTAs running
+    // at once share the K/V of few enough heads to stay in L2 (pairs of
+    // blocks on one CTA spread them over twice as many).
+    if (!packed && Nk > 0 && Nk >= 2 * static_cast<int64_t>(Nq)) {
+        CUtensorMap mq, mk, mv;
+        if (static_cast<int64_t>(Nk) * H * d * 2 >= (int64_t{1} << 40)) return FA_ERR_BAD_SHAPE;
+        if (make_map(&mq, q, c.rows, H, d, 128) || make_map_cache(&mk, k, B, Nk, H, d, 128) ||
+            make_map_cache(&mv, v, B, Nk, H, d, 128))
+            return FA_ERR_CUDA;
+        fa::FwdParams p;
+        p.g = c.g;
+        p.o = static_cast<__nv_bfloat16*>(o);
+        p.lse = lse;
+        p.scale_log2 = scale * 1.4426950408889634f;
+        p.error_word = st->error_word;
+        p.timeout_ns = g_fault_timeout_ns ? g_fault_timeout_ns : kDefaultTimeoutNs;
+        p.fault_skip_v = g_fault_mode == 1 ? 1 : 0;
+        p.nsplit = 1;
+        p.kv.seqused_k = nullptr;
+        p.kv.o_part = nullptr;
+        p.kv.lse_part = nullptr;
+        int grid = st->num_sms;
+        const int64_t items = static_cast<int64_t>(B) * H * ((Nq + 255) / 256);
+        if (items < grid) grid = static_cast<int>(items);
+        const int slot = prof_start(0, stream);
+        rc = d == 64 ? launch_fwd_cache<64>(mq, mk, mv, p, grid, stream)
+                     : launch_fwd_cache<128>(mq, mk, mv, p, grid, stream);
+        prof_stop(0, slot, stream);
+        return rc;
+    }
+
     // With no key rows at all every key tile is fully masked (each sequence
     // has nk = 0), but a tensor map cannot be empty: point the K/V maps at q,
     // whose tiles are then loaded, masked and contribute nothing.
@@ -517,15 +560,8 @@ int fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, void
         const int64_t items = static_cast<int64_t>(B) * H * ns * ((Nq + 255) / 256);
         if (items < grid) grid = static_cast<int>(items);
         const int slot = prof_start(0, stream);
-        if (d == 64) {
-            fa::fwd_kernel<64, false, true><<<grid, fa::FwdCfg<64>::THREADS, fa::FwdCfg<64>::SMEM_BYTES,
-                                              stream>>>(mq, mk, mv, p);
-            rc = cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
-        } else {
-            fa::fwd_kernel<128, false, true><<<grid, fa::FwdCfg<128>::THREADS, fa::FwdCfg<128>::SMEM_BYTES,
-                                               stream>>>(mq, mk, mv, p);
-            rc = cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
-        }
+        rc = d == 64 ? launch_fwd_cache<64>(mq, mk, mv, p, grid, stream)
+                     : launch_fwd_cache<128>(mq, mk, mv, p, grid, stream);
         prof_stop(0, slot, stream);
         if (rc != FA_OK || ns == 1) return rc;
         const int64_t warps = rows_q * H;
