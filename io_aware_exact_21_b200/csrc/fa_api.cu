@@ -130,6 +130,8 @@ int device_setup(DeviceState** out) {
             allow_smem(fa::fwd_kernel<128, true>, fa::FwdCfg<128, true>::SMEM_BYTES) != cudaSuccess ||
             allow_smem(fa::fwd_kernel<64, false, true>, fa::FwdCfg<64>::SMEM_BYTES) != cudaSuccess ||
             allow_smem(fa::fwd_kernel<128, false, true>, fa::FwdCfg<128>::SMEM_BYTES) != cudaSuccess ||
+            allow_smem(fa::fwd_kernel<64, false, false, true>, fa::FwdCfg<64>::SMEM_BYTES) != cudaSuccess ||
+            allow_smem(fa::fwd_kernel<128, false, false, true>, fa::FwdCfg<128>::SMEM_BYTES) != cudaSuccess ||
             allow_smem(fa::quantize_fp8_kernel<true, false>, fa::QuantCfg::SMEM_BYTES) != cudaSuccess ||
             allow_smem(fa::quantize_fp8_kernel<false, false>, fa::QuantCfg::SMEM_BYTES) != cudaSuccess ||
             allow_smem(fa::quantize_fp8_kernel<false, true>, fa::QuantCfg::SMEM_BYTES) != cudaSuccess ||
@@ -137,7 +139,9 @@ int device_setup(DeviceState** out) {
             return FA_ERR_CUDA;
         if (!regs_pool_ok(fa::fwd_kernel<64>) || !regs_pool_ok(fa::fwd_kernel<128>) ||
             !regs_pool_ok(fa::fwd_kernel<128, true>) || !regs_pool_ok(fa::fwd_kernel<64, false, true>) ||
-            !regs_pool_ok(fa::fwd_kernel<128, false, true>) || !regs_pool_ok(fa::dkdv_kernel<64>) ||
+            !regs_pool_ok(fa::fwd_kernel<128, false, true>) ||
+            !regs_pool_ok(fa::fwd_kernel<64, false, false, true>) ||
+            !regs_pool_ok(fa::fwd_kernel<128, false, false, true>) || !regs_pool_ok(fa::dkdv_kernel<64>) ||
             !regs_pool_ok(fa::dkdv_kernel<128>) || !regs_pool_ok(fa::dq_kernel<64>) ||
             !regs_pool_ok(fa::dq_kernel<128>) || !regs_pool_ok(fa::dkdvq_kernel))
             return FA_ERR_CUDA;
@@ -245,11 +249,11 @@ int validate_common(int B, int H, int N, int d, float scale, int causal, int win
     return FA_OK;
 }
 
-template <int D>
+template <int D, bool kSingles = false>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                const fa::FwdParams& p, int grid, cudaStream_t stream) {
-    fa::fwd_kernel<D><<<grid, fa::FwdCfg<D>::THREADS, fa::FwdCfg<D>::SMEM_BYTES, stream>>>(
-        mq, mk, mv, p);
+    fa::fwd_kernel<D, false, false, kSingles><<<grid, fa::FwdCfg<D>::THREADS, fa::FwdCfg<D>::SMEM_BYTES,
+                                                 stream>>>(mq, mk, mv, p);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -467,9 +471,17 @@ int fa_fwd_kv(const void* q, const void* k, const void* v, void* o, float* lse, 
         const int64_t items = static_cast<int64_t>(B) * H * ((Nq + 255) / 256);
         if (items < grid) grid = static_cast<int>(items);
     }
+    // packed batches holding at least twice as many key rows as query rows
+    // (chunks after cached prefixes): one block per work unit, as for the
+    // fixed-length case above
+    const bool singles = packed && Nk >= 2 * static_cast<int64_t>(Nq);
     const int slot = prof_start(0, stream);
-    rc = d == 64 ? launch_fwd<64>(mq, mk, mv, p, grid, stream)
-                 : launch_fwd<128>(mq, mk, mv, p, grid, stream);
+    if (singles)
+        rc = d == 64 ? launch_fwd<64, true>(mq, mk, mv, p, grid, stream)
+                     : launch_fwd<128, true>(mq, mk, mv, p, grid, stream);
+    else
+        rc = d == 64 ? launch_fwd<64>(mq, mk, mv, p, grid, stream)
+                     : launch_fwd<128>(mq, mk, mv, p, grid, stream);
     prof_stop(0, slot, stream);
     return rc;
 }

@@ -58,6 +58,12 @@
 // right-aligned instead, as keys [nk - 128, nk) -- rows before 0 are outside
 // the map and arrive as zeros -- with the keys below the tile's own start
 // (those of the tile before it) masked out in the softmax.
+//
+// kSingles = true (always with kCache; also instantiated for packed cached-KV
+// prefill) walks every 256-row block as its own work unit instead of pairs of
+// blocks of one head (ItemIter's kSingles walk): where each head's keys far
+// outnumber its queries, pairs keep twice as many heads' K/V in flight as
+// singles do, more than L2 holds.
 #pragma once
 
 #include "dead_rows.cuh"
@@ -155,7 +161,7 @@ struct FwdCfg {
     static constexpr int SMEM_BYTES = OFF_PREFIX + 2 * (kMaxVarlenSeqs + 1) * 4 + kMaxSortedSeqs * 2 + 1024;
 };
 
-template <int D, bool kF8 = false, bool kCache = false>
+template <int D, bool kF8 = false, bool kCache = false, bool kSingles = kCache>
 __global__ void __launch_bounds__(FwdCfg<D, kF8>::THREADS, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
            const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -163,6 +169,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     static_assert(!kF8 || D == 128, "the FP8 variant is built for d = 128");
     static_assert(!(kF8 && kCache), "no FP8 cache variant");
     static_assert(!kCache || C::BN == 128, "cache_tile_key0 assumes 128-key tiles");
+    static_assert(!kCache || kSingles, "the cache variant walks single blocks");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align_smem_1024(smem_raw);
     uint8_t* sQ = smem + C::OFF_Q;
@@ -229,7 +236,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         sch.total_units = sch.g.B * sch.g.H * sch.blocks_of(sch.g.N);
     } else {
         sch.total_units = build_schedule_prefix(p.g, C::ROWS, prefix, prefix + kMaxVarlenSeqs + 1,
-                                                scratch);  // has __syncthreads
+                                                scratch, true, kSingles);  // has __syncthreads
     }
     schedule_split_tail(sch);
     tc_fence_before();
@@ -252,7 +259,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             bool ok = true;
             bool skipped = false;
             uint32_t skipped_at = 0xffffffffu;
-            ItemIter<true, kCache> it;
+            ItemIter<true, kSingles, !kCache> it;
             int s, h, blk;
             for (; ok && it.next(sch, s, h, blk); ++item_it) {
                 [[maybe_unused]] int split = 0;
@@ -347,7 +354,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             if constexpr (!kF8 && !kCache) {
                 if (p.g.cu_seqlens_k) {
                     uint32_t cnt = 0, land_par = 0;
-                    ItemIter<true, kCache> it;
+                    ItemIter<true, kSingles, !kCache> it;
                     int s, h, blk;
                     while (it.next(sch, s, h, blk)) {
                         const SeqSpan sp = sch.span(s);
@@ -417,7 +424,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     }
                 }
             };
-            ItemIter<true, kCache> it;
+            ItemIter<true, kSingles, !kCache> it;
             int s, h, blk;
             for (; ok && it.next(sch, s, h, blk); ++item_it) {
                 [[maybe_unused]] int split = 0;
@@ -511,7 +518,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         const float sl2 = p.scale_log2;
         uint32_t step = 0, item_it = 0;
         bool ok = true;
-        ItemIter<true, kCache> it;
+        ItemIter<true, kSingles, !kCache> it;
         int s, h, blk;
         for (; ok && it.next(sch, s, h, blk); ++item_it) {
             [[maybe_unused]] int split = 0;

@@ -234,15 +234,17 @@ struct Schedule {
 // (pairs), then, with kTail and a non-zero order, its blocks of the snake
 // tail round by round.  Without kTail the walk is pairs alone.
 //
-// kSingles (fixed length only): every block is a unit of its own, in
-// sequence-major, head, block order, dealt in rounds of gridDim.x CTAs,
-// forwards in even rounds and backwards in odd ones.  For blocks of similar
+// kSingles: every block is a unit of its own, in sequence-major (packed:
+// rank-major, longest first), head, block order, dealt in rounds of
+// gridDim.x CTAs, forwards in even rounds and backwards in odd ones.  For blocks of similar
 // cost (a chunk of queries after a long cached prefix) this balances as well
 // as pairs do, and the CTAs that run at the same time then share the K/V of
 // about gridDim.x / (blocks per head) heads -- half as many as with pairs,
 // whose two blocks of a head run one after the other on one CTA -- so the
-// heads in flight fit in L2.  total_units is then B * H * blocks.
-template <bool kTail, bool kSingles = false>
+// heads in flight fit in L2.  total_units is then the number of blocks times
+// H (build_schedule_prefix with singles = true).  kMayPack = false leaves
+// out the packed decoding for callers that are fixed-length by construction.
+template <bool kTail, bool kSingles = false, bool kMayPack = true>
 struct ItemIter {
     int w;        // pairs: next unit
     int half;
@@ -255,6 +257,21 @@ struct ItemIter {
             const int u = round * G + ((round & 1) ? G - 1 - x : x);
             if (u >= sch.total_units) return false;
             ++round;
+            if (kMayPack && sch.g.cu_seqlens) {
+                // packed (build_schedule_prefix with singles): the unit prefix
+                // counts blocks, in rank order
+                int lo = 0, hi = sch.g.B - 1;
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (sch.uprefix[mid] * sch.g.H <= u) lo = mid; else hi = mid - 1;
+                }
+                s = sch.ranked() ? sch.ranked_seqs()[lo] : lo;
+                const int nb = sch.uprefix[lo + 1] - sch.uprefix[lo];
+                const int local = u - sch.uprefix[lo] * sch.g.H;
+                h = local / nb;
+                blk = local - h * nb;
+                return true;
+            }
             const int nb = sch.blocks_of(sch.g.N);
             const int per_seq = sch.g.H * nb;
             s = u / per_seq;
@@ -340,10 +357,10 @@ __device__ __forceinline__ int schedule_order(const Geometry& g, int cost_grows_
 __device__ __forceinline__ int build_schedule_prefix(const Geometry& g, int rows_per_item,
                                                      int* bprefix, int* uprefix,
                                                      int* scratch /* 2 * blockDim */,
-                                                     bool with_rank = true) {
+                                                     bool with_rank = true, bool singles = false) {
     if (!g.cu_seqlens) {
         const int nb = (g.N + rows_per_item - 1) / rows_per_item;
-        return g.B * g.H * ((nb + 1) >> 1);
+        return g.B * g.H * (singles ? nb : ((nb + 1) >> 1));
     }
     const bool sort = with_rank && g.B <= kMaxSortedSeqs;
     short* rank_seq = reinterpret_cast<short*>(uprefix + kMaxVarlenSeqs + 1);
@@ -364,7 +381,7 @@ __device__ __forceinline__ int build_schedule_prefix(const Geometry& g, int rows
             }
             rank_seq[r] = static_cast<short>(s);
         }
-        uprefix[r + 1] = (nb + 1) >> 1;
+        uprefix[r + 1] = singles ? nb : (nb + 1) >> 1;
     }
     __syncthreads();
     // inclusive prefix sums over [1, B]: per-thread chunks, then chunk offsets

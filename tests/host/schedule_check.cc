@@ -225,6 +225,63 @@ void check_singles() {
                 }
 }
 
+// The singles walk over packed batches (unit prefix in blocks, ranked
+// longest first up to kMaxSortedSeqs sequences, in index order above):
+// every (sequence, head, block) exactly once.
+void check_singles_packed(std::mt19937& rng) {
+    for (int trial = 0; trial < 40; ++trial) {
+        const int B = trial < 30 ? 1 + static_cast<int>(rng() % 20) : 250 + static_cast<int>(rng() % 20);
+        const int H = 1 + static_cast<int>(rng() % 4);
+        std::vector<int> lens(B), cu(B + 1, 0);
+        for (int s = 0; s < B; ++s) {
+            lens[s] = (rng() % 5 == 0) ? 0 : static_cast<int>(rng() % 1500);
+            cu[s + 1] = cu[s] + lens[s];
+        }
+        fa::Geometry g{};
+        g.B = B;
+        g.H = H;
+        g.N = 0;
+        g.T = cu[B];
+        g.cu_seqlens = cu.data();
+        std::vector<int> bpre(fa::kMaxVarlenSeqs + 1), upre(fa::kMaxVarlenSeqs + 1 + fa::kMaxSortedSeqs);
+        std::vector<int> scratch(2);
+        blockDim.x = 1;
+        threadIdx.x = 0;
+        fa::Schedule sch{};
+        sch.g = g;
+        sch.rows_per_item = 256;
+        sch.bprefix = bpre.data();
+        sch.uprefix = upre.data();
+        sch.total_units = fa::build_schedule_prefix(g, 256, bpre.data(), upre.data(), scratch.data(), true, true);
+        for (int G : {1, 13, 148}) {
+            gridDim.x = G;
+            std::map<std::tuple<int, int, int>, int> seen;
+            for (int c = 0; c < G; ++c) {
+                blockIdx.x = c;
+                fa::ItemIter<true, true> it;
+                int s, h, blk, guard = 0;
+                while (it.next(sch, s, h, blk)) {
+                    if (++guard > 1000000) {
+                        fail("packed singles walk does not end", c, G, B, 0);
+                        break;
+                    }
+                    ++seen[std::make_tuple(s, h, blk)];
+                }
+            }
+            size_t expected = 0;
+            for (int s = 0; s < B; ++s)
+                for (int h = 0; h < H; ++h)
+                    for (int b = 0; b < (lens[s] + 255) / 256; ++b) {
+                        ++expected;
+                        auto f = seen.find(std::make_tuple(s, h, b));
+                        if (f == seen.end() || f->second != 1)
+                            fail("packed singles block visited != once", s, h, b, f == seen.end() ? 0 : f->second);
+                    }
+            if (seen.size() != expected) fail("packed singles walk leaves the batch", (int)seen.size(), (int)expected, G, B);
+        }
+    }
+}
+
 // first_dead_row against a row-by-row count: the first row of a 128-row tile
 // at global row row0 that lies at or past cu[B] (128 if none); no rows are
 // dead without a packed batch.
@@ -345,6 +402,7 @@ int main() {
     check_bounds(rng);
     check_dead_rows(rng);
     check_singles();
+    check_singles_packed(rng);
     if (failures) {
         std::printf("%d violations\n", failures);
         return 1;

@@ -87,6 +87,20 @@ def test_fwd_kv_packed_elementwise(pairs, causal, window):
     assert_lse_with_empty_rows(lse, L)
 
 
+@pytest.mark.parametrize("causal,window", [(False, 0), (True, 0), (True, 50)])
+def test_fwd_kv_packed_many_sequences_long_caches(causal, window):
+    # 300 sequences (more than are ranked by length), keys at least twice the
+    # queries in total, so the single-block walk runs in index order
+    rng = np.random.default_rng(17)
+    nq = [int(x) for x in rng.integers(0, 40, 300)]
+    nk = [int(x) + 2 * q for x, q in zip(rng.integers(0, 300, 300), nq)]
+    x = varlen_kv_inputs(nq, nk, 1, 64, seed=18)
+    o, lse = run_kv(x, causal, window)
+    O, L = oracle_kv(x, causal, window, 1 / math.sqrt(64))
+    assert_close_bf16(o, O, "O")
+    assert_lse_with_empty_rows(lse, L)
+
+
 @pytest.mark.parametrize("Nq", [1, 200, 1000])
 @pytest.mark.parametrize("window", [0, 100])
 def test_fwd_kv_is_suffix_of_self_attention(Nq, window):
