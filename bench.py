@@ -650,7 +650,6 @@ def run_prefill_kv(args, rank, world, device):
     clocks.start()
     barrier()
     torch.cuda.synchronize(device)
-    fa.fa_profile_begin()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
@@ -660,8 +659,15 @@ def run_prefill_kv(args, rank, world, device):
     torch.cuda.synchronize(device)
     barrier()
     elapsed = e0.elapsed_time(e1)
-    prof = fa.fa_profile_end()
     clk = clocks.stop()
+    # per-kernel times: the same steps once more with an event pair around
+    # every launch, kept out of the timed region above (on a call of a tenth
+    # of a millisecond the extra events would show in its time)
+    fa.fa_profile_begin()
+    for _ in range(args.steps):
+        step(q, k, v, o, lse)
+    torch.cuda.synchronize(device)
+    prof = fa.fa_profile_end()
     assert fa.fa_get_device_error() == 0
 
     # end to end: each step copies Q, K, V in from pinned host memory and O,
@@ -789,7 +795,6 @@ def run_decode(args, rank, world, device):
     clocks.start()
     barrier()
     torch.cuda.synchronize(device)
-    fa.fa_profile_begin()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
@@ -799,8 +804,15 @@ def run_decode(args, rank, world, device):
     torch.cuda.synchronize(device)
     barrier()
     elapsed = e0.elapsed_time(e1)
-    prof = fa.fa_profile_end()
     clk = clocks.stop()
+    # per-kernel times: the same steps once more with an event pair around
+    # every launch, kept out of the timed region above (on a call of a tenth
+    # of a millisecond the extra events would show in its time)
+    fa.fa_profile_begin()
+    for _ in range(args.steps):
+        step(q, lens, o, lse)
+    torch.cuda.synchronize(device)
+    prof = fa.fa_profile_end()
     assert fa.fa_get_device_error() == 0
 
     # end to end: per step the new query and the cache lengths come from pinned
@@ -940,7 +952,6 @@ def run_fp8(args, rank, world, device):
     clocks.start()
     barrier()
     torch.cuda.synchronize(device)
-    fa.fa_profile_begin()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
@@ -950,8 +961,15 @@ def run_fp8(args, rank, world, device):
     torch.cuda.synchronize(device)
     barrier()
     elapsed = e0.elapsed_time(e1)
-    prof = fa.fa_profile_end()
     clk = clocks.stop()
+    # per-kernel times: the same steps once more with an event pair around
+    # every launch, kept out of the timed region above (on a call of a tenth
+    # of a millisecond the extra events would show in its time)
+    fa.fa_profile_begin()
+    for _ in range(args.steps):
+        step(q, k, v, o, lse)
+    torch.cuda.synchronize(device)
+    prof = fa.fa_profile_end()
     assert fa.fa_get_device_error() == 0
 
     pin = {n: host[n].pin_memory() for n in ("q", "k", "v")}
