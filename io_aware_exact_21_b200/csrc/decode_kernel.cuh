@@ -126,6 +126,9 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 2)
 decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
               const DecodeParams p) {
     using C = DecCfg<D>;
+    // the merge launched after this grid (programmatic dependent launch) may
+    // be scheduled now; it waits for this grid's completion before reading
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align_smem_1024(smem_raw);
     float* sq = reinterpret_cast<float*>(smem + C::OFF_Q);
@@ -439,6 +442,9 @@ __global__ void __launch_bounds__(256)
 combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
                __nv_bfloat16* __restrict__ o, float* __restrict__ lse, int rows, int H, int Nq,
                int nsplit) {
+    // launched as a programmatic dependent of the split kernel: wait until it
+    // has completed and its partials are visible (returns at once otherwise)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = lane_id();
     if (warp_global >= rows * H) return;

@@ -340,10 +340,22 @@ int launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const fa::Decode
         const int64_t warps = static_cast<int64_t>(p.B) * p.Nq * p.H;
         const int blocks = static_cast<int>((warps + 7) / 8);
         const int slot2 = prof_start(5, stream);
-        fa::combine_kernel<D><<<blocks, 256, 0, stream>>>(p.o_part, p.lse_part, p.o, p.lse,
-                                                           p.B * p.Nq, p.H, p.Nq, p.nsplit);
+        // programmatic dependent launch: the merge's CTAs are scheduled while
+        // the split kernel's last wave runs and wait on the device for it
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(blocks);
+        cfg.blockDim = dim3(256);
+        cfg.dynamicSmemBytes = 0;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, fa::combine_kernel<D>, p.o_part, p.lse_part, p.o,
+                                                 p.lse, p.B * p.Nq, p.H, p.Nq, p.nsplit);
         prof_stop(5, slot2, stream);
-        if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+        if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
     }
     return FA_OK;
 }
