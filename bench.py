@@ -71,8 +71,8 @@ TRAFFIC = {
              "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh", "dead_rows.cuh"), "sha": "84e074c227182110"},
     "dq": {"bytes_per_launch": 2 * (271.92e6 + 49.39e6), "workload": "train",
            "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh", "dead_rows.cuh"), "sha": "84e074c227182110"},
-    "decode": {"bytes_per_launch": 792.89e6 + 4.95e6, "workload": "decode",
-               "sources": ("decode_kernel.cuh", "sm100.cuh"), "sha": "34b0f87f0cc6cfec"},
+    "decode": {"bytes_per_launch": 792.83e6 + 4.23e6, "workload": "decode",
+               "sources": ("decode_kernel.cuh", "sm100.cuh"), "sha": "5d5936e38ab0d8c6"},
     "fwd_kv": {"bytes_per_launch": 305.31e6 + 23.29e6, "workload": "prefill_kv",
                "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh", "dead_rows.cuh"),
                "sha": "d349d740a3d5dd8b"},
