@@ -74,10 +74,28 @@ def test_nan_rows_past_the_batch(lens, causal, window, mode):
         assert_close_bf16(t, r[name], name)
 
 
+@pytest.mark.parametrize("lens,causal,window", [([100, 300, 77], True, 0), ([129, 5], False, 0),
+                                                ([1000, 64], True, 33)])
+@pytest.mark.parametrize("mode", ["two_kernel", "noalloc"])
+def test_nan_rows_past_the_batch_d64(lens, causal, window, mode):
+    x = varlen_inputs(len(lens), 0, 0, 3, 64, seed=7 + sum(lens), with_dout=True, lengths=lens)
+    got = run_self(x, causal, window, mode, float("nan"))
+    ref = run_self(x, causal, window, mode, 0.0)
+    for name, a, b in zip(("o", "lse", "dq", "dk", "dv"), got, ref):
+        assert torch.equal(a, b), "%s differs with NaN padding" % name
+    cu = x["cu_seqlens"]
+    r = orc.bwd(x["q"], x["k"], x["v"], x["dout"], 1 / math.sqrt(64), causal=causal,
+                window=window, cu_seqlens=cu)
+    assert_close_bf16(got[0], r["o"], "O")
+    for name, t in zip(("dq", "dk", "dv"), got[2:]):
+        assert_close_bf16(t, r[name], name)
+
+
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("lq,lk,causal", [([50, 200], [300, 700], True), ([17, 129], [129, 255], False),
                                           ([40], [1000], True)])
-def test_nan_rows_past_the_batch_cached_kv(lq, lk, causal):
-    x = varlen_kv_inputs(lq, lk, 2, 128, seed=3 + sum(lk))
+def test_nan_rows_past_the_batch_cached_kv(lq, lk, causal, d):
+    x = varlen_kv_inputs(lq, lk, 2, d, seed=3 + sum(lk))
     Tq = int(x["cu_seqlens_q"][-1])
     outs = []
     for value in (float("nan"), 0.0):
@@ -89,7 +107,7 @@ def test_nan_rows_past_the_batch_cached_kv(lq, lk, causal):
         assert fa.fa_get_device_error() == 0
         outs.append((o[:Tq].clone(), lse[:, :Tq].clone()))
     assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
-    O, L = orc.fwd_kv(x["q"], x["k"], x["v"], 1 / math.sqrt(128), causal=causal,
+    O, L = orc.fwd_kv(x["q"], x["k"], x["v"], 1 / math.sqrt(d), causal=causal,
                       cu_seqlens_q=x["cu_seqlens_q"], cu_seqlens_k=x["cu_seqlens_k"])
     assert_close_bf16(outs[0][0], O, "O")
     g = to64(outs[0][1])
