@@ -63,21 +63,21 @@ NOMINAL_BF16_DENSE_TFLOPS = 2250.0
 # the kernel sources a capture was taken on: each entry carries a hash of their
 # comment-free text and is reported as null once that changes.
 TRAFFIC = {
-    "fwd": {"bytes_per_launch": 2 * (207.67e6 + 49.21e6), "workload": "train",
-            "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh", "dead_rows.cuh"), "sha": "d349d740a3d5dd8b"},
-    "dot": {"bytes_per_launch": 2 * (135.30e6 + 0.13e6), "workload": "train",
-            "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh", "dead_rows.cuh"), "sha": "84e074c227182110"},
-    "dkdv": {"bytes_per_launch": 2 * (274.90e6 + 104.28e6), "workload": "train",
-             "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh", "dead_rows.cuh"), "sha": "84e074c227182110"},
-    "dq": {"bytes_per_launch": 2 * (271.92e6 + 49.39e6), "workload": "train",
-           "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh", "dead_rows.cuh"), "sha": "84e074c227182110"},
+    "fwd": {"bytes_per_launch": 2 * (208.09e6 + 48.65e6), "workload": "train",
+            "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh", "dead_rows.cuh"), "sha": "088330ef957fa172"},
+    "dot": {"bytes_per_launch": 2 * (135.29e6 + 0.06e6), "workload": "train",
+            "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh", "dead_rows.cuh"), "sha": "3ba12ef752ee6178"},
+    "dkdv": {"bytes_per_launch": 2 * (274.15e6 + 104.73e6), "workload": "train",
+             "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh", "dead_rows.cuh"), "sha": "3ba12ef752ee6178"},
+    "dq": {"bytes_per_launch": 2 * (271.66e6 + 49.75e6), "workload": "train",
+           "sources": ("bwd_kernels.cuh", "schedule.cuh", "sm100.cuh", "dead_rows.cuh"), "sha": "3ba12ef752ee6178"},
     "decode": {"bytes_per_launch": 792.83e6 + 4.23e6, "workload": "decode",
                "sources": ("decode_kernel.cuh", "sm100.cuh"), "sha": "5d5936e38ab0d8c6"},
-    "fwd_kv": {"bytes_per_launch": 305.31e6 + 23.29e6, "workload": "prefill_kv",
+    "fwd_kv": {"bytes_per_launch": 305.29e6 + 23.11e6, "workload": "prefill_kv",
                "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh", "dead_rows.cuh"),
-               "sha": "d349d740a3d5dd8b"},
-    "fwd_fp8": {"bytes_per_launch": 2 * (100.99e6 + 34.74e6), "workload": "fp8",
-                "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh", "dead_rows.cuh"), "sha": "d349d740a3d5dd8b"},
+               "sha": "088330ef957fa172"},
+    "fwd_fp8": {"bytes_per_launch": 2 * (100.94e6 + 34.15e6), "workload": "fp8",
+                "sources": ("fwd_kernel.cuh", "schedule.cuh", "sm100.cuh", "dead_rows.cuh"), "sha": "088330ef957fa172"},
 }
 
 

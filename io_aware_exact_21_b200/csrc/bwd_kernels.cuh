@@ -540,7 +540,8 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                         ie > ib ? first_dead_row(p.g.cu_seqlens, p.g.B, sp.start + (ie - 1) * C::BS) : 128;
                     if (dead_r0 < 128) {
                         const int slot = (cnt + (ie - 1 - ib)) % C::NSTAGE;
-                        if (!mbar_wait(br.land + slot, (land_par >> slot) & 1u, wc)) break;
+                        // every lane waits; the warp leaves together if any lane gave up
+                        if (!__all_sync(0xffffffffu, mbar_wait(br.land + slot, (land_par >> slot) & 1u, wc))) break;
                         land_par ^= 1u << slot;
                         uint8_t* st = smem + C::OFF_ST + slot * 2 * C::TILE_BYTES;
                         zero_tile_rows(st, C::NBOX, dead_r0, lane, 32);
@@ -936,7 +937,8 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
                     const int dead_r0 = first_dead_row(p.g.cu_seqlens, p.g.B, sp.start + (je - 1) * C::BS);
                     if (dead_r0 < 128) {
                         const int slot = (cnt + (je - 1 - jb)) % C::NSTAGE;
-                        if (!mbar_wait(br.land + slot, (land_par >> slot) & 1u, wc)) break;
+                        // every lane waits; the warp leaves together if any lane gave up
+                        if (!__all_sync(0xffffffffu, mbar_wait(br.land + slot, (land_par >> slot) & 1u, wc))) break;
                         land_par ^= 1u << slot;
                         uint8_t* st = smem + C::OFF_ST + slot * 2 * C::TILE_BYTES;
                         zero_tile_rows(st, C::NBOX, dead_r0, lane, 32);

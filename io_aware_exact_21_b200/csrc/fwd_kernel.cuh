@@ -367,7 +367,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                         const int dead_r0 = first_dead_row(p.g.cu_seqlens_k, p.g.B, kp.start + (je - 1) * C::BN);
                         if (dead_r0 < 128) {
                             const int slot = (cnt + 2 * (je - 1 - jb) + 1) % C::NSLOT;
-                            if (!mbar_wait(land + slot, (land_par >> slot) & 1u, wc)) break;
+                            // every lane waits; the warp leaves together if any lane gave up
+                            if (!__all_sync(0xffffffffu, mbar_wait(land + slot, (land_par >> slot) & 1u, wc))) break;
                             land_par ^= 1u << slot;
                             zero_tile_rows(sKV + slot * C::TILE_BYTES, C::NBOX, dead_r0, lane, 32);
                             __syncwarp();
